@@ -1,0 +1,361 @@
+"""Benchmark of the DSA layer step (indexer -> top-k -> sparse MLA attention).
+
+Default workload: decode at 128K context -- 32 sequences, one query each,
+ctx_len 131072, index_topk 2048, 64 index heads x 128, 128 attention heads
+over a 576-wide latent (value = first 512).  A step is one pass of the whole
+path over one batch of synthetic inputs already resident in HBM.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload decode128k|decode128k_fp8|decode32k|prefill8k]
+
+Under torchrun (N > 1) every rank runs its own replica of the workload
+(decode shards by sequence, no collective): weak scaling, value = queries
+of all ranks / max-over-ranks time.  ``--impl reference`` times the CPU
+oracle (the only reference that exists for this path) on rank 0.
+"""
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def _peaks():
+    try:
+        with open(PEAKS_PATH) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", 0)), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during timing."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        sm.sort()
+        med = sm[len(sm) // 2] if sm else None
+        return {"sm_mhz": med, "sm_max_mhz": smax, "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def _workload_desc(wl):
+    return (f"{wl.name}: B={wl.batch}, n_q={wl.n_q}, ctx={wl.s_max}, index_topk={wl.topk}, "
+            f"H_I={wl.idx_heads}x{wl.idx_dim} ({'e4m3' if wl.idx_fp8 else wl.dtype}), "
+            f"H={wl.heads}, d_qk={wl.d_qk}, d_v={wl.d_v}")
+
+
+def _queries(wl):
+    return wl.batch * wl.n_q
+
+
+def _indexer_bytes(wl):
+    """Algorithmic HBM bytes of one indexer launch: every causal key row of the
+    index-key cache read once per query block (decode: once per query), plus
+    the query block, the head weights and the fp32 score row written."""
+    row = wl.idx_dim * (1 if wl.idx_fp8 else 2) + (4 if wl.idx_fp8 else 0)
+    if wl.n_q == 1:
+        keys = sum(wl.lengths())
+        return keys * row + wl.batch * (wl.idx_heads * wl.idx_dim * 2 + wl.idx_heads * 4) + keys * 4
+    pairs = sum(wl.n_q * (wl.n_q + 1) // 2 for _ in range(wl.batch))
+    return pairs * 4 + wl.batch * wl.s_max * row
+
+
+def _indexer_flops(wl):
+    if wl.n_q == 1:
+        pairs = sum(wl.lengths())
+    else:
+        pairs = wl.batch * wl.n_q * (wl.n_q + 1) // 2
+    return 2.0 * wl.idx_heads * wl.idx_dim * pairs
+
+
+def run_ours(args, wl):
+    import long_context_indexing_lightning_b200 as dsa
+
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    t = workloads.make_inputs(wl, dev, seed=rank)
+    shape = dsa.shape_from_workload(wl)
+    stream = torch.cuda.current_stream(dev)
+    ld = (wl.s_max + 3) // 4 * 4
+    scores = torch.empty(wl.batch, wl.n_q, ld, dtype=torch.float32, device=dev)
+    idx = torch.empty(wl.batch, wl.n_q, wl.topk, dtype=torch.int32, device=dev)
+    out = torch.empty(wl.batch, wl.n_q, wl.heads, wl.d_v, dtype=t["q"].dtype, device=dev)
+    ws_topk = torch.empty(max(1, dsa.workspace_bytes(shape, dsa.WS_TOPK)), dtype=torch.uint8, device=dev)
+    ws_attn = torch.empty(max(1, dsa.workspace_bytes(shape, dsa.WS_ATTN)), dtype=torch.uint8, device=dev)
+    k_idx, k_scale, q_idx, q_scale = t["k_idx"], None, t["q_idx"], None
+    q8 = qs = None
+    if wl.idx_fp8:
+        k_idx, k_scale = dsa.hadamard_quant_fp8(t["k_idx"])   # the cache as stored (quantise-on-write)
+        q8 = torch.empty(q_idx.shape, dtype=torch.uint8, device=dev)
+        qs = torch.empty(q_idx.shape[:-1], dtype=torch.float32, device=dev)
+        del t["k_idx"]
+
+    def step(ev=None):
+        if wl.idx_fp8:
+            dsa.hadamard_quant_fp8(q_idx, q8, qs, stream=stream)
+            qi, qsc = q8, qs
+        else:
+            qi, qsc = q_idx, None
+        if ev: ev[0].record(stream)
+        dsa.indexer_scores(shape, qi, k_idx, t["w"], t["ctx_len"], t["q_pos0"], scores=scores, q_scale=qsc,
+                           k_scale=k_scale, stream=stream)
+        if ev: ev[1].record(stream)
+        dsa.topk(shape, scores, t["ctx_len"], t["q_pos0"], idx=idx, workspace=ws_topk, stream=stream)
+        if ev: ev[2].record(stream)
+        dsa.sparse_mla_attn(shape, t["q"], t["kv"], idx, t["ctx_len"], out=out, workspace=ws_attn, stream=stream)
+        if ev: ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    rc, word = dsa.get_error(clear=True)
+    if rc != 0:
+        raise RuntimeError(f"device error word {word:#x} after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    if ws > 1:
+        torch.distributed.barrier()
+    total_ms = start.elapsed_time(end)
+    stage_ms = {"indexer": 0.0, "topk": 0.0, "attention": 0.0}
+    for e in evs:
+        stage_ms["indexer"] += e[0].elapsed_time(e[1])
+        stage_ms["topk"] += e[1].elapsed_time(e[2])
+        stage_ms["attention"] += e[2].elapsed_time(e[3])
+    stage_ms = {k: v / args.steps for k, v in stage_ms.items()}
+    rc, word = dsa.get_error(clear=True)
+    if rc != 0:
+        raise RuntimeError(f"device error word {word:#x} after timing")
+    if ws > 1:
+        tt = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_per_step = total_ms / args.steps
+
+    # end to end through the host-buffer entry point
+    e2e = _e2e(args, wl, dsa, shape, t, k_idx, k_scale, dev, stream)
+    if ws > 1:
+        tt = torch.tensor([e2e["ms"]], device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        e2e["ms"] = float(tt.item())
+
+    res = None
+    if rank == 0:
+        hbm, tf, tf_sus, src = _peaks()
+        idx_bytes = _indexer_bytes(wl)
+        idx_ms = stage_ms["indexer"]
+        achieved = idx_bytes / (idx_ms * 1e-3) / 1e9
+        q_total = _queries(wl) * ws
+        res = {
+            "metric": "DSA layer queries/s at 128K ctx" if wl.s_max == 131072 else f"DSA layer queries/s ({wl.name})",
+            "value": q_total / (ms_per_step * 1e-3),
+            "unit": "queries/s",
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if not wl.idx_fp8 else "bf16+e4m3-indexer",
+            "data": "synthetic (seeded gaussian, bf16)",
+            "config": {"workload": _workload_desc(wl), "global_batch": q_total, "seq_len": wl.s_max,
+                       "parallelism": f"replicas{ws}" if ws > 1 else "single",
+                       "l2": "inputs larger than L2 (index-key cache read each step)"},
+            "stages_ms": stage_ms,
+            "roofline": {"kernel": "indexer", "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                         "frac": achieved / hbm, "peak_source": f"{src} hbm_gbs", "traffic": None,
+                         "algorithmic_bytes": idx_bytes,
+                         "tensor_tflops": _indexer_flops(wl) / (idx_ms * 1e-3) / 1e12},
+            "gpu_launches": args.steps * (4 if wl.idx_fp8 else 3),
+            "clocks": clk,
+            "e2e": {"value": q_total / (e2e["ms"] * 1e-3), "unit": "queries/s",
+                    "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
+        }
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+    return res
+
+
+def _e2e(args, wl, dsa, shape, t, k_idx, k_scale, dev, stream):
+    """dsa_forward_host: this step's queries copied in from pinned memory, the
+    output copied back, caches resident on the device."""
+    pin = lambda x: x.cpu().pin_memory()
+    h = {k: pin(t[k]) for k in ("q_idx", "w", "q", "ctx_len", "q_pos0")}
+    h_out = torch.empty(wl.batch, wl.n_q, wl.heads, wl.d_v, dtype=t["q"].dtype).pin_memory()
+    wsb = torch.empty(dsa.workspace_bytes(shape, dsa.WS_FORWARD_HOST), dtype=torch.uint8, device=dev)
+    call = lambda: dsa.forward_host(shape, h["q_idx"], h["w"], h["q"], h["ctx_len"], h["q_pos0"], k_idx, t["kv"],
+                                    h_out, k_scale=k_scale, workspace=wsb, stream=stream)
+    for _ in range(max(1, args.warmup)):
+        call()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    s.record(stream)
+    for _ in range(args.steps):
+        call()
+    e.record(stream)
+    torch.cuda.synchronize(dev)
+    h2d = sum(v.numel() * v.element_size() for v in h.values())
+    d2h = h_out.numel() * h_out.element_size()
+    return {"ms": s.elapsed_time(e) / args.steps, "h2d": h2d, "d2h": d2h}
+
+
+def _oracle_sample(wl, n_rows, seed=0):
+    """The CPU oracle (as it stands) on `n_rows` query rows of the workload:
+    indexer scores -> top-k -> sparse attention.  Returns (seconds, rows)."""
+    import numpy as np
+    import oracle
+    sub = workloads.get(wl.name, batch=n_rows)
+    t = workloads.make_inputs(sub, "cuda" if torch.cuda.is_available() else "cpu", seed=seed)
+    h = {k: workloads.to_numpy(v) for k, v in t.items()}
+    rows = [(b, 0) for b in range(n_rows)]
+    t0 = time.perf_counter()
+    sc = oracle.indexer_scores(h["q_idx"], h["k_idx"], h["w"], h["ctx_len"], h["q_pos0"], rows=rows)
+    pos = np.array([h["q_pos0"][b] for b, _ in rows], dtype=np.int32)
+    idx = oracle.topk(np.where(np.isfinite(sc), sc, -np.inf).astype(np.float32), pos, sub.topk)
+    oracle.sparse_attn(h["q"], h["kv"], idx, sub.sm_scale, v=sub.d_v, rows=rows)
+    return time.perf_counter() - t0, n_rows
+
+
+def cpu_baseline(wl, n_rows=None):
+    import oracle
+    cores = oracle.num_threads()
+    n_rows = n_rows or max(1, min(wl.batch, cores))
+    secs, rows = _oracle_sample(wl, n_rows)
+    return {"value": rows / secs, "unit": "queries/s", "cores": cores, "kind": "oracle",
+            "sample": f"{rows} decode queries of the same workload (full {wl.s_max}-key context each), "
+                      f"{secs:.1f} s on {cores} host threads"}
+
+
+def run_reference(args, wl):
+    """The reference arm: the fp64 CPU oracle, timed on the host cores."""
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return None
+    import oracle
+    cores = oracle.num_threads()
+    n_rows = max(1, min(wl.batch, cores))
+    for _ in range(args.warmup and 1):
+        _oracle_sample(wl, 1, seed=99)
+    secs = 0.0
+    rows = 0
+    for i in range(args.steps):
+        s, r = _oracle_sample(wl, n_rows, seed=i)
+        secs += s
+        rows += r
+    value = rows / secs
+    line = {
+        "impl": "reference",
+        "metric": "DSA layer queries/s at 128K ctx" if wl.s_max == 131072 else f"DSA layer queries/s ({wl.name})",
+        "value": value, "unit": "queries/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded gaussian, bf16)",
+        "config": {"workload": _workload_desc(wl), "global_batch": n_rows, "seq_len": wl.s_max,
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": "queries/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: {n_rows} decode queries of the workload"},
+        "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    return line
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode128k", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    wl = workloads.get(args.workload)
+    if args.impl == "reference":
+        line = run_reference(args, wl)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    res = run_ours(args, wl)
+    ws, rank, _ = _dist()
+    if rank == 0:
+        if ws == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(wl)
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,234 @@
+/*
+ * dsa.h -- C ABI of libdsa.so, the DeepSeek Sparse Attention (DSA) layer
+ * step on one NVIDIA B200 (sm_100a).
+ *
+ * The step has three parts, each a CUDA kernel of this library:
+ *   1. Lightning-indexer scores of every query against every previous key of
+ *      the single-head indexer key cache (DeepSeek-V3.2 model doc,
+ *      Transformers, section "DeepSeek Sparse Attention (DSA)", item 1, and
+ *      the paragraph on the indexer's own key cache);
+ *   2. per-query top-index_topk selection (same section, item 2);
+ *   3. MLA attention over the selected latent rows only (same section,
+ *      item 2: O(index_topk) per query instead of O(L)).
+ * Shapes follow section DeepseekV32Config (index_n_heads 64, index_head_dim
+ * 128, index_topk 2048, num_attention_heads 128, kv_lora_rank 512,
+ * qk_rope_head_dim 64).
+ *
+ * Conventions for every entry point
+ *   - All tensor arguments are DEVICE pointers to row-major, contiguous
+ *     buffers in the layouts stated below, owned by the caller, except where
+ *     an argument is marked HOST.  The library keeps no pointer after a call.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream).  No call synchronises unless stated; none allocates device
+ *     memory; scratch space comes from the caller's `workspace`, sized with
+ *     dsa_workspace_bytes().
+ *   - Argument errors are reported synchronously by the return value and
+ *     nothing is enqueued.  A failed launch returns DSA_ERR_CUDA.  Errors
+ *     found by a kernel while it runs (a bounded wait that expired, an index
+ *     out of range) are recorded in a per-device error word inside the
+ *     library and read with dsa_get_error().
+ *   - Pointers fed to the tensor-memory-accelerator paths (q_idx, k_idx for
+ *     BF16 / E4M3) must be 16-byte aligned.
+ *   - Query t of sequence b sits at position pos = q_pos0[b] + t, and
+ *     0 <= q_pos0[b], q_pos0[b] + n_q <= ctx_len[b] <= s_max.  A query sees
+ *     the keys s <= pos ("previous keys" is read as including its own
+ *     position; a decode query is the newest token, already in the cache).
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DSA_OK = 0,
+    DSA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer */
+    DSA_ERR_UNSUPPORTED = 2,  /* valid but not implemented shape/dtype combination */
+    DSA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than dsa_workspace_bytes() */
+    DSA_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
+    DSA_ERR_TIMEOUT = 5,      /* (device) a bounded wait inside a kernel expired */
+    DSA_ERR_BAD_INDEX = 6     /* (device) an attention index was >= ctx_len and was skipped */
+} dsa_status_t;
+
+typedef enum {
+    DSA_F32 = 0,   /* IEEE fp32 */
+    DSA_BF16 = 1,  /* bfloat16 */
+    DSA_E4M3 = 2   /* OCP FP8 E4M3 codes (uint8) with fp32 per-row scales */
+} dsa_dtype_t;
+
+/* Shape and numeric options shared by every call (plain data, by pointer). */
+typedef struct {
+    int32_t batch;      /* B, sequences */
+    int32_t n_q;        /* queries per sequence (1 = decode) */
+    int32_t s_max;      /* cache capacity: rows per sequence of every cache */
+    int32_t idx_heads;  /* H_I, index_n_heads (64) */
+    int32_t idx_dim;    /* D_I, index_head_dim (128) */
+    int32_t topk;       /* k, index_topk (2048) */
+    int32_t heads;      /* H, attention heads (128) */
+    int32_t d_qk;       /* query/key width per head: 576 = kv_lora_rank 512 + rope 64 */
+    int32_t d_v;        /* value/output width per head (512, the latent) */
+    int32_t kv_heads;   /* 1 = absorbed MLA (one shared latent row per token, value = its
+                           first d_v columns); > 1 = MHA/GQA with a separate v tensor */
+    int32_t idx_dtype;  /* dsa_dtype_t of the indexer inputs: F32, BF16 or E4M3 */
+    int32_t attn_dtype; /* dsa_dtype_t of q, kv, v and out: F32 or BF16 */
+    float idx_scale;    /* > 0: multiplies each head's dot product inside the ReLU (1.0) */
+    float sm_scale;     /* softmax scale of the attention logits (1/sqrt(192) for MLA) */
+    int32_t q_chunk;    /* dsa_forward only: queries per sequence processed per round of
+                           indexer -> top-k -> attention; 0 = all n_q at once */
+} dsa_shape_t;
+
+/* Which workspace dsa_workspace_bytes() sizes. */
+enum { DSA_WS_TOPK = 0, DSA_WS_ATTN = 1, DSA_WS_FORWARD = 2, DSA_WS_FORWARD_HOST = 3 };
+
+/*
+ * Lightning-indexer scores (section DSA, item 1; key cache paragraph).
+ *   I[b,t,s] = sum_h w[b,t,h] * max(0, idx_scale * <q_idx[b,t,h,:], k_idx[b,s,:]>)
+ *              for s <= pos(b,t);  -inf for pos(b,t) < s < ctx_len[b].
+ * The per-head ReLU and the weights_proj weighting are this library's
+ * reading; the pages name the score but do not print its formula.
+ * Arguments
+ *   q_idx   [B][n_q][H_I][D_I]  idx_dtype (E4M3: codes of the Hadamard-rotated query)
+ *   q_scale [B][n_q][H_I] fp32  E4M3 only (else NULL): per (query, head) scale
+ *   k_idx   [B][s_max][D_I]     idx_dtype (E4M3: codes of the rotated key)
+ *   k_scale [B][s_max] fp32     E4M3 only (else NULL): per key scale
+ *   w       [B][n_q][H_I] fp32  head weights (the weights_proj output)
+ *   ctx_len, q_pos0 [B] int32   device
+ *   scores  [B][n_q][ld_scores] fp32 output; columns s < ctx_len[b] are
+ *           written, the rest of each row is left untouched.
+ *   ld_scores >= s_max, a multiple of 4.
+ * BF16 and E4M3 run on the tensor cores (tcgen05) and need D_I = 128 and
+ * H_I in {16, 32, 64, 128}; F32 runs on the CUDA cores for any D_I <= 256,
+ * H_I <= 128.  E4M3 scores equal the scores of the dequantised inputs.
+ */
+dsa_status_t dsa_indexer_scores(const dsa_shape_t *shape,
+                                const void *q_idx, const float *q_scale,
+                                const void *k_idx, const float *k_scale,
+                                const float *w,
+                                const int32_t *ctx_len, const int32_t *q_pos0,
+                                float *scores, int64_t ld_scores,
+                                void *stream);
+
+/*
+ * Fine-grained token selection (section DSA, item 2): for each query, the
+ * min(topk, pos+1) keys s <= pos with the largest scores; among equal scores
+ * the lower index wins (the pages are silent on ties; -0.0 equals +0.0).
+ * Arguments
+ *   scores [B][n_q][ld_scores] fp32, finite for s <= pos.
+ *   idx    [B][n_q][topk] int32 output: the kept indices in ascending order,
+ *          then -1 padding.
+ *   workspace: dsa_workspace_bytes(shape, DSA_WS_TOPK) bytes (may be 0).
+ * The selection is exact: it is decided on the fp32 bit patterns.
+ */
+dsa_status_t dsa_topk(const dsa_shape_t *shape,
+                      const float *scores, int64_t ld_scores,
+                      const int32_t *ctx_len, const int32_t *q_pos0,
+                      int32_t *idx,
+                      void *workspace, size_t workspace_bytes,
+                      void *stream);
+
+/*
+ * Attention over the selected keys only (section DSA, item 2).  For head h
+ * of query (b,t), over the listed keys j (entries < 0 are skipped):
+ *   l_j = sm_scale * <q[b,t,h,:], K[b,idx_j,:]>,  O = sum_j softmax(l)_j V[b,idx_j,:]
+ * kv_heads == 1 (absorbed MLA): K = kv[b,s,:] (d_qk wide), V = kv[b,s,:d_v],
+ * shared by all heads (v must be NULL).  kv_heads > 1: K = kv[b,s,g,:],
+ * V = v[b,s,g,:] with g = h / (H / kv_heads).
+ * Arguments
+ *   q   [B][n_q][H][d_qk]          attn_dtype
+ *   kv  [B][s_max][kv_heads][d_qk] attn_dtype
+ *   v   [B][s_max][kv_heads][d_v]  attn_dtype, or NULL when kv_heads == 1
+ *   idx [B][n_q][topk] int32; an entry >= ctx_len[b] is skipped and flagged
+ *       DSA_ERR_BAD_INDEX in the device error word.
+ *   out [B][n_q][H][d_v] attn_dtype output (BF16: rounded to nearest even)
+ *   lse [B][n_q][H] fp32 output or NULL: log-sum-exp of the scaled logits
+ *       (-inf, with out = 0, when no key is listed).
+ *   workspace: dsa_workspace_bytes(shape, DSA_WS_ATTN) bytes.
+ * BF16 with d_qk = 576, d_v = 512, kv_heads = 1, H a multiple of 64 runs on
+ * the tensor cores; F32 runs on the CUDA cores for d_qk, d_v in {32, 64,
+ * 128} (and the MLA sizes).
+ */
+dsa_status_t dsa_sparse_mla_attn(const dsa_shape_t *shape,
+                                 const void *q, const void *kv, const void *v,
+                                 const int32_t *idx, const int32_t *ctx_len,
+                                 void *out, float *lse,
+                                 void *workspace, size_t workspace_bytes,
+                                 void *stream);
+
+/*
+ * Hadamard rotation + FP8 quantisation of rows (section DSA, item 1: the
+ * reference indexer runs in FP8 after the orthogonal `rotate_activation`,
+ * Hq.Hk = q.k).  For each row r of `rows` rows of `dim` (= 128) elements:
+ *   y = H x (orthonormal Sylvester-Hadamard, entries +-1/sqrt(dim)),
+ *   scale[r] = max|y| / 448 (1 for an all-zero row),
+ *   x_fp8[r,:] = e4m3(y / scale[r]), round to nearest even, saturating.
+ * x: [rows][dim] in x_dtype (BF16 or F32); x_fp8 [rows][dim] uint8;
+ * scale [rows] fp32.  Used on keys when they enter the cache and on the
+ * indexer queries of each step.
+ */
+dsa_status_t dsa_hadamard_quant_fp8(const void *x, int32_t x_dtype, int64_t rows, int32_t dim,
+                                    uint8_t *x_fp8, float *scale, void *stream);
+
+/*
+ * The whole layer step: indexer scores -> top-k -> sparse attention, in
+ * rounds of shape->q_chunk queries per sequence (scores of one round live in
+ * the workspace).  Inputs as in the calls above, except with
+ * idx_dtype == E4M3: q_idx is BF16 [B][n_q][H_I][D_I] and is rotated and
+ * quantised inside the step (q_scale must be NULL), while k_idx/k_scale are
+ * the FP8 key cache as written by dsa_hadamard_quant_fp8.
+ *   idx_out [B][n_q][topk] int32 or NULL: the selected indices.
+ *   workspace: dsa_workspace_bytes(shape, DSA_WS_FORWARD) bytes.
+ */
+dsa_status_t dsa_forward(const dsa_shape_t *shape,
+                         const void *q_idx, const float *q_scale,
+                         const void *k_idx, const float *k_scale,
+                         const float *w,
+                         const void *q, const void *kv, const void *v,
+                         const int32_t *ctx_len, const int32_t *q_pos0,
+                         void *out, float *lse, int32_t *idx_out,
+                         void *workspace, size_t workspace_bytes,
+                         void *stream);
+
+/*
+ * dsa_forward with the per-step tensors in HOST memory: q_idx, w, q,
+ * ctx_len, q_pos0 (inputs) and out, lse (outputs; lse may be NULL) are HOST
+ * pointers (page-locked memory gives asynchronous copies), while the caches
+ * k_idx, k_scale, kv, v stay on the device as the layer's resident state.
+ * The call copies the inputs in (one cudaMemcpyAsync each), runs the step,
+ * copies the outputs back and synchronises `stream` before returning.
+ * workspace: dsa_workspace_bytes(shape, DSA_WS_FORWARD_HOST) bytes.
+ */
+dsa_status_t dsa_forward_host(const dsa_shape_t *shape,
+                              const void *h_q_idx, const float *h_w, const void *h_q,
+                              const int32_t *h_ctx_len, const int32_t *h_q_pos0,
+                              const void *k_idx, const float *k_scale,
+                              const void *kv, const void *v,
+                              void *h_out, float *h_lse,
+                              void *workspace, size_t workspace_bytes,
+                              void *stream);
+
+/* Bytes of device workspace a call needs (DSA_WS_*); 0 for an invalid shape. */
+size_t dsa_workspace_bytes(const dsa_shape_t *shape, int32_t which);
+
+/*
+ * Reads (and, if clear != 0, resets) the device error word of the current
+ * device.  Synchronises the device.  Returns DSA_OK, DSA_ERR_TIMEOUT or
+ * DSA_ERR_BAD_INDEX (the first recorded kind), or DSA_ERR_CUDA if the read
+ * itself failed.  `detail`, if not NULL, receives the raw word.
+ */
+dsa_status_t dsa_get_error(int32_t clear, uint32_t *detail);
+
+/* Static English text for a status code. */
+const char *dsa_status_string(dsa_status_t status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int32_t dsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

@@ -1,0 +1,213 @@
+"""Python binding of libdsa.so -- the DeepSeek Sparse Attention (DSA) layer
+step on one B200: Lightning-indexer scores, causal top-k selection, and MLA
+attention over the selected latent rows (DeepSeek-V3.2 model doc,
+Transformers, section "DeepSeek Sparse Attention (DSA)").
+
+This module only marshals arguments: torch tensors supply device memory and
+the current CUDA stream; every step runs in the library's CUDA kernels.  If
+the library is missing, importing the functions raises -- there is no CPU
+path.  Names and argument order follow ``include/dsa.h``.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdsa.so")
+
+DSA_F32, DSA_BF16, DSA_E4M3 = 0, 1, 2
+WS_TOPK, WS_ATTN, WS_FORWARD, WS_FORWARD_HOST = 0, 1, 2, 3
+
+STATUS = {
+    0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "DSA_ERR_WORKSPACE",
+    4: "DSA_ERR_CUDA", 5: "DSA_ERR_TIMEOUT", 6: "DSA_ERR_BAD_INDEX",
+}
+
+EXPORTS = (
+    "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_hadamard_quant_fp8", "dsa_forward",
+    "dsa_forward_host", "dsa_workspace_bytes", "dsa_get_error", "dsa_status_string", "dsa_version",
+)
+
+
+class DsaError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+class Shape(ctypes.Structure):
+    """Mirror of ``dsa_shape_t``."""
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("n_q", ctypes.c_int32), ("s_max", ctypes.c_int32),
+        ("idx_heads", ctypes.c_int32), ("idx_dim", ctypes.c_int32), ("topk", ctypes.c_int32),
+        ("heads", ctypes.c_int32), ("d_qk", ctypes.c_int32), ("d_v", ctypes.c_int32),
+        ("kv_heads", ctypes.c_int32), ("idx_dtype", ctypes.c_int32), ("attn_dtype", ctypes.c_int32),
+        ("idx_scale", ctypes.c_float), ("sm_scale", ctypes.c_float), ("q_chunk", ctypes.c_int32),
+    ]
+
+    def replace(self, **kw):
+        s = Shape()
+        ctypes.pointer(s)[0] = self
+        for k, v in kw.items():
+            setattr(s, k, v)
+        return s
+
+
+_lib = None
+
+
+def lib():
+    """Load libdsa.so (built in-tree by ``build.py``); raises if it is absent."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libdsa.so not built ({LIB_PATH}); run python -m long_context_indexing_lightning_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        P, S = ctypes.c_void_p, ctypes.POINTER(Shape)
+        i32, i64, sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+        L.dsa_indexer_scores.argtypes = [S, P, P, P, P, P, P, P, P, i64, P]
+        L.dsa_topk.argtypes = [S, P, i64, P, P, P, P, sz, P]
+        L.dsa_sparse_mla_attn.argtypes = [S, P, P, P, P, P, P, P, P, sz, P]
+        L.dsa_hadamard_quant_fp8.argtypes = [P, i32, i64, i32, P, P, P]
+        L.dsa_forward.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
+        L.dsa_forward_host.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
+        L.dsa_workspace_bytes.argtypes = [S, i32]
+        L.dsa_workspace_bytes.restype = sz
+        L.dsa_get_error.argtypes = [i32, ctypes.POINTER(ctypes.c_uint32)]
+        L.dsa_status_string.argtypes = [i32]
+        L.dsa_status_string.restype = ctypes.c_char_p
+        L.dsa_version.restype = i32
+        for name in EXPORTS:
+            if name not in ("dsa_workspace_bytes", "dsa_status_string", "dsa_version"):
+                getattr(L, name).restype = i32
+        _lib = L
+    return _lib
+
+
+def _p(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(rc, where):
+    if rc != 0:
+        raise DsaError(rc, where)
+
+
+def _dtype_code(t: torch.dtype) -> int:
+    return {torch.float32: DSA_F32, torch.bfloat16: DSA_BF16, torch.uint8: DSA_E4M3}[t]
+
+
+def make_shape(batch, n_q, s_max, idx_heads=64, idx_dim=128, topk=2048, heads=128, d_qk=576, d_v=512,
+               kv_heads=1, idx_dtype=DSA_BF16, attn_dtype=DSA_BF16, idx_scale=1.0, sm_scale=None,
+               q_chunk=0) -> Shape:
+    if sm_scale is None:
+        sm_scale = (192 ** -0.5) if kv_heads == 1 else d_qk ** -0.5
+    return Shape(batch, n_q, s_max, idx_heads, idx_dim, topk, heads, d_qk, d_v, kv_heads, idx_dtype,
+                 attn_dtype, float(idx_scale), float(sm_scale), q_chunk)
+
+
+def shape_from_workload(wl, q_chunk=0) -> Shape:
+    """Shape for a ``workloads.Workload`` (duck-typed: reads its fields)."""
+    dt = DSA_BF16 if wl.dtype == "bf16" else DSA_F32
+    return make_shape(wl.batch, wl.n_q, wl.s_max, wl.idx_heads, wl.idx_dim, wl.topk, wl.heads, wl.d_qk, wl.d_v,
+                      wl.kv_heads, DSA_E4M3 if wl.idx_fp8 else dt, dt, wl.idx_scale, wl.sm_scale, q_chunk)
+
+
+def workspace_bytes(shape: Shape, which: int) -> int:
+    return int(lib().dsa_workspace_bytes(ctypes.byref(shape), which))
+
+
+def _workspace(shape, which, ws, device):
+    n = workspace_bytes(shape, which)
+    if ws is None and n > 0:
+        ws = torch.empty(n, dtype=torch.uint8, device=device)
+    return ws, (ws.numel() if ws is not None else 0)
+
+
+def indexer_scores(shape, q_idx, k_idx, w, ctx_len, q_pos0, scores=None, q_scale=None, k_scale=None, ld=None,
+                   stream=None):
+    """Scores [B, n_q, ld] fp32 (see dsa_indexer_scores)."""
+    if scores is None:
+        ld = ld or ((shape.s_max + 3) // 4 * 4)
+        scores = torch.empty(shape.batch, shape.n_q, ld, dtype=torch.float32, device=k_idx.device)
+    ld = scores.stride(1) if scores.dim() == 3 else scores.stride(0)
+    _check(lib().dsa_indexer_scores(ctypes.byref(shape), _p(q_idx), _p(q_scale), _p(k_idx), _p(k_scale), _p(w),
+                                    _p(ctx_len), _p(q_pos0), _p(scores), ld, _stream(stream)),
+           "dsa_indexer_scores")
+    return scores
+
+
+def topk(shape, scores, ctx_len, q_pos0, idx=None, workspace=None, stream=None):
+    """Indices [B, n_q, topk] int32, ascending then -1 (see dsa_topk)."""
+    if idx is None:
+        idx = torch.empty(shape.batch, shape.n_q, shape.topk, dtype=torch.int32, device=scores.device)
+    ws, n = _workspace(shape, WS_TOPK, workspace, scores.device)
+    ld = scores.stride(1) if scores.dim() == 3 else scores.stride(0)
+    _check(lib().dsa_topk(ctypes.byref(shape), _p(scores), ld, _p(ctx_len), _p(q_pos0), _p(idx), _p(ws), n,
+                          _stream(stream)), "dsa_topk")
+    return idx
+
+
+def sparse_mla_attn(shape, q, kv, idx, ctx_len, out=None, v=None, lse=None, workspace=None, stream=None):
+    """Attention output [B, n_q, H, d_v] (see dsa_sparse_mla_attn)."""
+    if out is None:
+        out = torch.empty(shape.batch, shape.n_q, shape.heads, shape.d_v, dtype=q.dtype, device=q.device)
+    ws, n = _workspace(shape, WS_ATTN, workspace, q.device)
+    _check(lib().dsa_sparse_mla_attn(ctypes.byref(shape), _p(q), _p(kv), _p(v), _p(idx), _p(ctx_len), _p(out),
+                                     _p(lse), _p(ws), n, _stream(stream)), "dsa_sparse_mla_attn")
+    return out
+
+
+def hadamard_quant_fp8(x, x8=None, scale=None, stream=None):
+    """Rotate + quantise rows of 128: returns (codes uint8, scale fp32)."""
+    dim = x.shape[-1]
+    rows = x.numel() // dim
+    if x8 is None:
+        x8 = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if scale is None:
+        scale = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    _check(lib().dsa_hadamard_quant_fp8(_p(x), _dtype_code(x.dtype), rows, dim, _p(x8), _p(scale),
+                                        _stream(stream)), "dsa_hadamard_quant_fp8")
+    return x8, scale
+
+
+def forward(shape, q_idx, k_idx, w, q, kv, ctx_len, q_pos0, out=None, v=None, q_scale=None, k_scale=None,
+            lse=None, idx_out=None, workspace=None, stream=None):
+    """The whole layer step (see dsa_forward); returns out."""
+    if out is None:
+        out = torch.empty(shape.batch, shape.n_q, shape.heads, shape.d_v, dtype=q.dtype, device=q.device)
+    ws, n = _workspace(shape, WS_FORWARD, workspace, q.device)
+    _check(lib().dsa_forward(ctypes.byref(shape), _p(q_idx), _p(q_scale), _p(k_idx), _p(k_scale), _p(w), _p(q),
+                             _p(kv), _p(v), _p(ctx_len), _p(q_pos0), _p(out), _p(lse), _p(idx_out), _p(ws), n,
+                             _stream(stream)), "dsa_forward")
+    return out
+
+
+def forward_host(shape, h_q_idx, h_w, h_q, h_ctx_len, h_q_pos0, k_idx, kv, h_out, v=None, k_scale=None,
+                 h_lse=None, workspace=None, stream=None):
+    """The layer step with this step's tensors in host memory (see dsa_forward_host)."""
+    ws, n = _workspace(shape, WS_FORWARD_HOST, workspace, k_idx.device)
+    _check(lib().dsa_forward_host(ctypes.byref(shape), _p(h_q_idx), _p(h_w), _p(h_q), _p(h_ctx_len), _p(h_q_pos0),
+                                  _p(k_idx), _p(k_scale), _p(kv), _p(v), _p(h_out), _p(h_lse), _p(ws), n,
+                                  _stream(stream)), "dsa_forward_host")
+    return h_out
+
+
+def get_error(clear=True):
+    """(status, raw word) of the device error word; synchronises the device."""
+    word = ctypes.c_uint32(0)
+    rc = lib().dsa_get_error(1 if clear else 0, ctypes.byref(word))
+    return rc, word.value

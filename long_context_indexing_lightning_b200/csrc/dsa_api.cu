@@ -1,0 +1,521 @@
+// C ABI of libdsa.so: argument checks, workspace layout, dispatch to the
+// kernels, per-device set-up (SM count, error word, tensor-map encoder).
+// The operations and their sources are documented in include/dsa.h.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "dsa.h"
+#include "dsa_common.cuh"
+#include "dsa_internal.h"
+
+namespace dsa {
+
+// Per-device error word: bit kErrTimeout / kErrBadIndex, set by kernels.
+static __device__ uint32_t g_error_word[4];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mutex;
+int g_sm_count[kMaxDevices] = {};
+uint32_t* g_err_ptr[kMaxDevices] = {};
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+bool current_device(int* dev) { return cudaGetDevice(dev) == cudaSuccess && *dev >= 0 && *dev < kMaxDevices; }
+
+// One-time set-up of `dev` (must be the current device): SM count and the
+// device address of the error word.
+bool ensure_device(int dev) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_sm_count[dev] > 0 && g_err_ptr[dev] != nullptr) return true;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) return false;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess || p == nullptr) return false;
+  g_sm_count[dev] = sms;
+  g_err_ptr[dev] = static_cast<uint32_t*>(p);
+  return true;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool valid_dtype(int d) { return d == DSA_F32 || d == DSA_BF16 || d == DSA_E4M3; }
+
+size_t elem_size(int dtype) { return dtype == DSA_F32 ? 4 : (dtype == DSA_BF16 ? 2 : 1); }
+
+dsa_status_t check_shape(const dsa_shape_t* s) {
+  if (s == nullptr) return DSA_ERR_INVALID_ARG;
+  if (s->batch < 0 || s->n_q < 0 || s->s_max < 0) return DSA_ERR_INVALID_ARG;
+  if (s->idx_heads <= 0 || s->idx_dim <= 0 || s->topk <= 0) return DSA_ERR_INVALID_ARG;
+  if (s->heads <= 0 || s->d_qk <= 0 || s->d_v <= 0 || s->kv_heads <= 0) return DSA_ERR_INVALID_ARG;
+  if (s->heads % s->kv_heads != 0) return DSA_ERR_INVALID_ARG;
+  if (s->kv_heads == 1 && s->d_v > s->d_qk) return DSA_ERR_INVALID_ARG;
+  if (!valid_dtype(s->idx_dtype) || !(s->attn_dtype == DSA_F32 || s->attn_dtype == DSA_BF16))
+    return DSA_ERR_INVALID_ARG;
+  if (!(s->idx_scale > 0.f) || !std::isfinite(s->idx_scale)) return DSA_ERR_INVALID_ARG;
+  if (!std::isfinite(s->sm_scale)) return DSA_ERR_INVALID_ARG;
+  if (s->q_chunk < 0) return DSA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(s->batch) * s->s_max > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(s->batch) * s->n_q * s->idx_heads > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+// ------------------------------------------------------------- stages --
+dsa_status_t run_indexer(const dsa_shape_t* s, int dev, cudaStream_t st, int B, int n_q, int t_off,
+                         const void* q_idx, const float* q_scale, const void* k_idx, const float* k_scale,
+                         const float* w, const int32_t* ctx_len, const int32_t* q_pos0, float* scores,
+                         int64_t ld) {
+  IndexerArgs a;
+  a.device = dev;
+  a.stream = st;
+  a.B = B;
+  a.n_q = n_q;
+  a.s_max = s->s_max;
+  a.H = s->idx_heads;
+  a.D = s->idx_dim;
+  a.dtype = s->idx_dtype;
+  a.q_idx = q_idx;
+  a.q_scale = q_scale;
+  a.k_idx = k_idx;
+  a.k_scale = k_scale;
+  a.w = w;
+  a.ctx_len = ctx_len;
+  a.q_pos0 = q_pos0;
+  a.t_off = t_off;
+  a.scores = scores;
+  a.ld = ld;
+  a.idx_scale = s->idx_scale;
+  a.err = g_err_ptr[dev];
+  if (B == 0 || n_q == 0 || s->s_max == 0) return DSA_OK;
+  if (s->idx_dtype == DSA_F32) return indexer_simt(a);
+  return indexer_tc(a);
+}
+
+dsa_status_t run_topk(const dsa_shape_t* s, int dev, cudaStream_t st, int B, int n_q, int t_off, const float* scores,
+                      int64_t ld, const int32_t* ctx_len, const int32_t* q_pos0, int32_t* idx, void* ws,
+                      size_t ws_bytes) {
+  TopkArgs a;
+  a.device = dev;
+  a.stream = st;
+  a.B = B;
+  a.n_q = n_q;
+  a.s_max = s->s_max;
+  a.k = s->topk;
+  a.scores = scores;
+  a.ld = ld;
+  a.ctx_len = ctx_len;
+  a.q_pos0 = q_pos0;
+  a.t_off = t_off;
+  a.idx = idx;
+  a.ws = ws;
+  a.ws_bytes = ws_bytes;
+  a.err = g_err_ptr[dev];
+  if (B == 0 || n_q == 0) return DSA_OK;
+  return topk_radix(a);
+}
+
+dsa_status_t run_attn(const dsa_shape_t* s, int dev, cudaStream_t st, int B, int n_q, const void* q, const void* kv,
+                      const void* v, const int32_t* idx, const int32_t* ctx_len, void* out, float* lse, void* ws,
+                      size_t ws_bytes) {
+  AttnArgs a;
+  a.device = dev;
+  a.stream = st;
+  a.B = B;
+  a.n_q = n_q;
+  a.s_max = s->s_max;
+  a.H = s->heads;
+  a.KVH = s->kv_heads;
+  a.d_qk = s->d_qk;
+  a.d_v = s->d_v;
+  a.k = s->topk;
+  a.dtype = s->attn_dtype;
+  a.q = q;
+  a.kv = kv;
+  a.v = v;
+  a.idx = idx;
+  a.ctx_len = ctx_len;
+  a.out = out;
+  a.lse = lse;
+  a.sm_scale = s->sm_scale;
+  a.ws = ws;
+  a.ws_bytes = ws_bytes;
+  a.err = g_err_ptr[dev];
+  if (B == 0 || n_q == 0) return DSA_OK;
+  if (s->attn_dtype == DSA_BF16 && attn_tc_supported(a.H, a.d_qk, a.d_v, a.KVH)) return attn_tc(a);
+  return attn_simt(a);
+}
+
+// Workspace layout of dsa_forward (all offsets 256-byte aligned).
+struct FwdLayout {
+  int chunk;          // queries per sequence per round
+  int64_t ld;         // score row stride
+  size_t off_scores, off_idx, off_q8, off_qs, off_topk, off_attn;
+  size_t topk_bytes, attn_bytes;
+  size_t total;
+  // host-variant staging
+  size_t off_h_qidx, off_h_w, off_h_q, off_h_ctx, off_h_pos, off_h_out, off_h_lse;
+  size_t total_host;
+};
+
+FwdLayout forward_layout(const dsa_shape_t* s) {
+  FwdLayout L{};
+  const int B = s->batch;
+  L.chunk = (s->q_chunk > 0 && s->q_chunk < s->n_q) ? s->q_chunk : s->n_q;
+  L.ld = static_cast<int64_t>(align_up(static_cast<size_t>(std::max(s->s_max, 1)), 4));
+  size_t off = 0;
+  L.off_scores = off;
+  off = align_up(off + static_cast<size_t>(B) * L.chunk * L.ld * 4, 256);
+  L.off_idx = off;
+  off = align_up(off + static_cast<size_t>(B) * L.chunk * s->topk * 4, 256);
+  L.off_q8 = off;
+  L.off_qs = off;
+  if (s->idx_dtype == DSA_E4M3) {
+    off = align_up(off + static_cast<size_t>(B) * s->n_q * s->idx_heads * s->idx_dim, 256);
+    L.off_qs = off;
+    off = align_up(off + static_cast<size_t>(B) * s->n_q * s->idx_heads * 4, 256);
+  }
+  L.off_topk = off;
+  L.topk_bytes = topk_workspace_bytes(B, L.chunk, s->s_max, s->topk);
+  off = align_up(off + L.topk_bytes, 256);
+  L.off_attn = off;
+  L.attn_bytes = attn_workspace_bytes(B, L.chunk, s->heads, s->d_qk, s->d_v, s->kv_heads, s->topk, s->attn_dtype);
+  off = align_up(off + L.attn_bytes, 256);
+  L.total = off;
+  // staging for dsa_forward_host
+  const size_t ai = elem_size(s->idx_dtype == DSA_E4M3 ? DSA_BF16 : s->idx_dtype);
+  const size_t aa = elem_size(s->attn_dtype);
+  L.off_h_qidx = off;
+  off = align_up(off + static_cast<size_t>(B) * s->n_q * s->idx_heads * s->idx_dim * ai, 256);
+  L.off_h_w = off;
+  off = align_up(off + static_cast<size_t>(B) * s->n_q * s->idx_heads * 4, 256);
+  L.off_h_q = off;
+  off = align_up(off + static_cast<size_t>(B) * s->n_q * s->heads * s->d_qk * aa, 256);
+  L.off_h_ctx = off;
+  off = align_up(off + static_cast<size_t>(B) * 4, 256);
+  L.off_h_pos = off;
+  off = align_up(off + static_cast<size_t>(B) * 4, 256);
+  L.off_h_out = off;
+  off = align_up(off + static_cast<size_t>(B) * s->n_q * s->heads * s->d_v * aa, 256);
+  L.off_h_lse = off;
+  off = align_up(off + static_cast<size_t>(B) * s->n_q * s->heads * 4, 256);
+  L.total_host = off;
+  return L;
+}
+
+dsa_status_t check_indexer_inputs(const dsa_shape_t* s, const void* q_idx, const float* q_scale, const void* k_idx,
+                                  const float* k_scale, const float* w, const int32_t* ctx_len,
+                                  const int32_t* q_pos0) {
+  if (!q_idx || !k_idx || !w || !ctx_len || !q_pos0) return DSA_ERR_INVALID_ARG;
+  if (s->idx_dtype == DSA_E4M3 && (!q_scale || !k_scale)) return DSA_ERR_INVALID_ARG;
+  if (s->idx_dtype != DSA_F32) {
+    if (!aligned16(q_idx) || !aligned16(k_idx)) return DSA_ERR_INVALID_ARG;
+    if (s->idx_dim != 128) return DSA_ERR_UNSUPPORTED;
+    if (!indexer_tc_supported(s->idx_heads, s->idx_dim)) return DSA_ERR_UNSUPPORTED;
+  } else {
+    if (s->idx_dim > 256 || s->idx_heads > 128) return DSA_ERR_UNSUPPORTED;
+  }
+  return DSA_OK;
+}
+
+dsa_status_t check_attn_inputs(const dsa_shape_t* s, const void* q, const void* kv, const void* v, const void* idx,
+                               const void* ctx_len, const void* out) {
+  if (!q || !kv || !idx || !ctx_len || !out) return DSA_ERR_INVALID_ARG;
+  if (s->kv_heads == 1 && v != nullptr) return DSA_ERR_INVALID_ARG;
+  if (s->kv_heads > 1 && v == nullptr) return DSA_ERR_INVALID_ARG;
+  if (s->attn_dtype == DSA_BF16 && attn_tc_supported(s->heads, s->d_qk, s->d_v, s->kv_heads)) {
+    if (!aligned16(q) || !aligned16(kv) || !aligned16(out)) return DSA_ERR_INVALID_ARG;
+    return DSA_OK;
+  }
+  const bool simt_ok = (s->d_qk == 32 && s->d_v == 32) || (s->d_qk == 64 && s->d_v == 64) ||
+                       (s->d_qk == 128 && s->d_v == 128) || (s->d_qk == 576 && s->d_v == 512);
+  return simt_ok ? DSA_OK : DSA_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+int device_sm_count(int dev) { return (dev >= 0 && dev < kMaxDevices) ? g_sm_count[dev] : 0; }
+
+uint32_t* device_error_word(int dev) { return (dev >= 0 && dev < kMaxDevices) ? g_err_ptr[dev] : nullptr; }
+
+bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes, uint64_t inner,
+                  uint64_t rows, uint32_t box_inner, uint32_t box_rows) {
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (g_encode == nullptr) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return false;
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+  }
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * static_cast<uint64_t>(elem_bytes)};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool indexer_tc_supported(int H, int D) { return D == 128 && (H == 16 || H == 32 || H == 64 || H == 128); }
+
+}  // namespace dsa
+
+using namespace dsa;
+
+#define DSA_SETUP(dev)                                         \
+  int dev = 0;                                                 \
+  if (!current_device(&dev)) return DSA_ERR_CUDA;              \
+  if (!ensure_device(dev)) return DSA_ERR_CUDA;
+
+extern "C" {
+
+dsa_status_t dsa_indexer_scores(const dsa_shape_t* shape, const void* q_idx, const float* q_scale, const void* k_idx,
+                                const float* k_scale, const float* w, const int32_t* ctx_len, const int32_t* q_pos0,
+                                float* scores, int64_t ld_scores, void* stream) {
+  dsa_status_t st = check_shape(shape);
+  if (st != DSA_OK) return st;
+  st = check_indexer_inputs(shape, q_idx, q_scale, k_idx, k_scale, w, ctx_len, q_pos0);
+  if (st != DSA_OK) return st;
+  if (!scores || ld_scores < shape->s_max || (ld_scores & 3) != 0 || !aligned16(scores)) return DSA_ERR_INVALID_ARG;
+  DSA_SETUP(dev);
+  return run_indexer(shape, dev, static_cast<cudaStream_t>(stream), shape->batch, shape->n_q, 0, q_idx, q_scale,
+                     k_idx, k_scale, w, ctx_len, q_pos0, scores, ld_scores);
+}
+
+dsa_status_t dsa_topk(const dsa_shape_t* shape, const float* scores, int64_t ld_scores, const int32_t* ctx_len,
+                      const int32_t* q_pos0, int32_t* idx, void* workspace, size_t workspace_bytes, void* stream) {
+  dsa_status_t st = check_shape(shape);
+  if (st != DSA_OK) return st;
+  if (!scores || !ctx_len || !q_pos0 || !idx) return DSA_ERR_INVALID_ARG;
+  if (ld_scores < shape->s_max || (ld_scores & 3) != 0 || !aligned16(scores)) return DSA_ERR_INVALID_ARG;
+  const size_t need = topk_workspace_bytes(shape->batch, shape->n_q, shape->s_max, shape->topk);
+  if (workspace_bytes < need || (need > 0 && workspace == nullptr)) return DSA_ERR_WORKSPACE;
+  DSA_SETUP(dev);
+  return run_topk(shape, dev, static_cast<cudaStream_t>(stream), shape->batch, shape->n_q, 0, scores, ld_scores,
+                  ctx_len, q_pos0, idx, workspace, workspace_bytes);
+}
+
+dsa_status_t dsa_sparse_mla_attn(const dsa_shape_t* shape, const void* q, const void* kv, const void* v,
+                                 const int32_t* idx, const int32_t* ctx_len, void* out, float* lse, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  dsa_status_t st = check_shape(shape);
+  if (st != DSA_OK) return st;
+  st = check_attn_inputs(shape, q, kv, v, idx, ctx_len, out);
+  if (st != DSA_OK) return st;
+  const size_t need = attn_workspace_bytes(shape->batch, shape->n_q, shape->heads, shape->d_qk, shape->d_v,
+                                           shape->kv_heads, shape->topk, shape->attn_dtype);
+  if (workspace_bytes < need || (need > 0 && workspace == nullptr)) return DSA_ERR_WORKSPACE;
+  DSA_SETUP(dev);
+  return run_attn(shape, dev, static_cast<cudaStream_t>(stream), shape->batch, shape->n_q, q, kv, v, idx, ctx_len,
+                  out, lse, workspace, workspace_bytes);
+}
+
+dsa_status_t dsa_hadamard_quant_fp8(const void* x, int32_t x_dtype, int64_t rows, int32_t dim, uint8_t* x_fp8,
+                                    float* scale, void* stream) {
+  if (rows < 0 || dim <= 0) return DSA_ERR_INVALID_ARG;
+  if (rows > 0 && (!x || !x_fp8 || !scale)) return DSA_ERR_INVALID_ARG;
+  if (x_dtype != DSA_BF16 && x_dtype != DSA_F32) return DSA_ERR_INVALID_ARG;
+  if (dim != 128) return DSA_ERR_UNSUPPORTED;
+  if (((reinterpret_cast<uintptr_t>(x_fp8) & 3u) != 0) || ((reinterpret_cast<uintptr_t>(x) & 7u) != 0))
+    return DSA_ERR_INVALID_ARG;
+  DSA_SETUP(dev);
+  (void)dev;
+  return hadamard_quant(x, x_dtype, rows, dim, x_fp8, scale, static_cast<cudaStream_t>(stream));
+}
+
+size_t dsa_workspace_bytes(const dsa_shape_t* shape, int32_t which) {
+  if (check_shape(shape) != DSA_OK) return 0;
+  switch (which) {
+    case DSA_WS_TOPK:
+      return topk_workspace_bytes(shape->batch, shape->n_q, shape->s_max, shape->topk);
+    case DSA_WS_ATTN:
+      return attn_workspace_bytes(shape->batch, shape->n_q, shape->heads, shape->d_qk, shape->d_v, shape->kv_heads,
+                                  shape->topk, shape->attn_dtype);
+    case DSA_WS_FORWARD:
+      return forward_layout(shape).total;
+    case DSA_WS_FORWARD_HOST:
+      return forward_layout(shape).total_host;
+    default:
+      return 0;
+  }
+}
+
+static dsa_status_t forward_impl(const dsa_shape_t* s, int dev, cudaStream_t st, const void* q_idx,
+                                 const float* q_scale, const void* k_idx, const float* k_scale, const float* w,
+                                 const void* q, const void* kv, const void* v, const int32_t* ctx_len,
+                                 const int32_t* q_pos0, void* out, float* lse, int32_t* idx_out, uint8_t* ws,
+                                 const FwdLayout& L) {
+  const int B = s->batch, n_q = s->n_q;
+  if (B == 0 || n_q == 0) return DSA_OK;
+  dsa_status_t rc;
+  // FP8 indexer: rotate + quantise this step's queries
+  const void* qi = q_idx;
+  const float* qsc = q_scale;
+  dsa_shape_t si = *s;
+  if (s->idx_dtype == DSA_E4M3) {
+    rc = hadamard_quant(q_idx, DSA_BF16, static_cast<int64_t>(B) * n_q * s->idx_heads, s->idx_dim, ws + L.off_q8,
+                        reinterpret_cast<float*>(ws + L.off_qs), st);
+    if (rc != DSA_OK) return rc;
+    qi = ws + L.off_q8;
+    qsc = reinterpret_cast<float*>(ws + L.off_qs);
+  }
+  float* scores = reinterpret_cast<float*>(ws + L.off_scores);
+  const size_t ei = elem_size(s->idx_dtype);
+  const size_t ea = elem_size(s->attn_dtype);
+  if (L.chunk == n_q) {
+    int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + L.off_idx);
+    rc = run_indexer(&si, dev, st, B, n_q, 0, qi, qsc, k_idx, k_scale, w, ctx_len, q_pos0, scores, L.ld);
+    if (rc != DSA_OK) return rc;
+    rc = run_topk(&si, dev, st, B, n_q, 0, scores, L.ld, ctx_len, q_pos0, idx, ws + L.off_topk, L.topk_bytes);
+    if (rc != DSA_OK) return rc;
+    return run_attn(&si, dev, st, B, n_q, q, kv, v, idx, ctx_len, out, lse, ws + L.off_attn, L.attn_bytes);
+  }
+  // Rounds of `chunk` queries, one sequence at a time (positions shift by t0).
+  for (int b = 0; b < B; ++b) {
+    for (int t0 = 0; t0 < n_q; t0 += L.chunk) {
+      const int c = std::min(L.chunk, n_q - t0);
+      const int64_t row0 = static_cast<int64_t>(b) * n_q + t0;
+      const uint8_t* qi_b = static_cast<const uint8_t*>(qi) + row0 * s->idx_heads * s->idx_dim * ei;
+      const float* qs_b = qsc ? qsc + row0 * s->idx_heads : nullptr;
+      const uint8_t* k_b = static_cast<const uint8_t*>(k_idx) + static_cast<int64_t>(b) * s->s_max * s->idx_dim * ei;
+      const float* ks_b = k_scale ? k_scale + static_cast<int64_t>(b) * s->s_max : nullptr;
+      const float* w_b = w + row0 * s->idx_heads;
+      int32_t* idx_b = idx_out ? idx_out + row0 * s->topk : reinterpret_cast<int32_t*>(ws + L.off_idx);
+      const uint8_t* q_b = static_cast<const uint8_t*>(q) + row0 * s->heads * s->d_qk * ea;
+      const uint8_t* kv_b =
+          static_cast<const uint8_t*>(kv) + static_cast<int64_t>(b) * s->s_max * s->kv_heads * s->d_qk * ea;
+      const uint8_t* v_b =
+          v ? static_cast<const uint8_t*>(v) + static_cast<int64_t>(b) * s->s_max * s->kv_heads * s->d_v * ea : nullptr;
+      uint8_t* out_b = static_cast<uint8_t*>(out) + row0 * s->heads * s->d_v * ea;
+      float* lse_b = lse ? lse + row0 * s->heads : nullptr;
+      rc = run_indexer(&si, dev, st, 1, c, t0, qi_b, qs_b, k_b, ks_b, w_b, ctx_len + b, q_pos0 + b, scores, L.ld);
+      if (rc != DSA_OK) return rc;
+      rc = run_topk(&si, dev, st, 1, c, t0, scores, L.ld, ctx_len + b, q_pos0 + b, idx_b, ws + L.off_topk,
+                    L.topk_bytes);
+      if (rc != DSA_OK) return rc;
+      rc = run_attn(&si, dev, st, 1, c, q_b, kv_b, v_b, idx_b, ctx_len + b, out_b, lse_b, ws + L.off_attn,
+                    L.attn_bytes);
+      if (rc != DSA_OK) return rc;
+    }
+  }
+  return DSA_OK;
+}
+
+static dsa_status_t check_forward(const dsa_shape_t* shape, const void* q_idx, const float* q_scale,
+                                  const void* k_idx, const float* k_scale, const float* w, const void* q,
+                                  const void* kv, const void* v, const int32_t* ctx_len, const int32_t* q_pos0,
+                                  const void* out, bool on_host) {
+  dsa_status_t st = check_shape(shape);
+  if (st != DSA_OK) return st;
+  if (shape->idx_dtype == DSA_E4M3) {
+    if (q_scale != nullptr || !k_scale || !q_idx || !k_idx || !w || !ctx_len || !q_pos0) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(k_idx) || (!on_host && !aligned16(q_idx))) return DSA_ERR_INVALID_ARG;
+    if (!indexer_tc_supported(shape->idx_heads, shape->idx_dim)) return DSA_ERR_UNSUPPORTED;
+  } else if (!on_host) {
+    st = check_indexer_inputs(shape, q_idx, q_scale, k_idx, k_scale, w, ctx_len, q_pos0);
+    if (st != DSA_OK) return st;
+  } else {
+    if (!q_idx || !k_idx || !w || !ctx_len || !q_pos0) return DSA_ERR_INVALID_ARG;
+  }
+  if (!q || !kv || !out) return DSA_ERR_INVALID_ARG;
+  if (!on_host) {
+    st = check_attn_inputs(shape, q, kv, v, /*idx*/ q, ctx_len, out);
+    if (st != DSA_OK) return st;
+  }
+  return DSA_OK;
+}
+
+dsa_status_t dsa_forward(const dsa_shape_t* shape, const void* q_idx, const float* q_scale, const void* k_idx,
+                         const float* k_scale, const float* w, const void* q, const void* kv, const void* v,
+                         const int32_t* ctx_len, const int32_t* q_pos0, void* out, float* lse, int32_t* idx_out,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  dsa_status_t st = check_forward(shape, q_idx, q_scale, k_idx, k_scale, w, q, kv, v, ctx_len, q_pos0, out, false);
+  if (st != DSA_OK) return st;
+  const FwdLayout L = forward_layout(shape);
+  if (workspace == nullptr || workspace_bytes < L.total || !aligned16(workspace)) return DSA_ERR_WORKSPACE;
+  DSA_SETUP(dev);
+  return forward_impl(shape, dev, static_cast<cudaStream_t>(stream), q_idx, q_scale, k_idx, k_scale, w, q, kv, v,
+                      ctx_len, q_pos0, out, lse, idx_out, static_cast<uint8_t*>(workspace), L);
+}
+
+dsa_status_t dsa_forward_host(const dsa_shape_t* shape, const void* h_q_idx, const float* h_w, const void* h_q,
+                              const int32_t* h_ctx_len, const int32_t* h_q_pos0, const void* k_idx,
+                              const float* k_scale, const void* kv, const void* v, void* h_out, float* h_lse,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  dsa_status_t st = check_forward(shape, h_q_idx, nullptr, k_idx, k_scale, h_w, h_q, kv, v, h_ctx_len, h_q_pos0,
+                                  h_out, true);
+  if (st != DSA_OK) return st;
+  const FwdLayout L = forward_layout(shape);
+  if (workspace == nullptr || workspace_bytes < L.total_host || !aligned16(workspace)) return DSA_ERR_WORKSPACE;
+  DSA_SETUP(dev);
+  const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int B = shape->batch, n_q = shape->n_q;
+  const size_t ai = elem_size(shape->idx_dtype == DSA_E4M3 ? DSA_BF16 : shape->idx_dtype);
+  const size_t aa = elem_size(shape->attn_dtype);
+  const size_t n_qidx = static_cast<size_t>(B) * n_q * shape->idx_heads * shape->idx_dim * ai;
+  const size_t n_w = static_cast<size_t>(B) * n_q * shape->idx_heads * 4;
+  const size_t n_q_b = static_cast<size_t>(B) * n_q * shape->heads * shape->d_qk * aa;
+  const size_t n_out = static_cast<size_t>(B) * n_q * shape->heads * shape->d_v * aa;
+  const size_t n_lse = static_cast<size_t>(B) * n_q * shape->heads * 4;
+  if (cudaMemcpyAsync(ws + L.off_h_qidx, h_q_idx, n_qidx, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+      cudaMemcpyAsync(ws + L.off_h_w, h_w, n_w, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+      cudaMemcpyAsync(ws + L.off_h_q, h_q, n_q_b, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
+      cudaMemcpyAsync(ws + L.off_h_ctx, h_ctx_len, static_cast<size_t>(B) * 4, cudaMemcpyHostToDevice, cs) !=
+          cudaSuccess ||
+      cudaMemcpyAsync(ws + L.off_h_pos, h_q_pos0, static_cast<size_t>(B) * 4, cudaMemcpyHostToDevice, cs) !=
+          cudaSuccess)
+    return DSA_ERR_CUDA;
+  dsa_shape_t s2 = *shape;
+  st = forward_impl(&s2, dev, cs, ws + L.off_h_qidx, nullptr, k_idx, k_scale, reinterpret_cast<float*>(ws + L.off_h_w),
+                    ws + L.off_h_q, kv, v, reinterpret_cast<int32_t*>(ws + L.off_h_ctx),
+                    reinterpret_cast<int32_t*>(ws + L.off_h_pos), ws + L.off_h_out,
+                    h_lse ? reinterpret_cast<float*>(ws + L.off_h_lse) : nullptr, nullptr, ws, L);
+  if (st != DSA_OK) return st;
+  if (cudaMemcpyAsync(h_out, ws + L.off_h_out, n_out, cudaMemcpyDeviceToHost, cs) != cudaSuccess) return DSA_ERR_CUDA;
+  if (h_lse && cudaMemcpyAsync(h_lse, ws + L.off_h_lse, n_lse, cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  return cudaStreamSynchronize(cs) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+dsa_status_t dsa_get_error(int32_t clear, uint32_t* detail) {
+  DSA_SETUP(dev);
+  uint32_t word[4] = {0, 0, 0, 0};
+  if (cudaDeviceSynchronize() != cudaSuccess) return DSA_ERR_CUDA;
+  if (cudaMemcpy(word, g_err_ptr[dev], sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return DSA_ERR_CUDA;
+  if (clear) {
+    const uint32_t zero[4] = {0, 0, 0, 0};
+    if (cudaMemcpy(g_err_ptr[dev], zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return DSA_ERR_CUDA;
+  }
+  if (detail) *detail = word[0];
+  if (word[0] & kErrTimeout) return DSA_ERR_TIMEOUT;
+  if (word[0] & kErrBadIndex) return DSA_ERR_BAD_INDEX;
+  return DSA_OK;
+}
+
+const char* dsa_status_string(dsa_status_t status) {
+  switch (status) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID_ARG: return "invalid argument";
+    case DSA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case DSA_ERR_WORKSPACE: return "workspace missing or too small";
+    case DSA_ERR_CUDA: return "CUDA error";
+    case DSA_ERR_TIMEOUT: return "a bounded wait inside a kernel expired";
+    case DSA_ERR_BAD_INDEX: return "attention index out of range (skipped)";
+  }
+  return "unknown status";
+}
+
+int32_t dsa_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,411 @@
+// Lightning-indexer scores on the 5th-generation tensor cores.
+//
+// DeepSeek-V3.2 model doc (Transformers), section "DeepSeek Sparse Attention
+// (DSA)", item 1: an index score of each query against all previous keys of
+// the indexer's single-head key cache (width index_head_dim = 128), combined
+// over index_n_heads = 64 heads.  Per (query t, key s):
+//     I[t,s] = sum_h w[t,h] * ReLU(scale * <q[t,h,:], k[s,:]>)   (s <= pos(t))
+// The FP8 instance (same item: the reference indexer runs in FP8 after a
+// Hadamard rotation) multiplies the e4m3 codes and folds the per-row scales
+// into the epilogue: I = k_scale[s] * sum_h (w * q_scale)[t,h] * ReLU(dot).
+//
+// Design (sm_100a):
+//   * One tile = 128 keys (MMA M) x N = QG queries * H_I heads (MMA N), K = 128.
+//     Keys on M means each epilogue thread owns one key's TMEM lane and does
+//     the ReLU-weighted head reduction from its own registers.
+//   * Warp-specialised persistent CTA: warp 0 issues TMA loads of key tiles
+//     (a ring of shared-memory stages) and of the query block, warp 1 issues
+//     tcgen05.mma into a ring of TMEM accumulators, the remaining warps run
+//     the epilogue (tcgen05.ld, ReLU, weighted head sum, causal mask, store).
+//   * Decode (one query per sequence) is HBM-bound on the key cache, so each
+//     CTA takes a contiguous run of key tiles (query block loaded once per
+//     sequence it touches).  Prefill is tensor-bound; its units are chunks of
+//     key tiles handed out in a scrambled order so the causal triangle
+//     balances across CTAs.  Key tiles wholly above the diagonal of a query
+//     block are not computed; the epilogue only writes -inf there.
+//   * Every mbarrier wait is bounded; on expiry the kernel records a timeout
+//     in the error word, drains its copies and MMAs, frees TMEM and returns.
+#include "dsa_common.cuh"
+#include "dsa_internal.h"
+
+namespace dsa {
+namespace {
+
+constexpr int kTileKeys = 128;  // MMA M
+constexpr int kIdxDim = 128;    // D_I
+
+template <bool kFP8, int kQG, int kHI, int kEpiWarps, int kStages, int kQBufs>
+struct IdxCfg {
+  static constexpr int N = kQG * kHI;
+  static constexpr int kElem = kFP8 ? 1 : 2;
+  static constexpr int kRowBytes = kIdxDim * kElem;          // 256 (bf16) or 128 (fp8)
+  static constexpr int kKBlocks = kRowBytes / 128;           // 128-byte swizzle atoms along K
+  static constexpr int kKTile = kTileKeys * kRowBytes;       // bytes of one key tile
+  static constexpr int kQTile = N * kRowBytes;               // bytes of one query block
+  static constexpr int kNumMma = kRowBytes / 32;             // each MMA consumes 32 bytes of K
+  static constexpr int kNumAcc = (N <= 64) ? 4 : (512 / N);  // TMEM accumulators
+  static constexpr int kTmemCols = (kNumAcc * N <= 256) ? 256 : 512;
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
+  static constexpr int kEpiThreads = 32 * kEpiWarps;
+  // shared memory offsets (from a 1024-aligned base)
+  static constexpr int kOffK = 0;
+  static constexpr int kOffQ = kOffK + kStages * kKTile;
+  static constexpr int kOffW = kOffQ + kQBufs * kQTile;
+  static constexpr int kOffBar = kOffW + 2 * kQG * kHI * 4;  // two weight buffers
+  static constexpr int kNumBars = 2 * kStages + 2 * kQBufs + 2 * kNumAcc + 1;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+  static_assert(N % 16 == 0 && N >= 16 && N <= 256, "MMA N");
+  static_assert(kHI % 16 == 0, "heads per query");
+  static_assert(kEpiWarps == 4 || (kEpiWarps == 8 && kQG % 2 == 0), "epilogue split");
+  static_assert(kKTile % 1024 == 0 && kQTile % 1024 == 0, "swizzle atom alignment");
+};
+
+struct Unit {
+  int b, t0, nq, L, p0, kt0, kt_comp, kt_end;
+};
+
+struct Sched {
+  int B, n_q, s_max, G, NC, TPC, nunits, contiguous;
+  int per_cta, scramble;
+  int t_off;  // position offset of query 0 of this call within its sequence
+};
+
+__device__ __forceinline__ int unit_id(const Sched& S, int cta, int i) {
+  if (S.contiguous) return cta * S.per_cta + i;  // caller bounds-checks
+  const int u = cta + i * static_cast<int>(gridDim.x);
+  return static_cast<int>((static_cast<int64_t>(u) * S.scramble) % S.nunits);
+}
+
+__device__ __forceinline__ int unit_count(const Sched& S, int cta) {
+  if (S.contiguous) {
+    const int beg = cta * S.per_cta;
+    return max(0, min(S.per_cta, S.nunits - beg));
+  }
+  return (S.nunits - cta + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
+}
+
+template <int kQG>
+__device__ __forceinline__ Unit get_unit(const Sched& S, int u, const int32_t* __restrict__ ctx_len,
+                                         const int32_t* __restrict__ q_pos0) {
+  Unit r;
+  const int c = u % S.NC;
+  const int bg = u / S.NC;
+  const int g = bg % S.G;
+  r.b = bg / S.G;
+  r.L = min(max(__ldg(ctx_len + r.b), 0), S.s_max);
+  r.p0 = max(__ldg(q_pos0 + r.b), 0) + S.t_off;
+  r.t0 = g * kQG;
+  r.nq = min(kQG, S.n_q - r.t0);
+  const int pmax = min(r.p0 + r.t0 + r.nq - 1, r.L - 1);
+  const int ntiles = (r.L + kTileKeys - 1) / kTileKeys;
+  r.kt0 = c * S.TPC;
+  r.kt_end = min(r.kt0 + S.TPC, ntiles);
+  r.kt_comp = min(r.kt_end, pmax >= 0 ? pmax / kTileKeys + 1 : 0);
+  if (r.kt_comp < r.kt0) r.kt_comp = r.kt0;
+  return r;
+}
+
+template <bool kFP8, int kQG, int kHI, int kEpiWarps, int kStages, int kQBufs>
+__global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQBufs>::kThreads, 1)
+    indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
+                      const float* __restrict__ w, const float* __restrict__ q_scale,
+                      const float* __restrict__ k_scale, const int32_t* __restrict__ ctx_len,
+                      const int32_t* __restrict__ q_pos0, float* __restrict__ scores, int64_t ld,
+                      float idx_scale, Sched S, uint32_t* err) {
+  using C = IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQBufs>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_addr(smem);
+  float* w_s = reinterpret_cast<float*>(smem + C::kOffW);
+  const uint32_t bar0 = sbase + C::kOffBar;
+  auto k_full = [&](int i) { return bar0 + 8u * i; };
+  auto k_empty = [&](int i) { return bar0 + 8u * (kStages + i); };
+  auto q_full = [&](int i) { return bar0 + 8u * (2 * kStages + i); };
+  auto q_empty = [&](int i) { return bar0 + 8u * (2 * kStages + kQBufs + i); };
+  auto acc_full = [&](int i) { return bar0 + 8u * (2 * kStages + 2 * kQBufs + i); };
+  auto acc_empty = [&](int i) { return bar0 + 8u * (2 * kStages + 2 * kQBufs + C::kNumAcc + i); };
+  const uint32_t mma_done = bar0 + 8u * (C::kNumBars - 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = lane_id();
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) { mbar_init(k_full(i), 1); mbar_init(k_empty(i), 1); }
+    for (int i = 0; i < kQBufs; ++i) { mbar_init(q_full(i), 1); mbar_init(q_empty(i), 1); }
+    for (int i = 0; i < C::kNumAcc; ++i) { mbar_init(acc_full(i), 1); mbar_init(acc_empty(i), C::kEpiThreads); }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&tmap_k);
+    tma_prefetch_map(&tmap_q);
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int cta = blockIdx.x;
+  const int nmine = unit_count(S, cta);
+
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer --
+    if (lane == 0) {
+      int st = 0, qb = 0;
+      uint32_t kph = 0, qph = 0;
+      int last_bg = -1;
+      uint32_t issued_k[kStages];
+      uint32_t issued_q[kQBufs];
+      for (int i = 0; i < kStages; ++i) issued_k[i] = 0;
+      for (int i = 0; i < kQBufs; ++i) issued_q[i] = 0;
+      for (int i = 0; i < nmine; ++i) {
+        const Unit U = get_unit<kQG>(S, unit_id(S, cta, i), ctx_len, q_pos0);
+        if (U.kt_comp <= U.kt0) continue;
+        const int bg = U.b * S.G + U.t0 / kQG;
+        if (bg != last_bg) {
+          if (last_bg >= 0) { if (++qb == kQBufs) { qb = 0; qph ^= 1; } }
+          if (!mbar_wait(q_empty(qb), qph ^ 1, abort_flag, err)) break;
+          mbar_arrive_expect_tx(q_full(qb), C::kQTile);
+          const int qrow = (U.b * S.n_q + U.t0) * kHI;
+          const uint32_t qdst = sbase + C::kOffQ + qb * C::kQTile;
+#pragma unroll
+          for (int kb = 0; kb < C::kKBlocks; ++kb)
+            tma_load_2d(qdst + kb * C::N * 128, &tmap_q, q_full(qb), kb * (128 / C::kElem), qrow);
+          issued_q[qb]++;
+          last_bg = bg;
+        }
+        bool ok = true;
+        for (int kt = U.kt0; kt < U.kt_comp; ++kt) {
+          if (!mbar_wait(k_empty(st), kph ^ 1, abort_flag, err)) { ok = false; break; }
+          mbar_arrive_expect_tx(k_full(st), C::kKTile);
+          const int krow = U.b * S.s_max + kt * kTileKeys;
+          const uint32_t kdst = sbase + C::kOffK + st * C::kKTile;
+#pragma unroll
+          for (int kb = 0; kb < C::kKBlocks; ++kb)
+            tma_load_2d(kdst + kb * kTileKeys * 128, &tmap_k, k_full(st), kb * (128 / C::kElem), krow);
+          issued_k[st]++;
+          if (++st == kStages) { st = 0; kph ^= 1; }
+        }
+        if (!ok) break;
+      }
+      // Drain: every copy this thread issued has landed before the CTA exits.
+      volatile int never = 0;
+      for (int i = 0; i < kStages; ++i)
+        if (issued_k[i]) mbar_wait(k_full(i), (issued_k[i] - 1) & 1, &never, err);
+      for (int i = 0; i < kQBufs; ++i)
+        if (issued_q[i]) mbar_wait(q_full(i), (issued_q[i] - 1) & 1, &never, err);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      constexpr uint32_t idesc = kFP8 ? idesc_e4m3_f32(kTileKeys, C::N) : idesc_bf16_f32(kTileKeys, C::N);
+      int st = 0, qb = 0, ab = 0;
+      uint32_t kph = 0, qph = 0, aph = 0;
+      int last_bg = -1;
+      for (int i = 0; i < nmine; ++i) {
+        const Unit U = get_unit<kQG>(S, unit_id(S, cta, i), ctx_len, q_pos0);
+        if (U.kt_comp <= U.kt0) continue;
+        const int bg = U.b * S.G + U.t0 / kQG;
+        if (bg != last_bg) {
+          if (last_bg >= 0) {
+            tc_commit(q_empty(qb));
+            if (++qb == kQBufs) { qb = 0; qph ^= 1; }
+          }
+          if (!mbar_wait(q_full(qb), qph, abort_flag, err)) break;
+          last_bg = bg;
+        }
+        const uint32_t qaddr = sbase + C::kOffQ + qb * C::kQTile;
+        bool ok = true;
+        for (int kt = U.kt0; kt < U.kt_comp; ++kt) {
+          if (!mbar_wait(acc_empty(ab), aph ^ 1, abort_flag, err)) { ok = false; break; }
+          if (!mbar_wait(k_full(st), kph, abort_flag, err)) { ok = false; break; }
+          tc_fence_after_sync();
+          const uint32_t kaddr = sbase + C::kOffK + st * C::kKTile;
+          const uint32_t d = tmem_base + static_cast<uint32_t>(ab * C::N);
+#pragma unroll
+          for (int kk = 0; kk < C::kNumMma; ++kk) {
+            const int kb = (kk * 32) / 128, within = (kk * 32) % 128;
+            const uint64_t ad = sdesc_kmajor_sw128(kaddr + kb * kTileKeys * 128 + within);
+            const uint64_t bd = sdesc_kmajor_sw128(qaddr + kb * C::N * 128 + within);
+            if (kFP8) tc_mma_f8(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
+            else tc_mma_f16(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(k_empty(st));
+          tc_commit(acc_full(ab));
+          if (++st == kStages) { st = 0; kph ^= 1; }
+          if (++ab == C::kNumAcc) { ab = 0; aph ^= 1; }
+        }
+        if (!ok) break;
+      }
+      // All MMAs issued above are complete before TMEM is released.
+      tc_commit(mma_done);
+      volatile int never = 0;
+      mbar_wait(mma_done, 0, &never, err);
+    }
+  } else {
+    // --------------------------------------------------- epilogue --
+    const int e = warp - 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;  // key within the tile == TMEM lane
+    const int jbeg = (kEpiWarps == 8) ? (e >> 2) * (kQG / 2) : 0;
+    const int jend = (kEpiWarps == 8) ? jbeg + kQG / 2 : kQG;
+    const int tid_e = threadIdx.x - 64;
+    int ab = 0, wb = 0;
+    uint32_t aph = 0;
+    int last_bg = -1;
+    for (int i = 0; i < nmine; ++i) {
+      const Unit U = get_unit<kQG>(S, unit_id(S, cta, i), ctx_len, q_pos0);
+      if (U.kt_end <= U.kt0) continue;
+      if (U.kt_comp > U.kt0) {
+        const int bg = U.b * S.G + U.t0 / kQG;
+        if (bg != last_bg) {
+          // head weights of this query block, with the score scale (and the
+          // per-(query, head) FP8 scale) folded in; double-buffered so the
+          // barrier only has to order writers against the previous readers
+          wb ^= 1;
+          named_bar_sync(1, C::kEpiThreads);
+          float* wd = w_s + wb * kQG * kHI;
+          for (int k = tid_e; k < kQG * kHI; k += C::kEpiThreads) {
+            const int j = k / kHI, h = k % kHI;
+            float v = 0.f;
+            if (j < U.nq) {
+              const int64_t o = (static_cast<int64_t>(U.b) * S.n_q + U.t0 + j) * kHI + h;
+              v = __ldg(w + o) * idx_scale;
+              if (kFP8) v *= __ldg(q_scale + o);
+            }
+            wd[k] = v;
+          }
+          named_bar_sync(1, C::kEpiThreads);
+          last_bg = bg;
+        }
+      }
+      const float* wd = w_s + wb * kQG * kHI;
+      bool ok = true;
+      for (int kt = U.kt0; kt < U.kt_comp; ++kt) {
+        if (!mbar_wait_warp(acc_full(ab), aph, abort_flag, err)) { ok = false; break; }
+        tc_fence_after_sync();
+        const int s = kt * kTileKeys + row;
+        float ks = 1.f;
+        if (kFP8 && s < U.L) ks = __ldg(k_scale + static_cast<int64_t>(U.b) * S.s_max + s);
+        const uint32_t tl = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(ab * C::N);
+#pragma unroll 1
+        for (int j = jbeg; j < jend; ++j) {
+          float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+          for (int c = 0; c < kHI; c += 16) {
+            float v[16];
+            tmem_ld16(tl + j * kHI + c, v);
+#pragma unroll
+            for (int x = 0; x < 16; x += 2) {
+              acc0 = fmaf(wd[j * kHI + c + x], fmaxf(v[x], 0.f), acc0);
+              acc1 = fmaf(wd[j * kHI + c + x + 1], fmaxf(v[x + 1], 0.f), acc1);
+            }
+          }
+          if (j < U.nq && s < U.L) {
+            const int p = U.p0 + U.t0 + j;
+            scores[(static_cast<int64_t>(U.b) * S.n_q + U.t0 + j) * ld + s] = (s <= p) ? (acc0 + acc1) * ks : -INFINITY;
+          }
+        }
+        tc_fence_before_sync();
+        mbar_arrive(acc_empty(ab));
+        if (++ab == C::kNumAcc) { ab = 0; aph ^= 1; }
+      }
+      if (!ok) break;
+      // key tiles entirely after every query of the block: -inf only
+      for (int kt = U.kt_comp; kt < U.kt_end; ++kt) {
+        const int s = kt * kTileKeys + row;
+        if (s < U.L)
+          for (int j = jbeg; j < min(jend, U.nq); ++j)
+            scores[(static_cast<int64_t>(U.b) * S.n_q + U.t0 + j) * ld + s] = -INFINITY;
+      }
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+template <bool kFP8, int kQG, int kHI, int kEpiWarps, int kStages, int kQBufs>
+dsa_status_t launch_indexer_tc(const IndexerArgs& a) {
+  using C = IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQBufs>;
+  auto kern = indexer_tc_kernel<kFP8, kQG, kHI, kEpiWarps, kStages, kQBufs>;
+  const int dev = a.device;
+  const int num_sms = device_sm_count(dev);
+
+  CUtensorMap tmk, tmq;
+  const CUtensorMapDataType dt = kFP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const uint32_t box_inner = 128 / C::kElem;
+  if (!make_tmap_2d(&tmk, a.k_idx, dt, C::kElem, kIdxDim, static_cast<uint64_t>(a.B) * a.s_max, box_inner,
+                    kTileKeys))
+    return DSA_ERR_CUDA;
+  if (!make_tmap_2d(&tmq, a.q_idx, dt, C::kElem, kIdxDim, static_cast<uint64_t>(a.B) * a.n_q * kHI, box_inner,
+                    C::N))
+    return DSA_ERR_CUDA;
+
+  Sched S;
+  S.B = a.B;
+  S.n_q = a.n_q;
+  S.s_max = a.s_max;
+  S.t_off = a.t_off;
+  S.G = (a.n_q + kQG - 1) / kQG;
+  const int tiles_per_row = (a.s_max + kTileKeys - 1) / kTileKeys;
+  const bool decode_like = (kQG == 1);
+  S.TPC = decode_like ? 1 : min(16, tiles_per_row);
+  S.NC = (tiles_per_row + S.TPC - 1) / S.TPC;
+  const int64_t nunits64 = static_cast<int64_t>(a.B) * S.G * S.NC;
+  if (nunits64 > INT32_MAX / 2) return DSA_ERR_UNSUPPORTED;
+  S.nunits = static_cast<int>(nunits64);
+  const int grid = static_cast<int>(std::min<int64_t>(S.nunits, num_sms));
+  S.contiguous = decode_like ? 1 : 0;
+  S.per_cta = (S.nunits + grid - 1) / grid;
+  // multiplier coprime to nunits for the scrambled order
+  int64_t mult = 40503;
+  while (std::gcd(mult, static_cast<int64_t>(S.nunits)) != 1) mult += 2;
+  S.scramble = static_cast<int>(mult % S.nunits == 0 ? 1 : mult % S.nunits);
+
+  static bool attr_done[64] = {};
+  if (dev < 64 && !attr_done[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    attr_done[dev] = true;
+  }
+  kern<<<grid, C::kThreads, C::kSmemBytes, a.stream>>>(tmk, tmq, a.w, a.q_scale, a.k_scale, a.ctx_len, a.q_pos0,
+                                                         a.scores, a.ld, a.idx_scale, S, a.err);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+}  // namespace
+
+dsa_status_t indexer_tc(const IndexerArgs& a) {
+  // decode (n_q == 1): one query per tile; prefill: a block of queries filling N.
+  const bool fp8 = (a.dtype == DSA_E4M3);
+  if (a.D != kIdxDim) return DSA_ERR_UNSUPPORTED;
+  const bool one = (a.n_q == 1);
+#define DSA_IDX_CASE(HI, QGP)                                                              \
+  if (a.H == HI) {                                                                         \
+    if (one) return fp8 ? launch_indexer_tc<true, 1, HI, 4, 12, 2>(a)                       \
+                        : launch_indexer_tc<false, 1, HI, 4, 5, 2>(a);                     \
+    return fp8 ? launch_indexer_tc<true, QGP, HI, ((QGP) % 2 == 0 ? 8 : 4), 6, 1>(a)       \
+               : launch_indexer_tc<false, QGP, HI, ((QGP) % 2 == 0 ? 8 : 4), 4, 1>(a);     \
+  }
+  DSA_IDX_CASE(64, 4)
+  DSA_IDX_CASE(32, 8)
+  DSA_IDX_CASE(16, 16)
+  DSA_IDX_CASE(128, 2)
+#undef DSA_IDX_CASE
+  return DSA_ERR_UNSUPPORTED;
+}
+
+}  // namespace dsa
