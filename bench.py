@@ -340,10 +340,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode128k", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling runs)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
-    wl = workloads.get(args.workload)
+    wl = workloads.get(args.workload, **({"batch": args.batch} if args.batch else {}))
     if args.impl == "reference":
         line = run_reference(args, wl)
         if line is not None:

@@ -66,31 +66,55 @@ struct Unit {
 };
 
 struct Sched {
-  int B, n_q, s_max, G, NC, TPC, nunits, contiguous;
-  int per_cta, scramble;
-  int t_off;  // position offset of query 0 of this call within its sequence
+  int B, n_q, s_max, G, tpr;  // tpr: key tiles per sequence row
+  int contiguous;             // 1: each CTA walks one contiguous run of tiles
+  int per_cta;                // contiguous: tiles per CTA
+  int TPC, NC, nunits, scramble;  // scrambled: units of TPC tiles
+  int t_off;                  // position offset of query 0 of this call within its sequence
 };
 
-__device__ __forceinline__ int unit_id(const Sched& S, int cta, int i) {
-  if (S.contiguous) return cta * S.per_cta + i;  // caller bounds-checks
-  const int u = cta + i * static_cast<int>(gridDim.x);
-  return static_cast<int>((static_cast<int64_t>(u) * S.scramble) % S.nunits);
-}
+// Walks the work of one CTA as units (one query block, a run of key tiles).
+// Contiguous mode cuts the CTA's run of tiles at query-block boundaries (one
+// division per unit); scrambled mode visits chunks of TPC tiles in a
+// multiplicative-hash order.  Every role of the CTA walks the same sequence.
+struct UnitIter {
+  int i, end;
+};
 
-__device__ __forceinline__ int unit_count(const Sched& S, int cta) {
+__device__ __forceinline__ UnitIter iter_begin(const Sched& S, int cta) {
+  UnitIter it;
   if (S.contiguous) {
-    const int beg = cta * S.per_cta;
-    return max(0, min(S.per_cta, S.nunits - beg));
+    const int64_t total = static_cast<int64_t>(S.B) * S.G * S.tpr;
+    const int64_t beg = static_cast<int64_t>(cta) * S.per_cta;
+    const int64_t end = beg + S.per_cta;
+    it.i = static_cast<int>(beg < total ? beg : total);
+    it.end = static_cast<int>(end < total ? end : total);
+  } else {
+    it.i = 0;
+    it.end = (S.nunits - cta + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
   }
-  return (S.nunits - cta + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
+  return it;
 }
 
 template <int kQG>
-__device__ __forceinline__ Unit get_unit(const Sched& S, int u, const int32_t* __restrict__ ctx_len,
-                                         const int32_t* __restrict__ q_pos0) {
-  Unit r;
-  const int c = u % S.NC;
-  const int bg = u / S.NC;
+__device__ __forceinline__ bool iter_next(const Sched& S, UnitIter& it, int cta, Unit& r,
+                                          const int32_t* __restrict__ ctx_len, const int32_t* __restrict__ q_pos0) {
+  if (it.i >= it.end) return false;
+  int bg, ka, kb;
+  if (S.contiguous) {
+    bg = it.i / S.tpr;
+    ka = it.i - bg * S.tpr;
+    kb = min(S.tpr, ka + (it.end - it.i));
+    it.i += kb - ka;
+  } else {
+    const int v = cta + it.i * static_cast<int>(gridDim.x);
+    const int u = static_cast<int>((static_cast<int64_t>(v) * S.scramble) % S.nunits);
+    ++it.i;
+    const int c = u % S.NC;
+    bg = u / S.NC;
+    ka = c * S.TPC;
+    kb = min(S.tpr, ka + S.TPC);
+  }
   const int g = bg % S.G;
   r.b = bg / S.G;
   r.L = min(max(__ldg(ctx_len + r.b), 0), S.s_max);
@@ -99,11 +123,11 @@ __device__ __forceinline__ Unit get_unit(const Sched& S, int u, const int32_t* _
   r.nq = min(kQG, S.n_q - r.t0);
   const int pmax = min(r.p0 + r.t0 + r.nq - 1, r.L - 1);
   const int ntiles = (r.L + kTileKeys - 1) / kTileKeys;
-  r.kt0 = c * S.TPC;
-  r.kt_end = min(r.kt0 + S.TPC, ntiles);
+  r.kt0 = ka;
+  r.kt_end = min(kb, ntiles);
   r.kt_comp = min(r.kt_end, pmax >= 0 ? pmax / kTileKeys + 1 : 0);
   if (r.kt_comp < r.kt0) r.kt_comp = r.kt0;
-  return r;
+  return true;
 }
 
 template <bool kFP8, int kQG, int kHI, int kEpiWarps, int kStages, int kQBufs>
@@ -154,7 +178,6 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
   const uint32_t tmem_base = *tmem_slot;
 
   const int cta = blockIdx.x;
-  const int nmine = unit_count(S, cta);
 
   if (warp == 0) {
     // ------------------------------------------------ TMA producer --
@@ -166,8 +189,9 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
       uint32_t issued_q[kQBufs];
       for (int i = 0; i < kStages; ++i) issued_k[i] = 0;
       for (int i = 0; i < kQBufs; ++i) issued_q[i] = 0;
-      for (int i = 0; i < nmine; ++i) {
-        const Unit U = get_unit<kQG>(S, unit_id(S, cta, i), ctx_len, q_pos0);
+      UnitIter it = iter_begin(S, cta);
+      Unit U;
+      while (iter_next<kQG>(S, it, cta, U, ctx_len, q_pos0)) {
         if (U.kt_comp <= U.kt0) continue;
         const int bg = U.b * S.G + U.t0 / kQG;
         if (bg != last_bg) {
@@ -207,11 +231,13 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
     // ------------------------------------------------- MMA issuer --
     if (lane == 0) {
       constexpr uint32_t idesc = kFP8 ? idesc_e4m3_f32(kTileKeys, C::N) : idesc_bf16_f32(kTileKeys, C::N);
+      const uint64_t a_desc0 = sdesc_kmajor_sw128(sbase + C::kOffK);
       int st = 0, qb = 0, ab = 0;
       uint32_t kph = 0, qph = 0, aph = 0;
       int last_bg = -1;
-      for (int i = 0; i < nmine; ++i) {
-        const Unit U = get_unit<kQG>(S, unit_id(S, cta, i), ctx_len, q_pos0);
+      UnitIter it = iter_begin(S, cta);
+      Unit U;
+      while (iter_next<kQG>(S, it, cta, U, ctx_len, q_pos0)) {
         if (U.kt_comp <= U.kt0) continue;
         const int bg = U.b * S.G + U.t0 / kQG;
         if (bg != last_bg) {
@@ -222,21 +248,21 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
           if (!mbar_wait(q_full(qb), qph, abort_flag, err)) break;
           last_bg = bg;
         }
-        const uint32_t qaddr = sbase + C::kOffQ + qb * C::kQTile;
+        const uint64_t bd0 = sdesc_kmajor_sw128(sbase + C::kOffQ + qb * C::kQTile);
         bool ok = true;
         for (int kt = U.kt0; kt < U.kt_comp; ++kt) {
           if (!mbar_wait(acc_empty(ab), aph ^ 1, abort_flag, err)) { ok = false; break; }
           if (!mbar_wait(k_full(st), kph, abort_flag, err)) { ok = false; break; }
           tc_fence_after_sync();
-          const uint32_t kaddr = sbase + C::kOffK + st * C::kKTile;
           const uint32_t d = tmem_base + static_cast<uint32_t>(ab * C::N);
+          const uint64_t ad0 = a_desc0 + static_cast<uint64_t>((st * C::kKTile) >> 4);
 #pragma unroll
           for (int kk = 0; kk < C::kNumMma; ++kk) {
-            const int kb = (kk * 32) / 128, within = (kk * 32) % 128;
-            const uint64_t ad = sdesc_kmajor_sw128(kaddr + kb * kTileKeys * 128 + within);
-            const uint64_t bd = sdesc_kmajor_sw128(qaddr + kb * C::N * 128 + within);
-            if (kFP8) tc_mma_f8(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
-            else tc_mma_f16(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
+            // descriptor start addresses advance in 16-byte units
+            const uint32_t a_off = ((kk * 32) / 128) * kTileKeys * 128 + (kk * 32) % 128;
+            const uint32_t b_off = ((kk * 32) / 128) * C::N * 128 + (kk * 32) % 128;
+            if (kFP8) tc_mma_f8(d, ad0 + (a_off >> 4), bd0 + (b_off >> 4), idesc, kk > 0 ? 1u : 0u);
+            else tc_mma_f16(d, ad0 + (a_off >> 4), bd0 + (b_off >> 4), idesc, kk > 0 ? 1u : 0u);
           }
           tc_commit(k_empty(st));
           tc_commit(acc_full(ab));
@@ -261,8 +287,9 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
     int ab = 0, wb = 0;
     uint32_t aph = 0;
     int last_bg = -1;
-    for (int i = 0; i < nmine; ++i) {
-      const Unit U = get_unit<kQG>(S, unit_id(S, cta, i), ctx_len, q_pos0);
+    UnitIter it = iter_begin(S, cta);
+    Unit U;
+    while (iter_next<kQG>(S, it, cta, U, ctx_len, q_pos0)) {
       if (U.kt_end <= U.kt0) continue;
       if (U.kt_comp > U.kt0) {
         const int bg = U.b * S.G + U.t0 / kQG;
@@ -299,12 +326,14 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
 #pragma unroll 1
         for (int j = jbeg; j < jend; ++j) {
           float acc0 = 0.f, acc1 = 0.f;
+          constexpr int kChunk = (kHI % 32 == 0) ? 32 : 16;
 #pragma unroll
-          for (int c = 0; c < kHI; c += 16) {
-            float v[16];
-            tmem_ld16(tl + j * kHI + c, v);
+          for (int c = 0; c < kHI; c += kChunk) {
+            float v[kChunk];
+            if (kChunk == 32) tmem_ld32(tl + j * kHI + c, v);
+            else tmem_ld16(tl + j * kHI + c, v);
 #pragma unroll
-            for (int x = 0; x < 16; x += 2) {
+            for (int x = 0; x < kChunk; x += 2) {
               acc0 = fmaf(wd[j * kHI + c + x], fmaxf(v[x], 0.f), acc0);
               acc1 = fmaf(wd[j * kHI + c + x + 1], fmaxf(v[x + 1], 0.f), acc1);
             }
@@ -360,16 +389,17 @@ dsa_status_t launch_indexer_tc(const IndexerArgs& a) {
   S.s_max = a.s_max;
   S.t_off = a.t_off;
   S.G = (a.n_q + kQG - 1) / kQG;
-  const int tiles_per_row = (a.s_max + kTileKeys - 1) / kTileKeys;
+  S.tpr = (a.s_max + kTileKeys - 1) / kTileKeys;
+  const int64_t total_tiles = static_cast<int64_t>(a.B) * S.G * S.tpr;
+  if (total_tiles > INT32_MAX / 2) return DSA_ERR_UNSUPPORTED;
   const bool decode_like = (kQG == 1);
-  S.TPC = decode_like ? 1 : min(16, tiles_per_row);
-  S.NC = (tiles_per_row + S.TPC - 1) / S.TPC;
-  const int64_t nunits64 = static_cast<int64_t>(a.B) * S.G * S.NC;
-  if (nunits64 > INT32_MAX / 2) return DSA_ERR_UNSUPPORTED;
-  S.nunits = static_cast<int>(nunits64);
-  const int grid = static_cast<int>(std::min<int64_t>(S.nunits, num_sms));
   S.contiguous = decode_like ? 1 : 0;
-  S.per_cta = (S.nunits + grid - 1) / grid;
+  S.TPC = decode_like ? 1 : std::min(16, S.tpr);
+  S.NC = (S.tpr + S.TPC - 1) / S.TPC;
+  S.nunits = static_cast<int>(static_cast<int64_t>(a.B) * S.G * S.NC);
+  const int64_t work = decode_like ? total_tiles : S.nunits;
+  const int grid = static_cast<int>(std::min<int64_t>(work, num_sms));
+  S.per_cta = static_cast<int>((total_tiles + grid - 1) / grid);
   // multiplier coprime to nunits for the scrambled order
   int64_t mult = 40503;
   while (std::gcd(mult, static_cast<int64_t>(S.nunits)) != 1) mult += 2;

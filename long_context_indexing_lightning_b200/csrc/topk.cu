@@ -2,18 +2,25 @@
 // previous keys (DeepSeek-V3.2 model doc, Transformers, section "DeepSeek
 // Sparse Attention (DSA)", item 2; index_topk defaults to 2048).
 //
-// Radix select on order-preserving 32-bit keys, no sort:
-//   * three histogram passes over the candidate row (digits of 11, 11 and
-//     10 bits, most significant first) in shared memory find the exact key T
-//     of the k-th largest score and how many keys equal to T to keep;
-//   * one ordered compaction pass keeps every key > T and the lowest-indexed
-//     keys == T (ties go to the lower index), emitting indices in ascending
-//     order.  Per-thread segment counts are combined with warp shuffles and a
-//     block prefix sum, so the output is deterministic.
-// One 1024-thread CTA per query row; rows with at most k candidates are
-// written directly.
+// Radix select on order-preserving 32-bit keys, no sort.  One query row is
+// split over a thread-block cluster of C CTAs (C = 1..16); each thread keeps
+// its PER consecutive keys in registers for the whole selection:
+//   * three histogram passes (digits of 11, 11 and 10 bits, most significant
+//     first) into shared memory; the C partial histograms are summed through
+//     distributed shared memory and every CTA finds the same digit of the
+//     k-th largest key, so after three passes all CTAs know the exact key T of
+//     the k-th largest score and how many keys equal to T to keep;
+//   * one ordered compaction: per-thread counts of keys > T and == T, a block
+//     prefix sum (warp shuffles), CTA totals exchanged across the cluster,
+//     then every kept index is written at its final position -- keys > T plus
+//     the lowest-indexed keys == T (ties go to the lower index), ascending.
+// Rows with at most k candidates are written directly.
+#include <cooperative_groups.h>
+
 #include "dsa_common.cuh"
 #include "dsa_internal.h"
+
+namespace cg = cooperative_groups;
 
 namespace dsa {
 namespace {
@@ -21,7 +28,7 @@ namespace {
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 2048;
-constexpr int kSeg = 8;  // consecutive elements per thread in the compaction pass
+constexpr int kMaxCluster = 16;
 
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v) {
   const int lane = lane_id();
@@ -33,8 +40,8 @@ __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v) {
   return v;
 }
 
-// Block-wide exclusive scan of one value per thread; returns the exclusive
-// prefix and writes the block total to *total.  Uses `wsum` (kWarps words).
+// Block-wide exclusive scan of one value per thread; the block total goes to
+// *total.  Uses `wsum` (kWarps + 1 words).
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* wsum, uint32_t* total) {
   const int lane = lane_id(), warp = threadIdx.x >> 5;
   const uint32_t incl = warp_incl_scan(v);
@@ -53,15 +60,21 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* wsum, 
   return res;
 }
 
-__global__ void __launch_bounds__(kThreads) topk_radix_kernel(const float* __restrict__ scores, int64_t ld,
-                                                              const int32_t* __restrict__ ctx_len,
-                                                              const int32_t* __restrict__ q_pos0, int t_off,
-                                                              int n_q, int s_max, int k, int32_t* __restrict__ idx) {
-  __shared__ uint32_t hist[kBins];
+template <int PER>
+__global__ void __launch_bounds__(kThreads, 1)
+    topk_cluster_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ ctx_len,
+                        const int32_t* __restrict__ q_pos0, int t_off, int n_q, int s_max, int k,
+                        int32_t* __restrict__ idx) {
+  __shared__ uint32_t hist[3][kBins];
+  __shared__ uint32_t merged[kBins];
   __shared__ uint32_t wsum[kWarps + 1];
   __shared__ uint32_t s_digit, s_above;
+  __shared__ uint32_t s_tot[2];
 
-  const int r = blockIdx.x;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int C = static_cast<int>(cluster.num_blocks());
+  const int c = static_cast<int>(cluster.block_rank());
+  const int r = blockIdx.x / C;
   const int b = r / n_q, t = r % n_q;
   const int L = min(max(ctx_len[b], 0), s_max);
   const int n = max(0, min(q_pos0[b] + t_off + t + 1, L));  // candidates s in [0, n)
@@ -69,9 +82,32 @@ __global__ void __launch_bounds__(kThreads) topk_radix_kernel(const float* __res
   const float* row = scores + static_cast<int64_t>(r) * ld;
   const int tid = threadIdx.x;
 
-  if (n <= k) {
-    for (int j = tid; j < k; j += kThreads) out[j] = j < n ? j : -1;
+  if (n <= k) {  // the same for every CTA of the cluster: nobody syncs
+    for (int j = c * kThreads + tid; j < k; j += C * kThreads) out[j] = j < n ? j : -1;
     return;
+  }
+
+  // this thread's keys: s = s0 .. s0 + PER - 1
+  const int s0 = (c * kThreads + tid) * PER;
+  uint32_t key[PER];
+  uint32_t vmask = 0;
+  if (s0 + PER <= n) {
+#pragma unroll
+    for (int e = 0; e < PER; e += 4) {
+      const float4 f = *reinterpret_cast<const float4*>(row + s0 + e);
+      key[e] = float_order_key(f.x);
+      key[e + 1] = float_order_key(f.y);
+      key[e + 2] = float_order_key(f.z);
+      key[e + 3] = float_order_key(f.w);
+    }
+    vmask = (PER == 32) ? 0xffffffffu : ((1u << PER) - 1u);
+  } else {
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      const bool v = s0 + e < n;
+      key[e] = v ? float_order_key(row[s0 + e]) : 0u;
+      vmask |= (v ? 1u : 0u) << e;
+    }
   }
 
   uint32_t prefix = 0, pmask = 0, remaining = static_cast<uint32_t>(k);
@@ -79,43 +115,32 @@ __global__ void __launch_bounds__(kThreads) topk_radix_kernel(const float* __res
   for (int pass = 0; pass < 3; ++pass) {
     const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
     const uint32_t dmask = pass == 2 ? 0x3FFu : 0x7FFu;
-    for (int i = tid; i < kBins; i += kThreads) hist[i] = 0;
+    for (int i = tid; i < kBins; i += kThreads) hist[pass][i] = 0;
     __syncthreads();
-    const int n4 = n >> 2;
-    const float4* row4 = reinterpret_cast<const float4*>(row);
-    for (int i = tid; i < n4; i += kThreads) {
-      const float4 f = row4[i];
-      const uint32_t u0 = float_order_key(f.x), u1 = float_order_key(f.y);
-      const uint32_t u2 = float_order_key(f.z), u3 = float_order_key(f.w);
-      if ((u0 & pmask) == prefix) atomicAdd(&hist[(u0 >> shift) & dmask], 1u);
-      if ((u1 & pmask) == prefix) atomicAdd(&hist[(u1 >> shift) & dmask], 1u);
-      if ((u2 & pmask) == prefix) atomicAdd(&hist[(u2 >> shift) & dmask], 1u);
-      if ((u3 & pmask) == prefix) atomicAdd(&hist[(u3 >> shift) & dmask], 1u);
-    }
-    for (int s = (n4 << 2) + tid; s < n; s += kThreads) {
-      const uint32_t u = float_order_key(row[s]);
-      if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & dmask], 1u);
+#pragma unroll
+    for (int e = 0; e < PER; ++e)
+      if (((vmask >> e) & 1u) && (key[e] & pmask) == prefix) atomicAdd(&hist[pass][(key[e] >> shift) & dmask], 1u);
+    cluster.sync();  // every CTA's histogram of this pass is complete
+    for (int i = tid; i < kBins; i += kThreads) {
+      uint32_t v = 0;
+      for (int q = 0; q < C; ++q) v += cluster.map_shared_rank(&hist[pass][0], q)[i];
+      merged[i] = v;
     }
     __syncthreads();
-    // Digit holding the remaining-th largest key: scan bins from the top.
-    if (tid < 32) {
-      const int lane = tid;
-      constexpr int kPer = kBins / 32;
-      const int top = kBins - 1 - lane * kPer;  // this lane scans bins top .. top-kPer+1
-      uint32_t local = 0;
-      for (int i = 0; i < kPer; ++i) local += hist[top - i];
-      const uint32_t incl = warp_incl_scan(local);
-      const uint32_t excl = incl - local;
-      if (excl < remaining && remaining <= incl) {
-        uint32_t cum = excl;
-        for (int i = 0; i < kPer; ++i) {
-          const uint32_t c = hist[top - i];
-          if (cum + c >= remaining) {
-            s_digit = static_cast<uint32_t>(top - i);
-            s_above = cum;
-            break;
-          }
-          cum += c;
+    {
+      // bins from the top, two per thread; a block prefix sum finds the bin
+      // holding the remaining-th largest key
+      const int b0 = kBins - 1 - 2 * tid;
+      const uint32_t c0 = merged[b0], c1 = merged[b0 - 1];
+      uint32_t tot;
+      const uint32_t excl = block_excl_scan(c0 + c1, wsum, &tot);
+      if (excl < remaining && remaining <= excl + c0 + c1) {
+        if (remaining <= excl + c0) {
+          s_digit = static_cast<uint32_t>(b0);
+          s_above = excl;
+        } else {
+          s_digit = static_cast<uint32_t>(b0 - 1);
+          s_above = excl + c0;
         }
       }
     }
@@ -128,41 +153,64 @@ __global__ void __launch_bounds__(kThreads) topk_radix_kernel(const float* __res
   const uint32_t T = prefix;
   const uint32_t take_eq = remaining;  // keys == T to keep, lowest index first
 
-  // Ordered compaction: thread `tid` owns elements [base + tid*kSeg, +kSeg).
-  uint32_t gt_done = 0, eq_done = 0;
-  for (int base = 0; base < n; base += kThreads * kSeg) {
-    const int s0 = base + tid * kSeg;
-    uint32_t keys[kSeg];
+  uint32_t gt = 0, eq = 0;
 #pragma unroll
-    for (int e = 0; e < kSeg; ++e) {
-      const int s = s0 + e;
-      keys[e] = (s < n) ? float_order_key(row[s]) : 0u;  // 0 is below every real key
-    }
-    uint32_t gt = 0, eq = 0;
-#pragma unroll
-    for (int e = 0; e < kSeg; ++e) {
-      gt += keys[e] > T;
-      eq += (s0 + e < n) && keys[e] == T;
-    }
-    uint32_t total;
-    const uint32_t pre = block_excl_scan((gt << 16) | eq, wsum, &total);
-    const uint32_t gt_before = gt_done + (pre >> 16);
-    uint32_t eq_rank = eq_done + (pre & 0xFFFFu);
-    uint32_t pos = gt_before + min(eq_rank, take_eq);
-#pragma unroll
-    for (int e = 0; e < kSeg; ++e) {
-      const int s = s0 + e;
-      if (s >= n) break;
-      if (keys[e] > T) {
-        out[pos++] = s;
-      } else if (keys[e] == T) {
-        if (eq_rank < take_eq) out[pos++] = s;
-        ++eq_rank;
-      }
-    }
-    gt_done += total >> 16;
-    eq_done += total & 0xFFFFu;
+  for (int e = 0; e < PER; ++e) {
+    const bool v = (vmask >> e) & 1u;
+    gt += (v && key[e] > T) ? 1u : 0u;
+    eq += (v && key[e] == T) ? 1u : 0u;
   }
+  uint32_t total;
+  const uint32_t pre = block_excl_scan((gt << 16) | eq, wsum, &total);
+  if (tid == 0) {
+    s_tot[0] = total >> 16;
+    s_tot[1] = total & 0xFFFFu;
+  }
+  cluster.sync();  // CTA totals visible across the cluster
+  uint32_t gt_off = 0, eq_off = 0;
+  for (int q = 0; q < c; ++q) {
+    const uint32_t* pt = cluster.map_shared_rank(&s_tot[0], q);
+    gt_off += pt[0];
+    eq_off += pt[1];
+  }
+  uint32_t eq_rank = eq_off + (pre & 0xFFFFu);
+  uint32_t pos = gt_off + (pre >> 16) + min(eq_rank, take_eq);
+#pragma unroll
+  for (int e = 0; e < PER; ++e) {
+    if (!((vmask >> e) & 1u)) continue;
+    if (key[e] > T) {
+      out[pos++] = s0 + e;
+    } else if (key[e] == T) {
+      if (eq_rank < take_eq) out[pos++] = s0 + e;
+      ++eq_rank;
+    }
+  }
+  cluster.sync();  // peers may still be reading this CTA's shared memory
+}
+
+template <int PER>
+dsa_status_t launch_topk(const TopkArgs& a, int C) {
+  auto kern = topk_cluster_kernel<PER>;
+  if (C > 8) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+      return DSA_ERR_UNSUPPORTED;
+  }
+  const int64_t rows = static_cast<int64_t>(a.B) * a.n_q;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(rows * C), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = a.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a.scores, a.ld, a.ctx_len, a.q_pos0, a.t_off, a.n_q, a.s_max,
+                                           a.k, a.idx);
+  return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 }  // namespace
@@ -172,10 +220,23 @@ size_t topk_workspace_bytes(int, int, int, int) { return 0; }
 dsa_status_t topk_radix(const TopkArgs& a) {
   const int64_t rows = static_cast<int64_t>(a.B) * a.n_q;
   if (rows == 0) return DSA_OK;
-  if (rows > INT32_MAX) return DSA_ERR_UNSUPPORTED;
-  topk_radix_kernel<<<static_cast<unsigned>(rows), kThreads, 0, a.stream>>>(
-      a.scores, a.ld, a.ctx_len, a.q_pos0, a.t_off, a.n_q, a.s_max, a.k, a.idx);
-  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  const int num_sms = std::max(1, device_sm_count(a.device));
+  const int64_t n_max = std::max(1, a.s_max);
+  // Keys per thread: 16 when the rows alone fill the GPU, fewer (more CTAs
+  // per row) for a handful of long rows; at most 16 CTAs per row.
+  int per = 16;
+  if (rows * ((n_max + 16 * kThreads - 1) / (16 * kThreads)) < 2 * num_sms) {
+    if ((n_max + 4 * kThreads - 1) / (4 * kThreads) <= 8) per = 4;
+    else if ((n_max + 8 * kThreads - 1) / (8 * kThreads) <= 8) per = 8;
+  }
+  const int64_t C = (n_max + static_cast<int64_t>(per) * kThreads - 1) / (static_cast<int64_t>(per) * kThreads);
+  if (C > kMaxCluster) return DSA_ERR_UNSUPPORTED;
+  if (rows * C > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  switch (per) {
+    case 4: return launch_topk<4>(a, static_cast<int>(C));
+    case 8: return launch_topk<8>(a, static_cast<int>(C));
+    default: return launch_topk<16>(a, static_cast<int>(C));
+  }
 }
 
 }  // namespace dsa
