@@ -12,11 +12,13 @@
 //     memory, so a CTA accumulates one 256-column half of it in TMEM; the
 //     two halves recompute the same logits (S = Q K^T, M = 128 heads).
 //   * Warps 0-3 gather the selected latent rows (1152 bytes each) into a
-//     2-stage shared-memory ring with cp.async, 16 bytes per thread, written
-//     straight into the 128-byte-swizzled K-major layout the MMA reads;
-//     rows that are padding (-1) or out of range are zero-filled.
+//     2-stage shared-memory ring with TMA row gathers (tile::gather4, four
+//     rows x 64 columns per instruction) into the 128-byte-swizzled K-major
+//     layout the MMA reads; padding (-1) or out-of-range rows are read at
+//     row -1, which TMA fills with zeros.
 //   * Warp 4 loads Q once with TMA and issues tcgen05.mma: S(j) for tile j
-//     (32 rows), then O += P(j-1) V(j-1), so the logits of the next tile are
+//     (32 rows) in three chunks, and O += P(j-1) V(j-1) as soon as P is ready
+//     (between chunks if need be), so the logits of the next tile are
 //     computed while the softmax warps work on the current one.
 //   * Warps 5-8 (thread = head = TMEM lane) run the online softmax in base 2:
 //     read S, mask, keep a running max that is only moved (and O rescaled in
@@ -40,9 +42,10 @@ constexpr int kBox = kRows * 128;       // bytes of one 64-column block of a til
 constexpr int kTile = kKB * kBox;       // 36 KB
 constexpr int kQBytes = kKB * kH * 128; // 144 KB
 constexpr int kStages = 2;
-constexpr int kProdThreads = 128;
 constexpr int kSoftThreads = 128;
-constexpr int kThreads = kProdThreads + 32 + kSoftThreads;  // 288
+constexpr int kGatherWarps = 4;
+constexpr int kMmaWarp = kGatherWarps;
+constexpr int kThreads = 32 * kGatherWarps + 32 + kSoftThreads;  // gather warps, MMA warp, 4 softmax warps
 constexpr int kTmemCols = 512;          // O half: cols [0,256), S buffers: [256,288), [288,320)
 constexpr int kSCol = 256;
 
@@ -85,6 +88,21 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn(int M, int N) {
   return idesc_bf16_f32(M, N) | (1u << 16);
 }
 
+// TMA row gather: rows r0..r3 of a 2-D tensor map, 64 columns from `col`,
+// written as four consecutive 128-byte swizzled rows at `dst`.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, uint32_t bar, int col, int r0,
+                                            int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
@@ -114,7 +132,8 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 
 
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, AttnParams P) {
+    attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_kv,
+                       AttnParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
@@ -147,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
-      mbar_init(kv_full(i), kProdThreads);
+      mbar_init(kv_full(i), kGatherWarps);
       mbar_init(kv_empty(i), 1);
       mbar_init(s_full(i), 1);
       mbar_init(s_empty(i), kSoftThreads);
@@ -159,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_addr(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
@@ -168,36 +187,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp < 4) {
-    // ------------------------------------------------ gather (cp.async) --
-    const int tid = threadIdx.x;
-    const char* kv_b = reinterpret_cast<const char*>(P.kv) + static_cast<int64_t>(b) * P.s_max * kDqk * 2;
+  if (warp < kGatherWarps) {
+    // -------------------------------------------------- gather (TMA) --
     bool bad = false;
-    // lane i of every producer warp holds the index of row i of the tile;
-    // the next tile's indices are fetched before this tile's copies go out
+    // lane i holds the (flattened) row of tile row i; the next tile's
+    // indices are fetched before this tile's gathers go out
     int nxt = (lane < nrows) ? __ldg(sel + lane) : -1;
+    const int grp = lane & 7;  // this lane gathers rows 4*grp .. 4*grp+3
     for (int j = 0; j < T; ++j) {
       const int st = j & 1;
       int cur = nxt;
       if (cur >= L) { bad = true; cur = -1; }
+      const int grow = cur >= 0 ? b * P.s_max + cur : -1;  // row -1 reads zeros
       const int jn = (j + 1) * kRows + lane;
       nxt = (j + 1 < T && jn < nrows) ? __ldg(sel + jn) : -1;
+      const int r0 = __shfl_sync(0xffffffffu, grow, 4 * grp + 0);
+      const int r1 = __shfl_sync(0xffffffffu, grow, 4 * grp + 1);
+      const int r2 = __shfl_sync(0xffffffffu, grow, 4 * grp + 2);
+      const int r3 = __shfl_sync(0xffffffffu, grow, 4 * grp + 3);
       if (!mbar_wait_warp(kv_empty(st), ((j >> 1) & 1) ^ 1, abort_flag, P.err)) break;
-      const uint32_t dst0 = sbase + kOffKV + st * kTile;
-#pragma unroll 6
-      for (int i = 0; i < kRows * 72 / kProdThreads; ++i) {
-        const int x = i * kProdThreads + tid;
-        const int row = x / 72, cc = x % 72;
-        const int s = __shfl_sync(0xffffffffu, cur, row);
-        const uint32_t dst = dst0 + (cc >> 3) * kBox + row * 128 + (((cc & 7) ^ (row & 7)) << 4);
-        const char* src = kv_b + (s >= 0 ? static_cast<int64_t>(s) * (kDqk * 2) + cc * 16 : 0);
-        cp_async16(dst, src, s >= 0 ? 16u : 0u);
-      }
-      cp_async_arrive(kv_full(st));
+      // warp w gathers the 64-column blocks w, w+4, w+8 of the tile; each
+      // warp's first lane adds its share of the bytes to the stage's barrier
+      int nblk = 0;
+      for (int kb = warp; kb < kKB; kb += kGatherWarps) ++nblk;
+      if (lane == 0) mbar_arrive_expect_tx(kv_full(st), nblk * 8 * 512);
+      __syncwarp();
+      const uint32_t dst0 = sbase + kOffKV + st * kTile + grp * 512;
+      for (int kb = warp + kGatherWarps * (lane >> 3); kb < kKB && (lane >> 3) < 3; kb += kGatherWarps * 4)
+        tma_gather4(dst0 + kb * kBox, &tmap_kv, kv_full(st), kb * 64, r0, r1, r2, r3);
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");
-    if (bad) raise_error(P.err, kErrBadIndex);
-  } else if (warp == 4) {
+    if (__any_sync(0xffffffffu, bad) && lane == 0) raise_error(P.err, kErrBadIndex);
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------- MMA issue --
     if (lane == 0) {
       const uint32_t qaddr = sbase + kOffQ;
@@ -226,22 +246,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Issue whichever of QK(nq) / PV(np) is ready (PV first), so the value
       // product of a tile -- which frees its stage for the next gather -- never
       // waits behind the logits of a tile whose rows are still in flight.
-      auto issue_qk = [&](int j) {
+      // S(j) = Q K(j)^T is issued in kQkParts chunks; a P(i) that becomes
+      // ready is issued between chunks, so the value product of a tile (which
+      // frees its stage for the next gather) never queues behind a whole QK.
+      constexpr int kQkMma = kDqk / 16;  // 36
+      constexpr int kQkParts = 3;
+      auto issue_qk_part = [&](int j, int part) {
         const int st = j & 1;
-        fence_proxy_async_smem();  // cp.async (generic proxy) writes -> tensor-core reads
-        tc_fence_after_sync();
+        if (part == 0) tc_fence_after_sync();
         const uint32_t d = tmem + kSCol + st * kRows;
         const uint64_t kv0 = kv_desc0 + static_cast<uint64_t>((st * kTile) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < kDqk / 16; ++kk) {
+        for (int q = 0; q < kQkMma / kQkParts; ++q) {
+          const int kk = part * (kQkMma / kQkParts) + q;
           // descriptor start addresses advance in 16-byte units
           const uint32_t a_off = (kk >> 2) * kH * 128 + (kk & 3) * 32;
           const uint32_t b_off = (kk >> 2) * kBox + (kk & 3) * 32;
           tc_mma_f16(d, q_desc0 + (a_off >> 4), kv0 + (b_off >> 4), idesc_s, kk > 0 ? 1u : 0u);
         }
-        tc_commit(s_full(st));
+        if (part == kQkParts - 1) tc_commit(s_full(st));
       };
-      int nq = 0, np = 0;
+      int nq = 0, np = 0, qpart = 0;  // QK(nq) has issued qpart chunks
       uint64_t t0 = 0;
       uint32_t spins = 0;
       while (ok && np < T) {
@@ -251,10 +276,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           spins = 0;
           continue;
         }
+        if (qpart > 0) {
+          issue_qk_part(nq, qpart);
+          if (++qpart == kQkParts) { qpart = 0; ++nq; }
+          spins = 0;
+          continue;
+        }
         if (nq < T && mbar_test_wait(kv_full(nq & 1), (nq >> 1) & 1) &&
             mbar_test_wait(s_empty(nq & 1), ((nq >> 1) & 1) ^ 1)) {
-          issue_qk(nq);
-          ++nq;
+          issue_qk_part(nq, 0);
+          qpart = 1;
           spins = 0;
           continue;
         }
@@ -280,11 +311,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
+    int sidx_next = (lane < nrows) ? __ldg(sel + lane) : -1;
     for (int j = 0; j < T; ++j) {
       const int st = j & 1;
-      // which rows of this tile are real
-      const int jr = j * kRows + lane;
-      int sidx = (jr < nrows) ? __ldg(sel + jr) : -1;
+      // which rows of this tile are real (indices fetched one tile ahead)
+      const int sidx = sidx_next;
+      const int jn = (j + 1) * kRows + lane;
+      sidx_next = (j + 1 < T && jn < nrows) ? __ldg(sel + jn) : -1;
       const uint32_t valid = __ballot_sync(0xffffffffu, sidx >= 0 && sidx < L);
       if (!mbar_wait_warp(s_full(st), (j >> 1) & 1, abort_flag, P.err)) { ok = false; break; }
       tc_fence_after_sync();
@@ -329,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float p[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          p[e] = (m_run == -INFINITY) ? 0.f : exp2f(s[c * 8 + e] - m_run);
+          p[e] = (m_run == -INFINITY) ? 0.f : fast_exp2(s[c * 8 + e] - m_run);
           psum += p[e];
         }
         st_shared_v4(prow + ((c ^ sw) << 4), pack_bf16(p[0], p[1]), pack_bf16(p[2], p[3]), pack_bf16(p[4], p[5]),
@@ -387,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before_sync();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tc_fence_after_sync();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -525,6 +558,10 @@ dsa_status_t attn_tc(const AttnArgs& a) {
   CUtensorMap tmq;
   if (!make_tmap_2d(&tmq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDqk, static_cast<uint64_t>(R) * kH, 64, kH))
     return DSA_ERR_CUDA;
+  CUtensorMap tmkv;
+  if (!make_tmap_2d(&tmkv, a.kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDqk, static_cast<uint64_t>(a.B) * a.s_max, 64,
+                    1))
+    return DSA_ERR_CUDA;
   static bool attr_done[64] = {};
   if (a.device < 64 && !attr_done[a.device]) {
     if (cudaFuncSetAttribute(attn_mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
@@ -533,7 +570,7 @@ dsa_status_t attn_tc(const AttnArgs& a) {
     attr_done[a.device] = true;
   }
   const unsigned grid = static_cast<unsigned>(R * p.splits * 2);
-  attn_mla_tc_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(tmq, P);
+  attn_mla_tc_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(tmq, tmkv, P);
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
   if (p.splits > 1) {
     attn_combine_kernel<<<dim3(static_cast<unsigned>(R), kH / kCombineHeads), 256, 0, a.stream>>>(P.part_o, P.part_ml, p.splits, P.out,
