@@ -210,6 +210,33 @@ dsa_status_t dsa_forward_host(const dsa_shape_t *shape,
                               void *workspace, size_t workspace_bytes,
                               void *stream);
 
+/*
+ * dsa_sparse_mla_attn without a workspace argument: the scratch memory that
+ * the split-K combine needs comes from a fixed array inside the library.
+ * The pages have no counterpart to this call; it exists for callers that
+ * cannot hand the library device memory on their decode path -- a serving
+ * loop whose device memory is planned once up front and may not grow, or a
+ * host program without a device allocator of its own (cudaMalloc, which can
+ * synchronise the whole device, is no substitute there).
+ * Arguments and results are those of dsa_sparse_mla_attn.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *   - The array is 32 MiB and lives on every GPU that loads the library until
+ *     the process exits.  A shape that would need more returns
+ *     DSA_ERR_WORKSPACE before anything is enqueued (on a 148-SM B200 no
+ *     shape needs more than about 20 MB).
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - Every call shares the one array and leaves the last call's partial
+ *     results in it; nothing in it has to start at zero.  Calls that overlap
+ *     on the GPU (different streams, or devices sharing a context) race on
+ *     it: serialise them.
+ */
+dsa_status_t dsa_sparse_mla_attn_static(const dsa_shape_t *shape,
+                                        const void *q, const void *kv, const void *v,
+                                        const int32_t *idx, const int32_t *ctx_len,
+                                        void *out, float *lse,
+                                        void *stream);
+
 /* Bytes of device workspace a call needs (DSA_WS_*); 0 for an invalid shape. */
 size_t dsa_workspace_bytes(const dsa_shape_t *shape, int32_t which);
 

@@ -27,6 +27,7 @@ STATUS = {
 EXPORTS = (
     "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_hadamard_quant_fp8", "dsa_forward",
     "dsa_forward_host", "dsa_workspace_bytes", "dsa_get_error", "dsa_status_string", "dsa_version",
+    "dsa_sparse_mla_attn_static",
 )
 
 
@@ -70,6 +71,7 @@ def lib():
         L.dsa_topk.argtypes = [S, P, i64, P, P, P, P, sz, P]
         L.dsa_sparse_mla_attn.argtypes = [S, P, P, P, P, P, P, P, P, sz, P]
         L.dsa_hadamard_quant_fp8.argtypes = [P, i32, i64, i32, P, P, P]
+        L.dsa_sparse_mla_attn_static.argtypes = [S, P, P, P, P, P, P, P, P]
         L.dsa_forward.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
         L.dsa_forward_host.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
         L.dsa_workspace_bytes.argtypes = [S, i32]
@@ -168,6 +170,16 @@ def sparse_mla_attn(shape, q, kv, idx, ctx_len, out=None, v=None, lse=None, work
     ws, n = _workspace(shape, WS_ATTN, workspace, q.device)
     _check(lib().dsa_sparse_mla_attn(ctypes.byref(shape), _p(q), _p(kv), _p(v), _p(idx), _p(ctx_len), _p(out),
                                      _p(lse), _p(ws), n, _stream(stream)), "dsa_sparse_mla_attn")
+    return out
+
+
+def sparse_mla_attn_static(shape, q, kv, idx, ctx_len, out=None, v=None, lse=None, stream=None):
+    """As sparse_mla_attn, with the split scratch in the library's fixed
+    device array instead of a workspace (see dsa_sparse_mla_attn_static)."""
+    if out is None:
+        out = torch.empty(shape.batch, shape.n_q, shape.heads, shape.d_v, dtype=q.dtype, device=q.device)
+    _check(lib().dsa_sparse_mla_attn_static(ctypes.byref(shape), _p(q), _p(kv), _p(v), _p(idx), _p(ctx_len),
+                                            _p(out), _p(lse), _stream(stream)), "dsa_sparse_mla_attn_static")
     return out
 
 

@@ -581,3 +581,16 @@ dsa_status_t attn_tc(const AttnArgs& a) {
 }
 
 }  // namespace dsa
+
+namespace dsa {
+// Exact scratch bytes the tensor-core attention needs for this shape on a
+// device with `num_sms` SMs (0 when it writes its output directly).
+size_t attn_scratch_bytes(int B, int n_q, int k, int num_sms) {
+  const int64_t R = static_cast<int64_t>(B) * n_q;
+  if (R == 0) return 0;
+  const SplitPlan p = plan_splits(R, k, num_sms);
+  if (p.splits <= 1) return 0;
+  const size_t items = static_cast<size_t>(R) * p.splits * 2;
+  return items * kH * kDvHalf * 4 + items * 2 * kH * 4;
+}
+}  // namespace dsa

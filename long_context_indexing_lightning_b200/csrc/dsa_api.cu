@@ -519,3 +519,60 @@ const char* dsa_status_string(dsa_status_t status) {
 int32_t dsa_version(void) { return 100; }
 
 }  // extern "C"
+
+// ------------------------------------------------ allocation-free attention --
+// dsa_sparse_mla_attn_static: the same attention, with the scratch memory of
+// the split-K combine taken from a fixed array inside this library instead
+// of a caller-provided workspace.  For callers that cannot hand the library
+// device memory on their decode path: a serving loop whose device memory is
+// planned once up front and may not grow, or a host program with no device
+// allocator of its own -- for both, cudaMalloc is also a poor fit because it
+// can synchronise the whole device.
+namespace dsa {
+namespace {
+
+// Capacity of the scratch array.  A 148-SM B200 needs at most about 20 MB
+// (decode with 37 queries per call); larger needs are rejected.
+constexpr size_t kStaticAttnScratchBytes = size_t(32) << 20;
+
+// File-scope device array: every GPU that loads this library holds it until
+// the process exits.  Host code must not pass `g_attn_scratch` itself to a
+// kernel -- in host code the name is a stand-in, not a device address -- but
+// the address obtained with cudaGetSymbolAddress below.
+__device__ __align__(256) unsigned char g_attn_scratch[kStaticAttnScratchBytes];
+
+std::mutex g_static_mutex;
+void* g_static_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on `dev` (the current device), looked
+// up once per device.
+void* static_attn_scratch(int dev) {
+  std::lock_guard<std::mutex> lock(g_static_mutex);
+  if (g_static_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_attn_scratch) != cudaSuccess) return nullptr;
+    g_static_scratch_ptr[dev] = p;
+  }
+  return g_static_scratch_ptr[dev];
+}
+
+}  // namespace
+}  // namespace dsa
+
+extern "C" dsa_status_t dsa_sparse_mla_attn_static(const dsa_shape_t* shape, const void* q, const void* kv,
+                                                   const void* v, const int32_t* idx, const int32_t* ctx_len,
+                                                   void* out, float* lse, void* stream) {
+  dsa_status_t st = check_shape(shape);
+  if (st != DSA_OK) return st;
+  st = check_attn_inputs(shape, q, kv, v, idx, ctx_len, out);
+  if (st != DSA_OK) return st;
+  DSA_SETUP(dev);
+  size_t need = 0;
+  if (shape->attn_dtype == DSA_BF16 && attn_tc_supported(shape->heads, shape->d_qk, shape->d_v, shape->kv_heads))
+    need = attn_scratch_bytes(shape->batch, shape->n_q, shape->topk, device_sm_count(dev));
+  if (need > kStaticAttnScratchBytes) return DSA_ERR_WORKSPACE;  // beyond the fixed capacity
+  void* scratch = static_attn_scratch(dev);
+  if (scratch == nullptr) return DSA_ERR_CUDA;
+  return run_attn(shape, dev, static_cast<cudaStream_t>(stream), shape->batch, shape->n_q, q, kv, v, idx, ctx_len,
+                  out, lse, scratch, kStaticAttnScratchBytes);
+}

@@ -84,6 +84,7 @@ size_t attn_workspace_bytes(int B, int n_q, int H, int d_qk, int d_v, int KVH, i
 dsa_status_t attn_tc(const AttnArgs& a);    // BF16 absorbed MLA, tensor cores
 dsa_status_t attn_simt(const AttnArgs& a);  // F32 (and BF16 shapes the tensor path does not take)
 bool attn_tc_supported(int H, int d_qk, int d_v, int KVH);
+size_t attn_scratch_bytes(int B, int n_q, int k, int num_sms);
 
 dsa_status_t hadamard_quant(const void* x, int x_dtype, int64_t rows, int dim, uint8_t* x8, float* scale,
                             cudaStream_t stream);
