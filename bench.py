@@ -128,6 +128,28 @@ def _indexer_flops(wl):
     return 2.0 * wl.idx_heads * wl.idx_dim * pairs
 
 
+def _attn_extra_launches(wl, dsa, shape):
+    """The split combine is a second attention launch when the split plan needs scratch."""
+    return 1 if dsa.workspace_bytes(shape, dsa.WS_ATTN) > 0 else 0
+
+
+# DRAM bytes per indexer launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum),
+# keyed by workload and by the SHA-256 of the indexer source the counters were taken on;
+# a changed kernel reports null.  Filled in from profiles/indexer_tc_decode128k.md.
+TRAFFIC = {}
+
+
+def _traffic(wl):
+    import hashlib
+    path = os.path.join(ROOT, "long_context_indexing_lightning_b200", "csrc", "indexer_tc.cu")
+    try:
+        sha = hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    rec = TRAFFIC.get(wl.name)
+    return rec[1] if rec and rec[0] == sha else None
+
+
 def run_ours(args, wl):
     import long_context_indexing_lightning_b200 as dsa
 
@@ -141,11 +163,7 @@ def run_ours(args, wl):
     shape = dsa.shape_from_workload(wl)
     stream = torch.cuda.current_stream(dev)
     ld = (wl.s_max + 3) // 4 * 4
-    scores = torch.empty(wl.batch, wl.n_q, ld, dtype=torch.float32, device=dev)
-    idx = torch.empty(wl.batch, wl.n_q, wl.topk, dtype=torch.int32, device=dev)
     out = torch.empty(wl.batch, wl.n_q, wl.heads, wl.d_v, dtype=t["q"].dtype, device=dev)
-    ws_topk = torch.empty(max(1, dsa.workspace_bytes(shape, dsa.WS_TOPK)), dtype=torch.uint8, device=dev)
-    ws_attn = torch.empty(max(1, dsa.workspace_bytes(shape, dsa.WS_ATTN)), dtype=torch.uint8, device=dev)
     k_idx, k_scale, q_idx, q_scale = t["k_idx"], None, t["q_idx"], None
     q8 = qs = None
     if wl.idx_fp8:
@@ -154,20 +172,40 @@ def run_ours(args, wl):
         qs = torch.empty(q_idx.shape[:-1], dtype=torch.float32, device=dev)
         del t["k_idx"]
 
-    def step(ev=None):
+    # prefill runs in rounds of `chunk` queries (positions shifted by the
+    # round's first query); decode is a single round
+    chunk = wl.n_q if wl.n_q <= args.q_chunk else args.q_chunk
+    rounds = []
+    for t0 in range(0, wl.n_q, chunk):
+        c = min(chunk, wl.n_q - t0)
+        sh = shape.replace(n_q=c)
+        rounds.append((t0, c, sh, (t["q_pos0"] + t0).contiguous()))
+    if len(rounds) > 1 and wl.batch != 1:
+        raise SystemExit("prefill rounds are cut per sequence: use batch 1")
+    scores = torch.empty(wl.batch, chunk, ld, dtype=torch.float32, device=dev)
+    idx = torch.empty(wl.batch, chunk, wl.topk, dtype=torch.int32, device=dev)
+    ws_topk = torch.empty(max(1, dsa.workspace_bytes(rounds[0][2], dsa.WS_TOPK)), dtype=torch.uint8, device=dev)
+    ws_attn = torch.empty(max(1, dsa.workspace_bytes(rounds[0][2], dsa.WS_ATTN)), dtype=torch.uint8, device=dev)
+
+    def step(evr=None):
+        """One pass of the whole path; evr = per-round event quadruples or None."""
         if wl.idx_fp8:
             dsa.hadamard_quant_fp8(q_idx, q8, qs, stream=stream)
             qi, qsc = q8, qs
         else:
             qi, qsc = q_idx, None
-        if ev: ev[0].record(stream)
-        dsa.indexer_scores(shape, qi, k_idx, t["w"], t["ctx_len"], t["q_pos0"], scores=scores, q_scale=qsc,
-                           k_scale=k_scale, stream=stream)
-        if ev: ev[1].record(stream)
-        dsa.topk(shape, scores, t["ctx_len"], t["q_pos0"], idx=idx, workspace=ws_topk, stream=stream)
-        if ev: ev[2].record(stream)
-        dsa.sparse_mla_attn(shape, t["q"], t["kv"], idx, t["ctx_len"], out=out, workspace=ws_attn, stream=stream)
-        if ev: ev[3].record(stream)
+        for ri, (t0, c, sh, pos0) in enumerate(rounds):
+            ev = evr[ri] if evr is not None else None
+            sl = slice(t0, t0 + c)
+            if ev: ev[0].record(stream)
+            dsa.indexer_scores(sh, qi[:, sl], k_idx, t["w"][:, sl], t["ctx_len"], pos0, scores=scores[:, :c],
+                               q_scale=None if qsc is None else qsc[:, sl], k_scale=k_scale, stream=stream)
+            if ev: ev[1].record(stream)
+            dsa.topk(sh, scores[:, :c], t["ctx_len"], pos0, idx=idx[:, :c], workspace=ws_topk, stream=stream)
+            if ev: ev[2].record(stream)
+            dsa.sparse_mla_attn(sh, t["q"][:, sl], t["kv"], idx[:, :c], t["ctx_len"], out=out[:, sl],
+                                workspace=ws_attn, stream=stream)
+            if ev: ev[3].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -176,7 +214,7 @@ def run_ours(args, wl):
     if rc != 0:
         raise RuntimeError(f"device error word {word:#x} after warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in rounds] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     if ws > 1:
@@ -194,10 +232,11 @@ def run_ours(args, wl):
         torch.distributed.barrier()
     total_ms = start.elapsed_time(end)
     stage_ms = {"indexer": 0.0, "topk": 0.0, "attention": 0.0}
-    for e in evs:
-        stage_ms["indexer"] += e[0].elapsed_time(e[1])
-        stage_ms["topk"] += e[1].elapsed_time(e[2])
-        stage_ms["attention"] += e[2].elapsed_time(e[3])
+    for per_step in evs:
+        for e in per_step:
+            stage_ms["indexer"] += e[0].elapsed_time(e[1])
+            stage_ms["topk"] += e[1].elapsed_time(e[2])
+            stage_ms["attention"] += e[2].elapsed_time(e[3])
     stage_ms = {k: v / args.steps for k, v in stage_ms.items()}
     rc, word = dsa.get_error(clear=True)
     if rc != 0:
@@ -209,7 +248,8 @@ def run_ours(args, wl):
     ms_per_step = total_ms / args.steps
 
     # end to end through the host-buffer entry point
-    e2e = _e2e(args, wl, dsa, shape, t, k_idx, k_scale, dev, stream)
+    e2e = _e2e(args, wl, dsa, dsa.shape_from_workload(wl, q_chunk=chunk if len(rounds) > 1 else 0), t, k_idx,
+               k_scale, dev, stream)
     if ws > 1:
         tt = torch.tensor([e2e["ms"]], device=dev)
         torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
@@ -218,14 +258,30 @@ def run_ours(args, wl):
     res = None
     if rank == 0:
         hbm, tf, tf_sus, src = _peaks()
-        idx_bytes = _indexer_bytes(wl)
         idx_ms = stage_ms["indexer"]
-        achieved = idx_bytes / (idx_ms * 1e-3) / 1e9
         q_total = _queries(wl) * ws
+        decode = wl.n_q == 1
+        if decode:
+            idx_bytes = _indexer_bytes(wl)
+            achieved = idx_bytes / (idx_ms * 1e-3) / 1e9
+            roof = {"kernel": "indexer", "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                    "frac": achieved / hbm, "peak_source": f"{src} hbm_gbs (of {src})",
+                    "traffic": _traffic(wl), "algorithmic_bytes": idx_bytes,
+                    "tensor_tflops": _indexer_flops(wl) / (idx_ms * 1e-3) / 1e12}
+            metric = ("DSA layer queries/s at 128K ctx" if wl.s_max == 131072
+                      else f"DSA layer queries/s ({wl.name})")
+        else:
+            flops = _indexer_flops(wl)
+            achieved = flops / (idx_ms * 1e-3) / 1e12
+            peak = tf_sus if tf_sus > 0 else tf
+            roof = {"kernel": "indexer", "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "peak_source": f"{src} bf16_tflops_sustained (of {src})",
+                    "traffic": _traffic(wl), "algorithmic_flops": flops}
+            metric = f"DSA layer prefill tokens/s ({wl.name})"
         res = {
-            "metric": "DSA layer queries/s at 128K ctx" if wl.s_max == 131072 else f"DSA layer queries/s ({wl.name})",
+            "metric": metric,
             "value": q_total / (ms_per_step * 1e-3),
-            "unit": "queries/s",
+            "unit": "queries/s" if decode else "tokens/s",
             "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -233,15 +289,15 @@ def run_ours(args, wl):
             "data": "synthetic (seeded gaussian, bf16)",
             "config": {"workload": _workload_desc(wl), "global_batch": q_total, "seq_len": wl.s_max,
                        "parallelism": f"replicas{ws}" if ws > 1 else "single",
-                       "l2": "inputs larger than L2 (index-key cache read each step)"},
+                       "q_chunk": chunk,
+                       "l2": "inputs larger than L2 (index-key cache read each step)" if decode
+                             else "latent cache fits L2 (9.4 MB at 8K); no flush between steps"},
             "stages_ms": stage_ms,
-            "roofline": {"kernel": "indexer", "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                         "frac": achieved / hbm, "peak_source": f"{src} hbm_gbs", "traffic": None,
-                         "algorithmic_bytes": idx_bytes,
-                         "tensor_tflops": _indexer_flops(wl) / (idx_ms * 1e-3) / 1e12},
-            "gpu_launches": args.steps * (4 if wl.idx_fp8 else 3),
+            "roofline": roof,
+            "gpu_launches": args.steps * (len(rounds) * (3 + _attn_extra_launches(wl, dsa, rounds[0][2]))
+                                          + (1 if wl.idx_fp8 else 0)),
             "clocks": clk,
-            "e2e": {"value": q_total / (e2e["ms"] * 1e-3), "unit": "queries/s",
+            "e2e": {"value": q_total / (e2e["ms"] * 1e-3), "unit": "queries/s" if decode else "tokens/s",
                     "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
         }
     if ws > 1:
@@ -274,19 +330,26 @@ def _e2e(args, wl, dsa, shape, t, k_idx, k_scale, dev, stream):
 
 def _oracle_sample(wl, n_rows, seed=0):
     """The CPU oracle (as it stands) on `n_rows` query rows of the workload:
-    indexer scores -> top-k -> sparse attention.  Returns (seconds, rows)."""
+    indexer scores -> top-k -> sparse attention.  Decode: `n_rows` sequences
+    of the workload's context; prefill: `n_rows` query rows drawn uniformly
+    from one sequence.  Returns (seconds, rows)."""
     import numpy as np
     import oracle
-    sub = workloads.get(wl.name, batch=n_rows)
-    t = workloads.make_inputs(sub, "cuda" if torch.cuda.is_available() else "cpu", seed=seed)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    if wl.n_q == 1:
+        sub = workloads.get(wl.name, batch=n_rows)
+        rows = [(b, 0) for b in range(n_rows)]
+    else:
+        sub = workloads.get(wl.name, batch=1)
+        rows = [(0, r) for r in workloads.sample_rows(wl.n_q, n_rows, seed=seed + 1)]
+    t = workloads.make_inputs(sub, dev, seed=seed)
     h = {k: workloads.to_numpy(v) for k, v in t.items()}
-    rows = [(b, 0) for b in range(n_rows)]
     t0 = time.perf_counter()
     sc = oracle.indexer_scores(h["q_idx"], h["k_idx"], h["w"], h["ctx_len"], h["q_pos0"], rows=rows)
-    pos = np.array([h["q_pos0"][b] for b, _ in rows], dtype=np.int32)
+    pos = np.array([h["q_pos0"][b] + r for b, r in rows], dtype=np.int32)
     idx = oracle.topk(np.where(np.isfinite(sc), sc, -np.inf).astype(np.float32), pos, sub.topk)
     oracle.sparse_attn(h["q"], h["kv"], idx, sub.sm_scale, v=sub.d_v, rows=rows)
-    return time.perf_counter() - t0, n_rows
+    return time.perf_counter() - t0, len(rows)
 
 
 def cpu_baseline(wl, n_rows=None):
@@ -294,9 +357,10 @@ def cpu_baseline(wl, n_rows=None):
     cores = oracle.num_threads()
     n_rows = n_rows or max(1, min(wl.batch, cores))
     secs, rows = _oracle_sample(wl, n_rows)
-    return {"value": rows / secs, "unit": "queries/s", "cores": cores, "kind": "oracle",
-            "sample": f"{rows} decode queries of the same workload (full {wl.s_max}-key context each), "
-                      f"{secs:.1f} s on {cores} host threads"}
+    what = (f"{rows} decode queries of the same workload (full {wl.s_max}-key context each)" if wl.n_q == 1
+            else f"{rows} query rows drawn uniformly from the {wl.n_q}-token prefill")
+    return {"value": rows / secs, "unit": "queries/s" if wl.n_q == 1 else "tokens/s", "cores": cores,
+            "kind": "oracle", "sample": f"{what}, {secs:.1f} s on {cores} host threads"}
 
 
 def run_reference(args, wl):
@@ -341,6 +405,7 @@ def main():
     ap.add_argument("--workload", default="decode128k", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling runs)")
+    ap.add_argument("--q-chunk", type=int, default=4096, help="prefill: queries per indexer/top-k/attention round")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

@@ -7,65 +7,76 @@
 // 512, qk_rope_head_dim 64): every head's 576-wide query meets one shared
 // 576-wide latent row per token; the value is the row's first 512 columns.
 //
-// One CTA = (query row, split of its selected list, half of d_v).
-//   * The output of one query (128 heads x 512 fp32) would fill all of tensor
-//     memory, so a CTA accumulates one 256-column half of it in TMEM; the
-//     two halves recompute the same logits (S = Q K^T, M = 128 heads).
-//   * Warps 0-3 gather the selected latent rows (1152 bytes each) into a
-//     2-stage shared-memory ring with TMA row gathers (tile::gather4, four
-//     rows x 64 columns per instruction) into the 128-byte-swizzled K-major
-//     layout the MMA reads; padding (-1) or out-of-range rows are read at
-//     row -1, which TMA fills with zeros.
-//   * Warp 4 loads Q once with TMA and issues tcgen05.mma: S(j) for tile j
-//     (32 rows) in three chunks, and O += P(j-1) V(j-1) as soon as P is ready
-//     (between chunks if need be), so the logits of the next tile are
-//     computed while the softmax warps work on the current one.
-//   * Warps 5-8 (thread = head = TMEM lane) run the online softmax in base 2:
-//     read S, mask, keep a running max that is only moved (and O rescaled in
-//     TMEM) when the tile max exceeds it by more than 2^8, write P as bf16
-//     into the part of the tile's stage that the value half does not use, and
-//     finally normalise O (or store an unnormalised partial for the split
-//     combine).
+// One thread-block cluster of two CTAs per (query row, split of its selected
+// list).  The 576 latent columns are cut at 256: CTA 0 owns columns [0, 256),
+// CTA 1 owns [256, 576).  Each CTA
+//   * gathers only its own columns of the selected rows (cp.async, 16 bytes a
+//     thread, into a 3-stage ring of 64-row tiles in the 128-byte-swizzled
+//     K-major layout the MMA reads; padding and out-of-range rows are zero
+//     filled),
+//   * keeps its columns of Q in tensor memory (A operand of the logits MMA),
+//   * computes its partial logits S_c = Q_c K_c^T (M = 128 heads, N = 64 rows),
+//   * swaps partials with the other CTA (a bulk copy of 32 KB into the other
+//     CTA's shared memory, completing on its barrier), so
+//     both hold the same S = S_0 + S_1 (fp32 addition is commutative, so the
+//     two sums are bit-identical) and run the same online softmax,
+//   * accumulates its 256-column half of the output, O_c += P V_c, in TMEM
+//     (V_0 = latent columns [0, 256), V_1 = [256, 512): each CTA's value half
+//     lies inside the columns it already gathered).
+// Warps: 0-3 gather, 4 issues tcgen05.mma, 5-8 (thread = head = TMEM lane)
+// load Q into TMEM and run the softmax in base 2 with a running max that only
+// moves (and O is rescaled in TMEM) when a tile max exceeds it by more than 8.
+// Long selections are split across clusters and merged by a small combine
+// kernel (log-sum-exp weights).  Every wait is bounded.
 #include "dsa_common.cuh"
 #include "dsa_internal.h"
 
 namespace dsa {
 namespace {
 
-constexpr int kH = 128;                 // heads == MMA M
-constexpr int kDqk = 576;               // latent 512 + rope 64
+constexpr int kH = 128;                  // heads == MMA M
+constexpr int kDqk = 576;                // latent 512 + rope 64
 constexpr int kDv = 512;
 constexpr int kDvHalf = 256;
-constexpr int kRows = 32;               // selected rows per tile (MMA N of S, K of PV)
-constexpr int kKB = kDqk / 64;          // 9 swizzle atoms of 64 columns
-constexpr int kBox = kRows * 128;       // bytes of one 64-column block of a tile (4 KB)
-constexpr int kTile = kKB * kBox;       // 36 KB
-constexpr int kQBytes = kKB * kH * 128; // 144 KB
-constexpr int kStages = 2;
-constexpr int kSoftThreads = 128;
+constexpr int kRows = 64;                // selected rows per tile (MMA N of S, K of PV)
+constexpr int kSplitCol = 256;           // CTA 0: columns [0, 256); CTA 1: [256, 576)
+constexpr int kAtomsMax = 5;             // 64-column swizzle atoms per CTA (CTA 0 uses 4)
+constexpr int kAtomBytes = kRows * 128;  // one atom of one tile: 8 KB
+constexpr int kStageBytes = kAtomsMax * kAtomBytes;  // 40 KB
+constexpr int kStages = 3;
 constexpr int kGatherWarps = 4;
-constexpr int kMmaWarp = kGatherWarps;
-constexpr int kThreads = 32 * kGatherWarps + 32 + kSoftThreads;  // gather warps, MMA warp, 4 softmax warps
-constexpr int kTmemCols = 512;          // O half: cols [0,256), S buffers: [256,288), [288,320)
-constexpr int kSCol = 256;
+constexpr int kMmaWarp = 4;
+constexpr int kSoftThreads = 128;
+constexpr int kThreads = 32 * kGatherWarps + 32 + kSoftThreads;  // 288
+// tensor memory: O half [0, 256), Q columns [256, 256 + 160), S [416, 480)
+constexpr int kTmemCols = 512;
+constexpr int kQCol = 256;
+constexpr int kSCol = 416;
 
 // shared memory map (from a 1024-aligned base)
-constexpr int kOffQ = 0;
-constexpr int kOffKV = kOffQ + kQBytes;
-constexpr int kOffBar = kOffKV + kStages * kTile;
-// barriers: kv_full[2], kv_empty[2], s_full[2], s_empty[2], p_full[2], o_done, q_full, mma_done
-constexpr int kNumBars = 13;
+constexpr int kOffKV = 0;
+constexpr int kOffP = kOffKV + kStages * kStageBytes;  // P: 128 heads x 64 rows bf16, SW128 K-major
+// partial logits, chunk-major [16 x 4 rows][128 heads] fp32: the other CTA's
+// (received by bulk copy) and this CTA's (sent from here)
+constexpr int kXBytes = kH * kRows * 4;
+constexpr int kOffXin = kOffP + kH * kRows * 2;
+constexpr int kOffXout = kOffXin + kXBytes;
+constexpr int kOffBar = kOffXout + kXBytes;
+// barriers: kv_full[3], kv_empty[3], s_full, s_empty, p_full, p_empty, o_done,
+//           q_ready, x_full, x_empty, mma_done, xout_free, xout_written, xin_read
+constexpr int kNumBars = 2 * kStages + 12;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;
 
 struct AttnParams {
+  const uint16_t* q;        // [R][128][576] bf16
   const uint16_t* kv;       // [B][s_max][576] bf16
   const int32_t* idx;       // [R][k]
   const int32_t* ctx_len;   // [B]
   __nv_bfloat16* out;       // [R][128][512]
   float* lse;               // [R][128] or null
   float* part_o;            // [R][S][2][128][256] (splits > 1)
-  float* part_ml;           // [R][S][2][128] : m then l (splits > 1)
+  float* part_ml;           // [R][S][2][2][128]: m then l (splits > 1)
   int n_q, s_max, k, splits, rows_per_split;
   float scale_log2;         // sm_scale * log2(e)
   uint32_t* err;
@@ -81,28 +92,13 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t
   d |= static_cast<uint64_t>(layout & 7u) << 61;
   return d;
 }
-constexpr uint32_t kLayoutSW128 = 2, kLayoutSW64 = 4;
+constexpr uint32_t kLayoutSW128 = 2;
 
 // kind::f16 instruction descriptor with B stored MN-major (N contiguous).
 __host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn(int M, int N) {
   return idesc_bf16_f32(M, N) | (1u << 16);
 }
 
-// TMA row gather: rows r0..r3 of a 2-D tensor map, 64 columns from `col`,
-// written as four consecutive 128-byte swizzled rows at `dst`.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, uint32_t bar, int col, int r0,
-                                            int r1, int r2, int r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ float fast_exp2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
@@ -116,65 +112,169 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* v) {
-  uint32_t u[16];
+__device__ __forceinline__ float4 ld_shared_v4f(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr)
+               : "memory");
+  return v;
+}
+// Distributed shared memory: the address of the same offset in CTA `rank`.
+__device__ __forceinline__ uint32_t map_peer(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st_cluster_v4f(uint32_t raddr, float a, float b, float c, float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(raddr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+// Arrive on an mbarrier of another CTA of the cluster, ordering this
+// thread's earlier shared-memory accesses before the arrival.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t raddr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(raddr) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Whole-warp bounded wait on a barrier that threads of the other CTA arrive on.
+__device__ __forceinline__ bool mbar_wait_warp_cluster(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                                       uint32_t* err) {
+  uint64_t t0 = 0;
+  for (uint32_t i = 0; i < kWaitLimitPolls; ++i) {
+    const bool ok = mbar_try_wait_cluster(bar, parity);
+    if (__all_sync(0xffffffffu, ok)) return true;
+    if ((i & 63u) == 63u) {
+      int stop = 0;
+      if (lane_id() == 0) {
+        const uint64_t now = global_timer_ns();
+        if (t0 == 0) t0 = now;
+        if (*abort_flag) stop = 1;
+        else if (now - t0 > kWaitLimitNs) stop = 2;
+      }
+      stop = __shfl_sync(0xffffffffu, stop, 0);
+      if (stop == 1) return false;
+      if (stop == 2) break;
+    }
+  }
+  if (lane_id() == 0) {
+    *abort_flag = 1;
+    raise_error(err, kErrTimeout);
+  }
+  __syncwarp();
+  return false;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* v) {
+  tmem_st16(taddr, v);
+  tmem_st16(taddr + 16, v + 16);
+}
+__device__ __forceinline__ void tmem_st32f(uint32_t taddr, const float* v) {
+  uint32_t u[32];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) u[i] = __float_as_uint(v[i]);
-  tmem_st16(taddr, u);
-#pragma unroll
-  for (int i = 0; i < 16; ++i) u[i] = __float_as_uint(v[16 + i]);
-  tmem_st16(taddr + 16, u);
+  for (int i = 0; i < 32; ++i) u[i] = __float_as_uint(v[i]);
+  tmem_st32(taddr, u);
 }
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
 }
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 
-__global__ void __launch_bounds__(kThreads, 1)
-    attn_mla_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_kv,
-                       AttnParams P) {
+// Gather this CTA's NA atoms (64 latent columns each) of the tile's 64 rows.
+// Lane l of each gather warp holds the global rows of tile rows l and l + 32.
+template <int NA>
+__device__ __forceinline__ void gather_tile(uint32_t dst0, const char* kv_b, int a0, int cur0, int cur1, int tid) {
+#pragma unroll 4
+  for (int i = 0; i < NA * 4; ++i) {
+    const int x = i * 128 + tid;
+    const int row = x / (NA * 8), cc = x % (NA * 8);
+    const int v0 = __shfl_sync(0xffffffffu, cur0, row & 31);
+    const int v1 = __shfl_sync(0xffffffffu, cur1, row & 31);
+    const int s = row < 32 ? v0 : v1;
+    const int kb = cc >> 3, c = cc & 7;
+    const uint32_t dst = dst0 + kb * kAtomBytes + row * 128 + ((c ^ (row & 7)) << 4);
+    const char* src = kv_b + (s >= 0 ? (static_cast<int64_t>(s) * kDqk + (a0 + kb) * 64) * 2 + c * 16 : 0);
+    cp_async16(dst, src, s >= 0 ? 16u : 0u);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
   const uint32_t bar0 = sbase + kOffBar;
   auto kv_full = [&](int i) { return bar0 + 8u * i; };
-  auto kv_empty = [&](int i) { return bar0 + 8u * (2 + i); };
-  auto s_full = [&](int i) { return bar0 + 8u * (4 + i); };
-  auto s_empty = [&](int i) { return bar0 + 8u * (6 + i); };
-  auto p_full = [&](int i) { return bar0 + 8u * (8 + i); };
-  const uint32_t o_done = bar0 + 8u * 10;
-  const uint32_t q_full = bar0 + 8u * 11;
-  const uint32_t mma_done = bar0 + 8u * 12;
+  auto kv_empty = [&](int i) { return bar0 + 8u * (kStages + i); };
+  const uint32_t s_full = bar0 + 8u * (2 * kStages + 0);
+  const uint32_t s_empty = bar0 + 8u * (2 * kStages + 1);
+  const uint32_t p_full = bar0 + 8u * (2 * kStages + 2);
+  const uint32_t p_empty = bar0 + 8u * (2 * kStages + 3);
+  const uint32_t o_done = bar0 + 8u * (2 * kStages + 4);
+  const uint32_t q_ready = bar0 + 8u * (2 * kStages + 5);
+  const uint32_t x_full = bar0 + 8u * (2 * kStages + 6);
+  const uint32_t x_empty = bar0 + 8u * (2 * kStages + 7);
+  const uint32_t mma_done = bar0 + 8u * (2 * kStages + 8);
+  const uint32_t xout_free = bar0 + 8u * (2 * kStages + 9);
+  const uint32_t xout_written = bar0 + 8u * (2 * kStages + 10);
+  const uint32_t xin_read = bar0 + 8u * (2 * kStages + 11);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = lane_id();
-  // work item
-  const int hv = blockIdx.x & 1;
-  const int sp = (blockIdx.x >> 1) % P.splits;
-  const int r = (blockIdx.x >> 1) / P.splits;
+  const uint32_t crank = cluster_rank();  // 0: latent columns [0, 256); 1: [256, 576)
+  const uint32_t peer = crank ^ 1u;
+  const int a0 = crank == 0 ? 0 : kSplitCol / 64;  // first 64-column atom of this CTA
+  const int natoms = crank == 0 ? kSplitCol / 64 : (kDqk - kSplitCol) / 64;
+  // work item of the cluster
+  const int item = blockIdx.x >> 1;
+  const int sp = item % P.splits;
+  const int r = item / P.splits;
   const int b = r / P.n_q;
   const int L = min(max(__ldg(P.ctx_len + b), 0), P.s_max);
   const int row0 = sp * P.rows_per_split;
   const int nrows = max(0, min(P.rows_per_split, P.k - row0));
   const int T = (nrows + kRows - 1) / kRows;
   const int32_t* sel = P.idx + static_cast<int64_t>(r) * P.k + row0;
-  const uint32_t p_off = hv == 0 ? 4u * kBox : 0u;    // P lives where this half's V does not
-  const uint32_t v_off = hv == 0 ? 0u : 4u * kBox;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(kv_full(i), kGatherWarps);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(kv_full(i), 32 * kGatherWarps);
       mbar_init(kv_empty(i), 1);
-      mbar_init(s_full(i), 1);
-      mbar_init(s_empty(i), kSoftThreads);
-      mbar_init(p_full(i), kSoftThreads);
     }
+    mbar_init(s_full, 1);
+    mbar_init(s_empty, kSoftThreads);
+    mbar_init(p_full, kSoftThreads);
+    mbar_init(p_empty, 1);
     mbar_init(o_done, 1);
-    mbar_init(q_full, 1);
+    mbar_init(q_ready, kSoftThreads);
+    mbar_init(x_full, 1);   // own arm (expect_tx) + the other CTA's bulk copy
+    mbar_init(x_empty, 1);  // arrived by the other CTA once it has read our partial
     mbar_init(mma_done, 1);
+    mbar_init(xout_free, 1);
+    mbar_init(xout_written, kSoftThreads);
+    mbar_init(xin_read, kSoftThreads);
+    if (T > 0) mbar_arrive_expect_tx(x_full, kXBytes);  // armed for tile 0
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -185,107 +285,74 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
+  cluster_sync_all();  // both CTAs' barriers exist before any remote arrival
   const uint32_t tmem = *tmem_slot;
 
   if (warp < kGatherWarps) {
-    // -------------------------------------------------- gather (TMA) --
+    // --------------------------------------------------- gather (cp.async) --
+    const int tid = threadIdx.x;
+    const char* kv_b = reinterpret_cast<const char*>(P.kv) + static_cast<int64_t>(b) * P.s_max * kDqk * 2;
     bool bad = false;
-    // lane i holds the (flattened) row of tile row i; the next tile's
-    // indices are fetched before this tile's gathers go out
-    int nxt = (lane < nrows) ? __ldg(sel + lane) : -1;
-    const int grp = lane & 7;  // this lane gathers rows 4*grp .. 4*grp+3
+    int nx0 = (lane < nrows) ? __ldg(sel + lane) : -1;
+    int nx1 = (lane + 32 < nrows) ? __ldg(sel + lane + 32) : -1;
     for (int j = 0; j < T; ++j) {
-      const int st = j & 1;
-      int cur = nxt;
-      if (cur >= L) { bad = true; cur = -1; }
-      const int grow = cur >= 0 ? b * P.s_max + cur : -1;  // row -1 reads zeros
+      const int st = j % kStages;
+      int cur0 = nx0, cur1 = nx1;
+      if (cur0 >= L) { bad = true; cur0 = -1; }
+      if (cur1 >= L) { bad = true; cur1 = -1; }
       const int jn = (j + 1) * kRows + lane;
-      nxt = (j + 1 < T && jn < nrows) ? __ldg(sel + jn) : -1;
-      const int r0 = __shfl_sync(0xffffffffu, grow, 4 * grp + 0);
-      const int r1 = __shfl_sync(0xffffffffu, grow, 4 * grp + 1);
-      const int r2 = __shfl_sync(0xffffffffu, grow, 4 * grp + 2);
-      const int r3 = __shfl_sync(0xffffffffu, grow, 4 * grp + 3);
-      if (!mbar_wait_warp(kv_empty(st), ((j >> 1) & 1) ^ 1, abort_flag, P.err)) break;
-      // warp w gathers the 64-column blocks w, w+4, w+8 of the tile; each
-      // warp's first lane adds its share of the bytes to the stage's barrier
-      int nblk = 0;
-      for (int kb = warp; kb < kKB; kb += kGatherWarps) ++nblk;
-      if (lane == 0) mbar_arrive_expect_tx(kv_full(st), nblk * 8 * 512);
-      __syncwarp();
-      const uint32_t dst0 = sbase + kOffKV + st * kTile + grp * 512;
-      for (int kb = warp + kGatherWarps * (lane >> 3); kb < kKB && (lane >> 3) < 3; kb += kGatherWarps * 4)
-        tma_gather4(dst0 + kb * kBox, &tmap_kv, kv_full(st), kb * 64, r0, r1, r2, r3);
+      nx0 = (j + 1 < T && jn < nrows) ? __ldg(sel + jn) : -1;
+      nx1 = (j + 1 < T && jn + 32 < nrows) ? __ldg(sel + jn + 32) : -1;
+      if (!mbar_wait_warp(kv_empty(st), ((j / kStages) & 1) ^ 1, abort_flag, P.err)) break;
+      const uint32_t dst0 = sbase + kOffKV + st * kStageBytes;
+      if (crank == 0) gather_tile<kSplitCol / 64>(dst0, kv_b, a0, cur0, cur1, tid);
+      else gather_tile<(kDqk - kSplitCol) / 64>(dst0, kv_b, a0, cur0, cur1, tid);
+      cp_async_arrive(kv_full(st));
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
     if (__any_sync(0xffffffffu, bad) && lane == 0) raise_error(P.err, kErrBadIndex);
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------- MMA issue --
     if (lane == 0) {
-      const uint32_t qaddr = sbase + kOffQ;
-      mbar_arrive_expect_tx(q_full, kQBytes);
-#pragma unroll 1
-      for (int kb = 0; kb < kKB; ++kb) tma_load_2d(qaddr + kb * kH * 128, &tmap_q, q_full, kb * 64, r * kH);
       constexpr uint32_t idesc_s = idesc_bf16_f32(kH, kRows);
       constexpr uint32_t idesc_o = idesc_bf16_f32_bmn(kH, kDvHalf);
-      const uint64_t q_desc0 = sdesc(qaddr, 16, 1024, kLayoutSW128);
-      const uint64_t kv_desc0 = sdesc(sbase + kOffKV, 16, 1024, kLayoutSW128);
-      const uint64_t p_desc0 = sdesc(sbase + kOffKV + p_off, 16, 512, kLayoutSW64);
-      const uint64_t v_desc0 = sdesc(sbase + kOffKV + v_off, kBox, 1024, kLayoutSW128);
-      bool ok = mbar_wait(q_full, 0, abort_flag, P.err);
-      auto do_pv = [&](int i) -> bool {
-        if (!mbar_wait(p_full(i & 1), (i >> 1) & 1, abort_flag, P.err)) return false;
-        tc_fence_after_sync();
-        const uint64_t st_off = static_cast<uint64_t>(((i & 1) * kTile) >> 4);
-#pragma unroll
-        for (int kk = 0; kk < kRows / 16; ++kk)
-          tc_mma_f16(tmem, p_desc0 + st_off + ((kk * 32) >> 4), v_desc0 + st_off + ((kk * 16 * 128) >> 4), idesc_o,
-                     (i > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(kv_empty(i & 1));
-        tc_commit(o_done);
-        return true;
-      };
-      // Issue whichever of QK(nq) / PV(np) is ready (PV first), so the value
-      // product of a tile -- which frees its stage for the next gather -- never
-      // waits behind the logits of a tile whose rows are still in flight.
-      // S(j) = Q K(j)^T is issued in kQkParts chunks; a P(i) that becomes
-      // ready is issued between chunks, so the value product of a tile (which
-      // frees its stage for the next gather) never queues behind a whole QK.
-      constexpr int kQkMma = kDqk / 16;  // 36
-      constexpr int kQkParts = 3;
-      auto issue_qk_part = [&](int j, int part) {
-        const int st = j & 1;
-        if (part == 0) tc_fence_after_sync();
-        const uint32_t d = tmem + kSCol + st * kRows;
-        const uint64_t kv0 = kv_desc0 + static_cast<uint64_t>((st * kTile) >> 4);
-#pragma unroll
-        for (int q = 0; q < kQkMma / kQkParts; ++q) {
-          const int kk = part * (kQkMma / kQkParts) + q;
-          // descriptor start addresses advance in 16-byte units
-          const uint32_t a_off = (kk >> 2) * kH * 128 + (kk & 3) * 32;
-          const uint32_t b_off = (kk >> 2) * kBox + (kk & 3) * 32;
-          tc_mma_f16(d, q_desc0 + (a_off >> 4), kv0 + (b_off >> 4), idesc_s, kk > 0 ? 1u : 0u);
-        }
-        if (part == kQkParts - 1) tc_commit(s_full(st));
-      };
-      int nq = 0, np = 0, qpart = 0;  // QK(nq) has issued qpart chunks
+      const uint64_t kv_desc0 = sdesc(sbase + kOffKV, 16, 1024, kLayoutSW128);      // K-major rows (logits)
+      const uint64_t v_desc0 = sdesc(sbase + kOffKV, kAtomBytes, 1024, kLayoutSW128);  // MN-major columns (value)
+      const uint64_t p_desc0 = sdesc(sbase + kOffP, 16, 1024, kLayoutSW128);
+      const uint32_t q_t = tmem + kQCol, s_t = tmem + kSCol;
+      bool ok = mbar_wait(q_ready, 0, abort_flag, P.err);
+      int nq = 0, np = 0;
       uint64_t t0 = 0;
       uint32_t spins = 0;
       while (ok && np < T) {
-        if (np < nq && mbar_test_wait(p_full(np & 1), (np >> 1) & 1)) {
-          ok = do_pv(np);
+        // O += P(np) V(np) as soon as P is written (frees the tile's stage)
+        if (np < nq && mbar_test_wait(p_full, np & 1)) {
+          tc_fence_after_sync();
+          const uint64_t st_off = static_cast<uint64_t>(((np % kStages) * kStageBytes) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < kRows / 16; ++kk)
+            tc_mma_f16(tmem, p_desc0 + ((kk * 32) >> 4), v_desc0 + st_off + ((kk * 16 * 128) >> 4), idesc_o,
+                       (np > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(kv_empty(np % kStages));
+          tc_commit(p_empty);
+          tc_commit(o_done);
           ++np;
           spins = 0;
           continue;
         }
-        if (qpart > 0) {
-          issue_qk_part(nq, qpart);
-          if (++qpart == kQkParts) { qpart = 0; ++nq; }
-          spins = 0;
-          continue;
-        }
-        if (nq < T && mbar_test_wait(kv_full(nq & 1), (nq >> 1) & 1) &&
-            mbar_test_wait(s_empty(nq & 1), ((nq >> 1) & 1) ^ 1)) {
-          issue_qk_part(nq, 0);
-          qpart = 1;
+        // S(nq) = Q_c K_c(nq)^T once its rows landed and S(nq-1) was read
+        if (nq < T && mbar_test_wait(kv_full(nq % kStages), (nq / kStages) & 1) &&
+            mbar_test_wait(s_empty, (nq & 1) ^ 1)) {
+          fence_proxy_async_smem();  // cp.async (generic proxy) writes -> tensor-core reads
+          tc_fence_after_sync();
+          const uint64_t kvs = kv_desc0 + static_cast<uint64_t>(((nq % kStages) * kStageBytes) >> 4);
+          const int nk = natoms * 4;
+          for (int kk = 0; kk < nk; ++kk) {
+            const uint32_t b_off = (kk >> 2) * kAtomBytes + (kk & 3) * 32;
+            tc_mma_f16_ts(s_t, q_t + kk * 8, kvs + (b_off >> 4), idesc_s, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(s_full);
+          ++nq;
           spins = 0;
           continue;
         }
@@ -305,30 +372,109 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(mma_done, 0, &never, P.err);
     }
   } else {
-    // ------------------------------------------------ softmax + output --
+    // ------------------------------------- Q to TMEM, softmax, output --
     const int quarter = warp & 3;
-    const int h = quarter * 32 + lane;                       // head == TMEM lane
+    const int h = quarter * 32 + lane;  // head == TMEM lane
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    {
+      // this CTA's columns of q[r, h, :] as packed bf16 pairs (element 2i in
+      // the low half of column i)
+      const uint4* qs = reinterpret_cast<const uint4*>(P.q + (static_cast<int64_t>(r) * kH + h) * kDqk + a0 * 64);
+      for (int c = 0; c < natoms * 64 / 32; ++c) {
+        uint32_t u[16];
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const uint4 x = __ldg(qs + c * 4 + v);
+          u[4 * v + 0] = x.x;
+          u[4 * v + 1] = x.y;
+          u[4 * v + 2] = x.z;
+          u[4 * v + 3] = x.w;
+        }
+        tmem_st16(tl + kQCol + c * 16, u);
+      }
+      tmem_st_wait();
+      tc_fence_before_sync();
+      mbar_arrive(q_ready);
+    }
+    const uint32_t xin = sbase + kOffXin, xout = sbase + kOffXout;
+    const uint32_t xin_peer = map_peer(xin, peer);
+    const uint32_t x_full_peer = map_peer(x_full, peer);
+    const uint32_t x_empty_peer = map_peer(x_empty, peer);
+    const bool leader = (h == 0);  // issues the bulk copy and the cross-CTA signals
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    int sidx_next = (lane < nrows) ? __ldg(sel + lane) : -1;
+    int nx0 = (lane < nrows) ? __ldg(sel + lane) : -1;
+    int nx1 = (lane + 32 < nrows) ? __ldg(sel + lane + 32) : -1;
     for (int j = 0; j < T; ++j) {
-      const int st = j & 1;
       // which rows of this tile are real (indices fetched one tile ahead)
-      const int sidx = sidx_next;
+      const uint32_t valid0 = __ballot_sync(0xffffffffu, nx0 >= 0 && nx0 < L);
+      const uint32_t valid1 = __ballot_sync(0xffffffffu, nx1 >= 0 && nx1 < L);
       const int jn = (j + 1) * kRows + lane;
-      sidx_next = (j + 1 < T && jn < nrows) ? __ldg(sel + jn) : -1;
-      const uint32_t valid = __ballot_sync(0xffffffffu, sidx >= 0 && sidx < L);
-      if (!mbar_wait_warp(s_full(st), (j >> 1) & 1, abort_flag, P.err)) { ok = false; break; }
+      nx0 = (j + 1 < T && jn < nrows) ? __ldg(sel + jn) : -1;
+      nx1 = (j + 1 < T && jn + 32 < nrows) ? __ldg(sel + jn + 32) : -1;
+      if (!mbar_wait_warp(s_full, j & 1, abort_flag, P.err)) { ok = false; break; }
       tc_fence_after_sync();
       float s[kRows];
-      tmem_ld32(tl + kSCol + st * kRows, s);
+      tmem_ld32(tl + kSCol, s);
+      tmem_ld32(tl + kSCol + 32, s + 32);
       tc_fence_before_sync();
-      mbar_arrive(s_empty(st));
+      mbar_arrive(s_empty);
+      // swap partial logits with the other CTA: stage mine locally, one
+      // thread copies the 32 KB into the other CTA's receive buffer ...
+      if (leader && j >= 1) {
+        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // previous copy has read xout
+        mbar_arrive(xout_free);
+      }
+      if (!mbar_wait_warp(xout_free, (j & 1) ^ 1, abort_flag, P.err)) { ok = false; break; }
+#pragma unroll
+      for (int c = 0; c < kRows / 4; ++c)
+        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(xout + (c * kH + h) * 16), "f"(s[4 * c]),
+                     "f"(s[4 * c + 1]), "f"(s[4 * c + 2]), "f"(s[4 * c + 3])
+                     : "memory");
+      fence_proxy_async_smem();
+      mbar_arrive(xout_written);
+      if (leader) {
+        bool go = mbar_wait(xout_written, j & 1, abort_flag, P.err);
+        if (go && j >= 1) {
+          // the other CTA has read our previous partial
+          go = false;
+          const uint64_t t0 = global_timer_ns();
+          for (uint32_t it = 0; it < kWaitLimitPolls; ++it) {
+            if (mbar_try_wait_cluster(x_empty, (j - 1) & 1)) { go = true; break; }
+            if ((it & 63u) == 63u && (*abort_flag || global_timer_ns() - t0 > kWaitLimitNs)) break;
+          }
+          if (!go && !*abort_flag) { *abort_flag = 1; raise_error(P.err, kErrTimeout); }
+        }
+        if (go) {
+          asm volatile(
+              "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n\t"
+              "cp.async.bulk.commit_group;" ::"r"(xin_peer),
+              "r"(xout), "r"(kXBytes), "r"(x_full_peer)
+              : "memory");
+        }
+      }
+      // ... and the other CTA's partial arrives in ours: S = S_0 + S_1 on both sides
+      if (!mbar_wait_warp_cluster(x_full, j & 1, abort_flag, P.err)) { ok = false; break; }
+#pragma unroll
+      for (int c = 0; c < kRows / 4; ++c) {
+        const float4 v = ld_shared_v4f(xin + (c * kH + h) * 16);
+        s[4 * c] += v.x;
+        s[4 * c + 1] += v.y;
+        s[4 * c + 2] += v.z;
+        s[4 * c + 3] += v.w;
+      }
+      mbar_arrive(xin_read);
+      if (leader) {
+        if (mbar_wait(xin_read, j & 1, abort_flag, P.err)) {
+          if (j + 1 < T) mbar_arrive_expect_tx(x_full, kXBytes);  // arm for the next tile
+          mbar_arrive_remote(x_empty_peer);
+        }
+      }
       float mt = -INFINITY;
 #pragma unroll
       for (int i = 0; i < kRows; ++i) {
-        s[i] = ((valid >> i) & 1u) ? s[i] * P.scale_log2 : -INFINITY;
+        const bool v = ((i < 32 ? (valid0 >> i) : (valid1 >> (i - 32))) & 1u) != 0;
+        s[i] = v ? s[i] * P.scale_log2 : -INFINITY;
         mt = fmaxf(mt, s[i]);
       }
       // move the running max only when the tile max exceeds it by > 8 (base 2)
@@ -345,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(tl + c, o);
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] *= f;
-          tmem_st32(tl + c, o);
+          tmem_st32f(tl + c, o);
         }
         tmem_st_wait();
       }
@@ -353,26 +499,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (m_run != -INFINITY) l_run *= exp2f(m_run - mt);
         m_run = mt;
       }
-      // P = 2^(s - m) in bf16, 64 bytes per head, 64-byte-swizzled K-major
-      const uint32_t prow = sbase + kOffKV + st * kTile + p_off + (h >> 3) * 512 + (h & 7) * 64;
-      const int sw = (h >> 1) & 3;
+      // P = 2^(s - m) in bf16: one 128-byte row per head, 128-byte-swizzled K-major
+      if (j >= 1 && !mbar_wait_warp(p_empty, (j - 1) & 1, abort_flag, P.err)) { ok = false; break; }
+      const uint32_t prow = sbase + kOffP + (h >> 3) * 1024 + (h & 7) * 128;
       float psum = 0.f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < kRows / 8; ++c) {
         float p[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           p[e] = (m_run == -INFINITY) ? 0.f : fast_exp2(s[c * 8 + e] - m_run);
           psum += p[e];
         }
-        st_shared_v4(prow + ((c ^ sw) << 4), pack_bf16(p[0], p[1]), pack_bf16(p[2], p[3]), pack_bf16(p[4], p[5]),
-                     pack_bf16(p[6], p[7]));
+        st_shared_v4(prow + ((c ^ (h & 7)) << 4), pack_bf16(p[0], p[1]), pack_bf16(p[2], p[3]),
+                     pack_bf16(p[4], p[5]), pack_bf16(p[6], p[7]));
       }
       l_run += psum;
       fence_proxy_async_smem();
       tc_fence_before_sync();
-      mbar_arrive(p_full(st));
+      mbar_arrive(p_full);
     }
+    if (leader) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     // ------------------------------------------------------------ output --
     if (ok && T >= 1) ok = mbar_wait_warp(o_done, (T - 1) & 1, abort_flag, P.err);
     if (ok) {
@@ -380,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t rh = static_cast<int64_t>(r) * kH + h;
       if (P.splits == 1) {
         const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-        __nv_bfloat16* dst = P.out + rh * kDv + hv * kDvHalf;
+        __nv_bfloat16* dst = P.out + rh * kDv + crank * kDvHalf;
 #pragma unroll 1
         for (int c = 0; c < kDvHalf; c += 32) {
           float o[32];
@@ -397,11 +544,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<uint4*>(dst + c + q * 8) = v;
           }
         }
-        if (P.lse != nullptr && hv == 0)
+        if (P.lse != nullptr && crank == 0)
           P.lse[rh] = l_run > 0.f ? (m_run + log2f(l_run)) * 0.6931471805599453f : -INFINITY;
       } else {
-        const int64_t item = (static_cast<int64_t>(r) * P.splits + sp) * 2 + hv;
-        float* dst = P.part_o + (item * kH + h) * kDvHalf;
+        const int64_t it = (static_cast<int64_t>(r) * P.splits + sp) * 2 + crank;
+        float* dst = P.part_o + (it * kH + h) * kDvHalf;
 #pragma unroll 1
         for (int c = 0; c < kDvHalf; c += 32) {
           float o[32];
@@ -412,8 +559,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int q = 0; q < 8; ++q)
             *reinterpret_cast<float4*>(dst + c + q * 4) = make_float4(o[q * 4], o[q * 4 + 1], o[q * 4 + 2], o[q * 4 + 3]);
         }
-        P.part_ml[(item * 2 + 0) * kH + h] = m_run;
-        P.part_ml[(item * 2 + 1) * kH + h] = l_run;
+        P.part_ml[(it * 2 + 0) * kH + h] = m_run;
+        P.part_ml[(it * 2 + 1) * kH + h] = l_run;
       }
     }
   }
@@ -424,6 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after_sync();
     tmem_dealloc(tmem, kTmemCols);
   }
+  cluster_sync_all();  // no CTA leaves while the other may still touch its shared memory
 }
 }  // namespace
 }  // namespace dsa
@@ -432,12 +580,11 @@ namespace dsa {
 namespace {
 
 constexpr int kMaxSplits = 16;
-
 constexpr int kCombineHeads = 8;  // heads per combine block
 
 // Merge the per-split partial outputs of each query: O = sum_i 2^(m_i - M) O_i
 // / sum_i 2^(m_i - M) l_i with M = max_i m_i (base-2 log-sum-exp combine).
-// Block = (query, group of 8 heads); 256 threads, 4 output columns each step.
+// Block = (query, group of 8 heads); 256 threads, 4 output columns a step.
 __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restrict__ part_o,
                                                            const float* __restrict__ part_ml, int splits,
                                                            __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
@@ -449,16 +596,16 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
     const int h = h0 + tid;
     float M = -INFINITY;
     for (int i = 0; i < splits; ++i) {
-      const int64_t item = (static_cast<int64_t>(r) * splits + i) * 2;
-      const float m = part_ml[(item * 2 + 0) * kH + h];
-      const float l = part_ml[(item * 2 + 1) * kH + h];
+      const int64_t it = (static_cast<int64_t>(r) * splits + i) * 2;
+      const float m = part_ml[(it * 2 + 0) * kH + h];
+      const float l = part_ml[(it * 2 + 1) * kH + h];
       if (l > 0.f) M = fmaxf(M, m);
     }
     float Ls = 0.f;
     for (int i = 0; i < splits; ++i) {
-      const int64_t item = (static_cast<int64_t>(r) * splits + i) * 2;
-      const float m = part_ml[(item * 2 + 0) * kH + h];
-      const float l = part_ml[(item * 2 + 1) * kH + h];
+      const int64_t it = (static_cast<int64_t>(r) * splits + i) * 2;
+      const float m = part_ml[(it * 2 + 0) * kH + h];
+      const float l = part_ml[(it * 2 + 1) * kH + h];
       const float wgt = (l > 0.f) ? exp2f(m - M) : 0.f;
       coef[i][tid] = wgt;
       Ls += wgt * l;
@@ -470,8 +617,8 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
   }
   __syncthreads();
 #pragma unroll
-  for (int it = 0; it < kCombineHeads * (kDv / 4) / 256; ++it) {
-    const int x = it * 256 + tid;
+  for (int itr = 0; itr < kCombineHeads * (kDv / 4) / 256; ++itr) {
+    const int x = itr * 256 + tid;
     const int hl = x / (kDv / 4);
     const int c4 = x % (kDv / 4);
     const int h = h0 + hl;
@@ -479,8 +626,8 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
     const int cc = (c4 % (kDvHalf / 4)) * 4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int i = 0; i < splits; ++i) {
-      const int64_t item = (static_cast<int64_t>(r) * splits + i) * 2 + hv;
-      const float4 o = __ldg(reinterpret_cast<const float4*>(part_o + (item * kH + h) * kDvHalf + cc));
+      const int64_t it = (static_cast<int64_t>(r) * splits + i) * 2 + hv;
+      const float4 o = __ldg(reinterpret_cast<const float4*>(part_o + (it * kH + h) * kDvHalf + cc));
       const float c = coef[i][hl];
       acc.x = fmaf(c, o.x, acc.x);
       acc.y = fmaf(c, o.y, acc.y);
@@ -498,6 +645,8 @@ struct SplitPlan {
   int splits, rows_per_split;
 };
 
+// Splits of each query's selected list so that clusters (2 SMs each) cover
+// the GPU: none when the queries alone fill it.
 SplitPlan plan_splits(int64_t R, int k, int num_sms) {
   SplitPlan p;
   int s = 1;
@@ -508,6 +657,12 @@ SplitPlan plan_splits(int64_t R, int k, int num_sms) {
   p.rows_per_split = std::max(rps, kRows);
   p.splits = (k + p.rows_per_split - 1) / p.rows_per_split;
   return p;
+}
+
+size_t scratch_bytes(int64_t R, const SplitPlan& p) {
+  if (p.splits <= 1) return 0;
+  const size_t items = static_cast<size_t>(R) * p.splits * 2;
+  return items * kH * kDvHalf * 4 + items * 2 * kH * 4;
 }
 
 }  // namespace
@@ -521,10 +676,13 @@ size_t attn_workspace_bytes(int B, int n_q, int H, int d_qk, int d_v, int KVH, i
   const int64_t R = static_cast<int64_t>(B) * n_q;
   // the split plan depends on the SM count; size for the largest plan any
   // B200-class part (<= 256 SMs) would pick
-  const SplitPlan p = plan_splits(R, k, 256);
-  if (p.splits <= 1) return 0;
-  const size_t items = static_cast<size_t>(R) * p.splits * 2;
-  return items * kH * kDvHalf * 4 + items * 2 * kH * 4;
+  return scratch_bytes(R, plan_splits(R, k, 256));
+}
+
+size_t attn_scratch_bytes(int B, int n_q, int k, int num_sms) {
+  const int64_t R = static_cast<int64_t>(B) * n_q;
+  if (R == 0) return 0;
+  return scratch_bytes(R, plan_splits(R, k, num_sms));
 }
 
 dsa_status_t attn_tc(const AttnArgs& a) {
@@ -534,6 +692,7 @@ dsa_status_t attn_tc(const AttnArgs& a) {
   const SplitPlan p = plan_splits(R, a.k, num_sms);
   if (R * p.splits * 2 > INT32_MAX) return DSA_ERR_UNSUPPORTED;
   AttnParams P;
+  P.q = static_cast<const uint16_t*>(a.q);
   P.kv = static_cast<const uint16_t*>(a.kv);
   P.idx = a.idx;
   P.ctx_len = a.ctx_len;
@@ -549,19 +708,12 @@ dsa_status_t attn_tc(const AttnArgs& a) {
   P.part_o = nullptr;
   P.part_ml = nullptr;
   if (p.splits > 1) {
-    const size_t items = static_cast<size_t>(R) * p.splits * 2;
-    const size_t need = items * kH * kDvHalf * 4 + items * 2 * kH * 4;
+    const size_t need = scratch_bytes(R, p);
     if (a.ws == nullptr || a.ws_bytes < need) return DSA_ERR_WORKSPACE;
+    const size_t items = static_cast<size_t>(R) * p.splits * 2;
     P.part_o = static_cast<float*>(a.ws);
     P.part_ml = P.part_o + items * kH * kDvHalf;
   }
-  CUtensorMap tmq;
-  if (!make_tmap_2d(&tmq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDqk, static_cast<uint64_t>(R) * kH, 64, kH))
-    return DSA_ERR_CUDA;
-  CUtensorMap tmkv;
-  if (!make_tmap_2d(&tmkv, a.kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDqk, static_cast<uint64_t>(a.B) * a.s_max, 64,
-                    1))
-    return DSA_ERR_CUDA;
   static bool attr_done[64] = {};
   if (a.device < 64 && !attr_done[a.device]) {
     if (cudaFuncSetAttribute(attn_mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
@@ -569,28 +721,25 @@ dsa_status_t attn_tc(const AttnArgs& a) {
       return DSA_ERR_CUDA;
     attr_done[a.device] = true;
   }
-  const unsigned grid = static_cast<unsigned>(R * p.splits * 2);
-  attn_mla_tc_kernel<<<grid, kThreads, kSmemBytes, a.stream>>>(tmq, tmkv, P);
-  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(R * p.splits * 2), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = a.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, attn_mla_tc_kernel, P) != cudaSuccess) return DSA_ERR_CUDA;
   if (p.splits > 1) {
-    attn_combine_kernel<<<dim3(static_cast<unsigned>(R), kH / kCombineHeads), 256, 0, a.stream>>>(P.part_o, P.part_ml, p.splits, P.out,
-                                                                       a.lse);
+    attn_combine_kernel<<<dim3(static_cast<unsigned>(R), kH / kCombineHeads), 256, 0, a.stream>>>(
+        P.part_o, P.part_ml, p.splits, P.out, a.lse);
     if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
   }
   return DSA_OK;
 }
 
-}  // namespace dsa
-
-namespace dsa {
-// Exact scratch bytes the tensor-core attention needs for this shape on a
-// device with `num_sms` SMs (0 when it writes its output directly).
-size_t attn_scratch_bytes(int B, int n_q, int k, int num_sms) {
-  const int64_t R = static_cast<int64_t>(B) * n_q;
-  if (R == 0) return 0;
-  const SplitPlan p = plan_splits(R, k, num_sms);
-  if (p.splits <= 1) return 0;
-  const size_t items = static_cast<size_t>(R) * p.splits * 2;
-  return items * kH * kDvHalf * 4 + items * 2 * kH * 4;
-}
 }  // namespace dsa

@@ -76,12 +76,19 @@ def get(name: str, **overrides) -> Workload:
     return replace(wl, **overrides) if overrides else wl
 
 
+_DRAW = 1 << 26  # elements per fp32 draw (bounds the temporary buffer)
+
+
 def _randn_into(out: torch.Tensor, gen: torch.Generator, std: float):
-    """Fill ``out`` with N(0, std^2) drawn in fp32, one leading-axis slice at a time."""
+    """Fill ``out`` with N(0, std^2) drawn in fp32, in consecutive pieces of at
+    most 2^26 elements (one leading-axis slice at a time)."""
     flat = out.view(out.shape[0], -1)
     for i in range(flat.shape[0]):
-        x = torch.randn(flat.shape[1], generator=gen, device=out.device, dtype=torch.float32)
-        flat[i].copy_(x.mul_(std))
+        row = flat[i]
+        for j in range(0, row.numel(), _DRAW):
+            n = min(_DRAW, row.numel() - j)
+            x = torch.randn(n, generator=gen, device=out.device, dtype=torch.float32)
+            row[j:j + n].copy_(x.mul_(std))
 
 
 def make_inputs(wl: Workload, device="cpu", seed: int = 0, attention: bool = True):
