@@ -287,11 +287,25 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
     int ab = 0, wb = 0;
     uint32_t aph = 0;
     int last_bg = -1;
+    float wreg[kQG == 1 ? kHI : 1];
     UnitIter it = iter_begin(S, cta);
     Unit U;
     while (iter_next<kQG>(S, it, cta, U, ctx_len, q_pos0)) {
       if (U.kt_end <= U.kt0) continue;
-      if (U.kt_comp > U.kt0) {
+      if (kQG == 1 && U.kt_comp > U.kt0) {
+        // one query: its head weights live in registers
+        const int bg = U.b * S.G + U.t0;
+        if (bg != last_bg) {
+          const int64_t o = (static_cast<int64_t>(U.b) * S.n_q + U.t0) * kHI;
+#pragma unroll
+          for (int h = 0; h < kHI; ++h) {
+            float v = __ldg(w + o + h) * idx_scale;
+            if (kFP8) v *= __ldg(q_scale + o + h);
+            wreg[h] = v;
+          }
+          last_bg = bg;
+        }
+      } else if (U.kt_comp > U.kt0) {
         const int bg = U.b * S.G + U.t0 / kQG;
         if (bg != last_bg) {
           // head weights of this query block, with the score scale (and the
@@ -323,6 +337,23 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
         float ks = 1.f;
         if (kFP8 && s < U.L) ks = __ldg(k_scale + static_cast<int64_t>(U.b) * S.s_max + s);
         const uint32_t tl = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(ab * C::N);
+        if constexpr (kQG == 1 && kHI == 64) {
+          float v0[32], v1[32];
+          tmem_ld32x2(tl, tl + 32, v0, v1);
+          float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+#pragma unroll
+          for (int x = 0; x < 32; x += 2) {
+            acc0 = fmaf(wreg[x], fmaxf(v0[x], 0.f), acc0);
+            acc1 = fmaf(wreg[x + 1], fmaxf(v0[x + 1], 0.f), acc1);
+            acc2 = fmaf(wreg[32 + x], fmaxf(v1[x], 0.f), acc2);
+            acc3 = fmaf(wreg[33 + x], fmaxf(v1[x + 1], 0.f), acc3);
+          }
+          if (s < U.L) {
+            const int p = U.p0 + U.t0;
+            scores[(static_cast<int64_t>(U.b) * S.n_q + U.t0) * ld + s] =
+                (s <= p) ? ((acc0 + acc1) + (acc2 + acc3)) * ks : -INFINITY;
+          }
+        } else
 #pragma unroll 1
         for (int j = jbeg; j < jend; ++j) {
           float acc0 = 0.f, acc1 = 0.f;

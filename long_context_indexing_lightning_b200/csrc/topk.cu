@@ -25,9 +25,8 @@ namespace cg = cooperative_groups;
 namespace dsa {
 namespace {
 
-constexpr int kThreads = 1024;
-constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 2048;
+constexpr int kMaxWarps = 32;
 constexpr int kMaxCluster = 16;
 
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v) {
@@ -41,16 +40,18 @@ __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v) {
 }
 
 // Block-wide exclusive scan of one value per thread; the block total goes to
-// *total.  Uses `wsum` (kWarps + 1 words).
+// *total.  Uses `wsum` (kMaxWarps + 1 words).
+template <int kThreads>
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* wsum, uint32_t* total) {
+  constexpr int kWarps = kThreads / 32;
   const int lane = lane_id(), warp = threadIdx.x >> 5;
   const uint32_t incl = warp_incl_scan(v);
   if (lane == 31) wsum[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    const uint32_t x = wsum[lane];
+    const uint32_t x = lane < kWarps ? wsum[lane] : 0u;
     const uint32_t xi = warp_incl_scan(x);
-    wsum[lane] = xi - x;
+    if (lane < kWarps) wsum[lane] = xi - x;
     if (lane == 31) wsum[kWarps] = xi;
   }
   __syncthreads();
@@ -60,14 +61,14 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* wsum, 
   return res;
 }
 
-template <int PER>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int PER, int kThreads>
+__global__ void __launch_bounds__(kThreads, 1024 / kThreads)
     topk_cluster_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ ctx_len,
                         const int32_t* __restrict__ q_pos0, int t_off, int n_q, int s_max, int k,
                         int32_t* __restrict__ idx) {
   __shared__ uint32_t hist[3][kBins];
   __shared__ uint32_t merged[kBins];
-  __shared__ uint32_t wsum[kWarps + 1];
+  __shared__ uint32_t wsum[kMaxWarps + 1];
   __shared__ uint32_t s_digit, s_above;
   __shared__ uint32_t s_tot[2];
 
@@ -128,19 +129,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
     {
-      // bins from the top, two per thread; a block prefix sum finds the bin
-      // holding the remaining-th largest key
-      const int b0 = kBins - 1 - 2 * tid;
-      const uint32_t c0 = merged[b0], c1 = merged[b0 - 1];
+      // bins from the top, kBins / kThreads per thread; a block prefix sum
+      // finds the bin holding the remaining-th largest key
+      constexpr int kPerT = kBins / kThreads;
+      const int btop = kBins - 1 - kPerT * tid;
+      uint32_t cnt[kPerT];
+      uint32_t mine = 0;
+#pragma unroll
+      for (int q = 0; q < kPerT; ++q) {
+        cnt[q] = merged[btop - q];
+        mine += cnt[q];
+      }
       uint32_t tot;
-      const uint32_t excl = block_excl_scan(c0 + c1, wsum, &tot);
-      if (excl < remaining && remaining <= excl + c0 + c1) {
-        if (remaining <= excl + c0) {
-          s_digit = static_cast<uint32_t>(b0);
-          s_above = excl;
-        } else {
-          s_digit = static_cast<uint32_t>(b0 - 1);
-          s_above = excl + c0;
+      const uint32_t excl = block_excl_scan<kThreads>(mine, wsum, &tot);
+      if (excl < remaining && remaining <= excl + mine) {
+        uint32_t cum = excl;
+#pragma unroll
+        for (int q = 0; q < kPerT; ++q) {
+          if (cum < remaining && remaining <= cum + cnt[q]) {
+            s_digit = static_cast<uint32_t>(btop - q);
+            s_above = cum;
+          }
+          cum += cnt[q];
         }
       }
     }
@@ -161,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     eq += (v && key[e] == T) ? 1u : 0u;
   }
   uint32_t total;
-  const uint32_t pre = block_excl_scan((gt << 16) | eq, wsum, &total);
+  const uint32_t pre = block_excl_scan<kThreads>((gt << 16) | eq, wsum, &total);
   if (tid == 0) {
     s_tot[0] = total >> 16;
     s_tot[1] = total & 0xFFFFu;
@@ -188,9 +198,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   cluster.sync();  // peers may still be reading this CTA's shared memory
 }
 
-template <int PER>
+template <int PER, int kThreads>
 dsa_status_t launch_topk(const TopkArgs& a, int C) {
-  auto kern = topk_cluster_kernel<PER>;
+  auto kern = topk_cluster_kernel<PER, kThreads>;
   if (C > 8) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
       return DSA_ERR_UNSUPPORTED;
@@ -222,21 +232,16 @@ dsa_status_t topk_radix(const TopkArgs& a) {
   if (rows == 0) return DSA_OK;
   const int num_sms = std::max(1, device_sm_count(a.device));
   const int64_t n_max = std::max(1, a.s_max);
-  // Keys per thread: 16 when the rows alone fill the GPU, fewer (more CTAs
-  // per row) for a handful of long rows; at most 16 CTAs per row.
-  int per = 16;
-  if (rows * ((n_max + 16 * kThreads - 1) / (16 * kThreads)) < 2 * num_sms) {
-    if ((n_max + 4 * kThreads - 1) / (4 * kThreads) <= 8) per = 4;
-    else if ((n_max + 8 * kThreads - 1) / (8 * kThreads) <= 8) per = 8;
-  }
-  const int64_t C = (n_max + static_cast<int64_t>(per) * kThreads - 1) / (static_cast<int64_t>(per) * kThreads);
+  // 512 threads x 32 keys (16K keys, two CTAs per SM) per cluster rank; when
+  // a handful of long rows would leave SMs idle, 8 keys a thread instead
+  // (more CTAs per row); at most 16 CTAs per row.
+  constexpr int kT = 512;
+  int per = 32;
+  if (rows * ((n_max + 32 * kT - 1) / (32 * kT)) < 2 * num_sms && (n_max + 8 * kT - 1) / (8 * kT) <= 8) per = 8;
+  const int64_t C = (n_max + static_cast<int64_t>(per) * kT - 1) / (static_cast<int64_t>(per) * kT);
   if (C > kMaxCluster) return DSA_ERR_UNSUPPORTED;
   if (rows * C > INT32_MAX) return DSA_ERR_UNSUPPORTED;
-  switch (per) {
-    case 4: return launch_topk<4>(a, static_cast<int>(C));
-    case 8: return launch_topk<8>(a, static_cast<int>(C));
-    default: return launch_topk<16>(a, static_cast<int>(C));
-  }
+  return per == 8 ? launch_topk<8, kT>(a, static_cast<int>(C)) : launch_topk<32, kT>(a, static_cast<int>(C));
 }
 
 }  // namespace dsa
