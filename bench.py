@@ -98,6 +98,23 @@ class ClockSampler:
         return {"sm_mhz": med, "sm_max_mhz": smax, "samples": len(sm), "reasons": sorted(reasons)}
 
 
+def max_over_ranks(value: float, device) -> float:
+    """The largest `value` over all ranks of the default process group (a
+    timing aggregation; every rank calls it at the same point)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _metric_name(wl):
+    if wl.n_q == 1:
+        return "DSA layer queries/s at 128K ctx" if wl.s_max == 131072 else f"DSA layer queries/s ({wl.name})"
+    return f"DSA layer prefill tokens/s ({wl.name})"
+
+
 def _workload_desc(wl):
     return (f"{wl.name}: B={wl.batch}, n_q={wl.n_q}, ctx={wl.s_max}, index_topk={wl.topk}, "
             f"H_I={wl.idx_heads}x{wl.idx_dim} ({'e4m3' if wl.idx_fp8 else wl.dtype}), "
@@ -244,19 +261,13 @@ def run_ours(args, wl):
     rc, word = dsa.get_error(clear=True)
     if rc != 0:
         raise RuntimeError(f"device error word {word:#x} after timing")
-    if ws > 1:
-        tt = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(total_ms, dev)
     ms_per_step = total_ms / args.steps
 
     # end to end through the host-buffer entry point
     e2e = _e2e(args, wl, dsa, dsa.shape_from_workload(wl, q_chunk=chunk if len(rounds) > 1 else 0), t, k_idx,
                k_scale, dev, stream)
-    if ws > 1:
-        tt = torch.tensor([e2e["ms"]], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        e2e["ms"] = float(tt.item())
+    e2e["ms"] = max_over_ranks(e2e["ms"], dev)
 
     res = None
     if rank == 0:
@@ -271,8 +282,7 @@ def run_ours(args, wl):
                     "frac": achieved / hbm, "peak_source": f"{src} hbm_gbs (of {src})",
                     "traffic": _traffic(wl), "algorithmic_bytes": idx_bytes,
                     "tensor_tflops": _indexer_flops(wl) / (idx_ms * 1e-3) / 1e12}
-            metric = ("DSA layer queries/s at 128K ctx" if wl.s_max == 131072
-                      else f"DSA layer queries/s ({wl.name})")
+            metric = _metric_name(wl)
         else:
             flops = _indexer_flops(wl)
             achieved = flops / (idx_ms * 1e-3) / 1e12
@@ -280,7 +290,7 @@ def run_ours(args, wl):
             roof = {"kernel": "indexer", "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "peak_source": f"{src} bf16_tflops_sustained (of {src})",
                     "traffic": _traffic(wl), "algorithmic_flops": flops}
-            metric = f"DSA layer prefill tokens/s ({wl.name})"
+            metric = _metric_name(wl)
         res = {
             "metric": metric,
             "value": q_total / (ms_per_step * 1e-3),
@@ -358,7 +368,7 @@ def _oracle_sample(wl, n_rows, seed=0):
 def cpu_baseline(wl, n_rows=None):
     import oracle
     cores = oracle.num_threads()
-    n_rows = n_rows or max(1, min(wl.batch, cores))
+    n_rows = n_rows or (max(1, min(wl.batch, cores)) if wl.n_q == 1 else cores)
     secs, rows = _oracle_sample(wl, n_rows)
     what = (f"{rows} decode queries of the same workload (full {wl.s_max}-key context each)" if wl.n_q == 1
             else f"{rows} query rows drawn uniformly from the {wl.n_q}-token prefill")
@@ -373,7 +383,7 @@ def run_reference(args, wl):
         return None
     import oracle
     cores = oracle.num_threads()
-    n_rows = max(1, min(wl.batch, cores))
+    n_rows = max(1, min(wl.batch, cores)) if wl.n_q == 1 else cores
     for _ in range(args.warmup and 1):
         _oracle_sample(wl, 1, seed=99)
     secs = 0.0
@@ -383,17 +393,18 @@ def run_reference(args, wl):
         secs += s
         rows += r
     value = rows / secs
+    unit = "queries/s" if wl.n_q == 1 else "tokens/s"
     line = {
         "impl": "reference",
-        "metric": "DSA layer queries/s at 128K ctx" if wl.s_max == 131072 else f"DSA layer queries/s ({wl.name})",
-        "value": value, "unit": "queries/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "metric": _metric_name(wl),
+        "value": value, "unit": unit, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic (seeded gaussian, bf16)",
         "config": {"workload": _workload_desc(wl), "global_batch": n_rows, "seq_len": wl.s_max,
                    "parallelism": "host cores"},
-        "cpu_baseline": {"value": value, "unit": "queries/s", "cores": cores, "kind": "oracle",
-                         "sample": f"each step: {n_rows} decode queries of the workload"},
-        "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+                         "sample": f"each step: {n_rows} query rows of the workload"},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
     return line

@@ -248,6 +248,16 @@ size_t dsa_workspace_bytes(const dsa_shape_t *shape, int32_t which);
  */
 dsa_status_t dsa_get_error(int32_t clear, uint32_t *detail);
 
+/*
+ * Diagnostic with no counterpart on the pages: enqueues a one-thread kernel
+ * whose bounded wait on a barrier is never completed.  After the library's
+ * wait limit (about 2 s) it gives up, records DSA_ERR_TIMEOUT in the device
+ * error word and returns, exactly as a stalled pipeline wait in the other
+ * kernels would; the context stays usable.  Read the result with
+ * dsa_get_error().
+ */
+dsa_status_t dsa_selftest_wait_timeout(void *stream);
+
 /* Static English text for a status code. */
 const char *dsa_status_string(dsa_status_t status);
 

@@ -27,7 +27,7 @@ STATUS = {
 EXPORTS = (
     "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_hadamard_quant_fp8", "dsa_forward",
     "dsa_forward_host", "dsa_workspace_bytes", "dsa_get_error", "dsa_status_string", "dsa_version",
-    "dsa_sparse_mla_attn_static",
+    "dsa_sparse_mla_attn_static", "dsa_selftest_wait_timeout",
 )
 
 
@@ -72,6 +72,7 @@ def lib():
         L.dsa_sparse_mla_attn.argtypes = [S, P, P, P, P, P, P, P, P, sz, P]
         L.dsa_hadamard_quant_fp8.argtypes = [P, i32, i64, i32, P, P, P]
         L.dsa_sparse_mla_attn_static.argtypes = [S, P, P, P, P, P, P, P, P]
+        L.dsa_selftest_wait_timeout.argtypes = [P]
         L.dsa_forward.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
         L.dsa_forward_host.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
         L.dsa_workspace_bytes.argtypes = [S, i32]
@@ -216,6 +217,11 @@ def forward_host(shape, h_q_idx, h_w, h_q, h_ctx_len, h_q_pos0, k_idx, kv, h_out
                                   _p(k_idx), _p(k_scale), _p(kv), _p(v), _p(h_out), _p(h_lse), _p(ws), n,
                                   _stream(stream)), "dsa_forward_host")
     return h_out
+
+
+def selftest_wait_timeout(stream=None):
+    """Enqueue the bounded-wait diagnostic (see dsa_selftest_wait_timeout)."""
+    _check(lib().dsa_selftest_wait_timeout(_stream(stream)), "dsa_selftest_wait_timeout")
 
 
 def get_error(clear=True):

@@ -518,6 +518,11 @@ const char* dsa_status_string(dsa_status_t status) {
 
 int32_t dsa_version(void) { return 100; }
 
+dsa_status_t dsa_selftest_wait_timeout(void* stream) {
+  DSA_SETUP(dev);
+  return selftest_wait_timeout(g_err_ptr[dev], static_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"
 
 // ------------------------------------------------ allocation-free attention --

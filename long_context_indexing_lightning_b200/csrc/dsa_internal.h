@@ -86,6 +86,8 @@ dsa_status_t attn_simt(const AttnArgs& a);  // F32 (and BF16 shapes the tensor p
 bool attn_tc_supported(int H, int d_qk, int d_v, int KVH);
 size_t attn_scratch_bytes(int B, int n_q, int k, int num_sms);
 
+dsa_status_t selftest_wait_timeout(uint32_t* err, cudaStream_t stream);
+
 dsa_status_t hadamard_quant(const void* x, int x_dtype, int64_t rows, int dim, uint8_t* x8, float* scale,
                             cudaStream_t stream);
 

@@ -422,3 +422,26 @@ def test_forward_fp8_matches_oracle_fp8_path():
     o_rec = [rec(o8_idx, o_idx, r) for r in range(wl.batch)]
     assert abs(np.mean(g_rec) - np.mean(o_rec)) <= 0.01, (g_rec, o_rec)
     assert torch.isfinite(out.float()).all()
+
+
+@pytest.mark.slow
+def test_forward_decode128k_full_size_sampled_sequences():
+    """The benchmark's configuration (32 queries at 131072 keys, k = 2048, same
+    split plan): the step runs on all 32 sequences; the oracle checks three."""
+    wl = workloads.get("decode128k")
+    t = workloads.make_inputs(wl, DEV, seed=0)
+    shape = dsa.shape_from_workload(wl)
+    idx_out = torch.empty(wl.batch, 1, wl.topk, dtype=torch.int32, device=DEV)
+    out = dsa.forward(shape, t["q_idx"], t["k_idx"], t["w"], t["q"], t["kv"], t["ctx_len"], t["q_pos0"],
+                      idx_out=idx_out)
+    torch.cuda.synchronize()
+    picked = [0, 13, 31]
+    sub = {k: t[k][picked].contiguous() for k in ("q_idx", "k_idx", "w", "q", "kv", "ctx_len", "q_pos0")}
+    rows = [(i, 0) for i in range(len(picked))]
+    o_idx, o_sc = _oracle_idx_for(sub, wl, rows)
+    g_idx = idx_out.reshape(wl.batch, wl.topk)[picked].cpu().numpy()
+    check_idx_valid(g_idx, _pos(H(sub["q_pos0"]), rows), wl.topk)
+    check_topk_near_ties(g_idx, o_idx, o_sc, wl.topk)
+    o = _attn_oracle(sub, o_idx, wl, rows)
+    got = out[picked].float().cpu().numpy().reshape(len(picked), wl.heads, wl.d_v).astype(np.float64)
+    assert np.abs(got - o).max() <= ATTN_ATOL_BF16
