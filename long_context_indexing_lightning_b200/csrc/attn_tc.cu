@@ -9,25 +9,36 @@
 //
 // One thread-block cluster of two CTAs per (query row, split of its selected
 // list).  The 576 latent columns are cut at 256: CTA 0 owns columns [0, 256),
-// CTA 1 owns [256, 576).  Each CTA
+// CTA 1 owns [256, 576); CTA c also owns the softmax of heads [64c, 64c + 64).
+// Per 64-row tile, each CTA
 //   * gathers only its own columns of the selected rows (cp.async, 16 bytes a
-//     thread, into a 3-stage ring of 64-row tiles in the 128-byte-swizzled
-//     K-major layout the MMA reads; padding and out-of-range rows are zero
-//     filled),
-//   * keeps its columns of Q in tensor memory (A operand of the logits MMA),
-//   * computes its partial logits S_c = Q_c K_c^T (M = 128 heads, N = 64 rows),
-//   * swaps partials with the other CTA (a bulk copy of 32 KB into the other
-//     CTA's shared memory, completing on its barrier), so
-//     both hold the same S = S_0 + S_1 (fp32 addition is commutative, so the
-//     two sums are bit-identical) and run the same online softmax,
+//     thread, into a 3-stage ring in the 128-byte-swizzled K-major layout the
+//     MMA reads; padding and out-of-range rows are zero filled),
+//   * computes its partial logits S_c = Q_c K_c^T for all 128 heads (M = 128,
+//     N = 64, Q_c held in tensor memory),
+//   * reduce-scatter: ships the partial logits of the other CTA's 64 heads
+//     (16 KB, one bulk copy into the other CTA's shared memory) and adds the
+//     partial it receives for its own 64 heads, so each CTA holds the full
+//     S = S_0 + S_1 for the heads whose softmax it runs,
+//   * runs the online softmax of its 64 heads (base 2; the running max only
+//     moves, and O is rescaled in TMEM, when a tile max exceeds it by more
+//     than 8) and writes their P rows in bf16,
+//   * all-gather: ships those P rows (8 KB) and the heads' running max and
+//     partial sums to the other CTA, which rescales its O rows of those heads
+//     when the max moved,
 //   * accumulates its 256-column half of the output, O_c += P V_c, in TMEM
 //     (V_0 = latent columns [0, 256), V_1 = [256, 512): each CTA's value half
 //     lies inside the columns it already gathered).
-// Warps: 0-3 gather, 4 issues tcgen05.mma, 5-8 (thread = head = TMEM lane)
-// load Q into TMEM and run the softmax in base 2 with a running max that only
-// moves (and O is rescaled in TMEM) when a tile max exceeds it by more than 8.
-// Long selections are split across clusters and merged by a small combine
-// kernel (log-sum-exp weights).  Every wait is bounded.
+// Exchange buffers, P and the row statistics are double buffered so that
+// tile j's exchange overlaps tile j-1's softmax, and the softmax warps read
+// tile j+1's logits before they wait for tile j's partial.
+// Warps: 0-3 gather, 4 issues tcgen05.mma, 5-12 (two per TMEM lane quarter,
+// thread = head = TMEM lane): in the quarters of this CTA's own heads both
+// warps run the softmax, 32 of the tile's 64 columns each; in the other
+// quarters one warp ships the partial logits and one applies the other CTA's
+// P statistics to this CTA's O rows.  Long selections are split across
+// clusters and merged by a small combine kernel (log-sum-exp weights).  Every
+// wait is bounded.
 #include "dsa_common.cuh"
 #include "dsa_internal.h"
 
@@ -35,6 +46,7 @@ namespace dsa {
 namespace {
 
 constexpr int kH = 128;                  // heads == MMA M
+constexpr int kHHalf = 64;               // heads whose softmax one CTA runs
 constexpr int kDqk = 576;                // latent 512 + rope 64
 constexpr int kDv = 512;
 constexpr int kDvHalf = 256;
@@ -46,27 +58,34 @@ constexpr int kStageBytes = kAtomsMax * kAtomBytes;  // 40 KB
 constexpr int kStages = 3;
 constexpr int kGatherWarps = 4;
 constexpr int kMmaWarp = 4;
-constexpr int kSoftThreads = 128;
-constexpr int kThreads = 32 * kGatherWarps + 32 + kSoftThreads;  // 288
+constexpr int kSoftWarps = 8;
+constexpr int kThreads = 32 * (kGatherWarps + 1 + kSoftWarps);  // 416
 // tensor memory: O half [0, 256), Q columns [256, 256 + 160), S [416, 480)
 constexpr int kTmemCols = 512;
 constexpr int kQCol = 256;
 constexpr int kSCol = 416;
 
-// shared memory map (from a 1024-aligned base)
+// shared memory map (from a 1024-aligned base); [2] = double buffered by tile parity
+constexpr int kPBytes = kH * kRows * 2;      // P: 128 heads x 64 rows bf16, SW128 K-major
+constexpr int kPHalfBytes = kPBytes / 2;     // the 64 rows of one CTA's heads (contiguous)
+constexpr int kXBytes = kHHalf * kRows * 4;  // partial logits of 64 heads: [16 x 4 rows][64 heads] fp32
+constexpr int kStatBytes = 3 * kHHalf * 4;   // per head: running max, partial sum of each softmax warp
 constexpr int kOffKV = 0;
-constexpr int kOffP = kOffKV + kStages * kStageBytes;  // P: 128 heads x 64 rows bf16, SW128 K-major
-// partial logits, chunk-major [16 x 4 rows][128 heads] fp32: the other CTA's
-// (received by bulk copy) and this CTA's (sent from here)
-constexpr int kXBytes = kH * kRows * 4;
-constexpr int kOffXin = kOffP + kH * kRows * 2;
-constexpr int kOffXout = kOffXin + kXBytes;
-constexpr int kOffBar = kOffXout + kXBytes;
-// barriers: kv_full[3], kv_empty[3], s_full, s_empty, p_full, p_empty, o_done,
-//           q_ready, x_full, x_empty, mma_done, xout_free, xout_written, xin_read
-constexpr int kNumBars = 2 * kStages + 12;
+constexpr int kOffP = kOffKV + kStages * kStageBytes;
+constexpr int kOffXin = kOffP + 2 * kPBytes;      // partial logits received for this CTA's heads
+constexpr int kOffXout = kOffXin + 2 * kXBytes;   // partial logits of the other CTA's heads, to ship
+constexpr int kOffStOut = kOffXout + 2 * kXBytes; // statistics of this CTA's heads, to ship
+constexpr int kOffStIn = kOffStOut + 2 * kStatBytes;
+constexpr int kOffRed = kOffStIn + 2 * kStatBytes;  // tile max of each softmax warp: [2][2 warps][64]
+// barriers: kv_full[3], kv_empty[3], q_ready, s_full, s_empty, mma_done, fin,
+// pside_done, then 11 double-buffered ones (see the enum in the kernel)
+constexpr int kNumDBars = 11;
+constexpr int kNumBars = 2 * kStages + 6 + 2 * kNumDBars;
+constexpr int kOffBar = kOffRed + 2 * 2 * kHHalf * 4;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory");
+static_assert(kOffP % 1024 == 0 && kPBytes % 1024 == 0, "P tiles must stay 1024-aligned");
 
 struct AttnParams {
   const uint16_t* q;        // [R][128][576] bf16
@@ -76,7 +95,7 @@ struct AttnParams {
   __nv_bfloat16* out;       // [R][128][512]
   float* lse;               // [R][128] or null
   float* part_o;            // [R][S][2][128][256] (splits > 1)
-  float* part_ml;           // [R][S][2][2][128]: m then l (splits > 1)
+  float* part_ml;           // [R][S][2][128]: m then l (splits > 1)
   int n_q, s_max, k, splits, rows_per_split;
   float scale_log2;         // sm_scale * log2(e)
   uint32_t* err;
@@ -123,10 +142,6 @@ __device__ __forceinline__ uint32_t map_peer(uint32_t saddr, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
-}
-__device__ __forceinline__ void st_cluster_v4f(uint32_t raddr, float a, float b, float c, float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(raddr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
 }
 // Arrive on an mbarrier of another CTA of the cluster, ordering this
 // thread's earlier shared-memory accesses before the arrival.
@@ -218,6 +233,55 @@ __device__ __forceinline__ void gather_tile(uint32_t dst0, const char* kv_b, int
   }
 }
 
+// Single-thread bounded wait on a barrier that the other CTA arrives on.
+__device__ __forceinline__ bool mbar_wait_cluster1(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                                   uint32_t* err) {
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 0; i < kWaitLimitPolls; ++i) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((i & 63u) == 63u) {
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) break;
+    }
+  }
+  *abort_flag = 1;
+  raise_error(err, kErrTimeout);
+  return false;
+}
+// Bulk copy of `bytes` from this CTA's shared memory into the other CTA's,
+// completing on the other CTA's barrier (addresses already mapped).
+__device__ __forceinline__ void bulk_to_peer(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "r"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's bulk groups still read their source.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+__device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+// Scale 32-column chunks [c0, c1) of this thread's O row in TMEM by f.
+__device__ __forceinline__ void rescale_o_cols(uint32_t tl, int c0, int c1, float f) {
+#pragma unroll 1
+  for (int c = c0; c < c1; c += 32) {
+    float o[32];
+    tmem_ld32(tl + c, o);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) o[i] *= f;
+    tmem_st32f(tl + c, o);
+  }
+  tmem_st_wait();
+}
+
 __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -225,24 +289,33 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
   const uint32_t bar0 = sbase + kOffBar;
   auto kv_full = [&](int i) { return bar0 + 8u * i; };
   auto kv_empty = [&](int i) { return bar0 + 8u * (kStages + i); };
-  const uint32_t s_full = bar0 + 8u * (2 * kStages + 0);
-  const uint32_t s_empty = bar0 + 8u * (2 * kStages + 1);
-  const uint32_t p_full = bar0 + 8u * (2 * kStages + 2);
-  const uint32_t p_empty = bar0 + 8u * (2 * kStages + 3);
-  const uint32_t o_done = bar0 + 8u * (2 * kStages + 4);
-  const uint32_t q_ready = bar0 + 8u * (2 * kStages + 5);
-  const uint32_t x_full = bar0 + 8u * (2 * kStages + 6);
-  const uint32_t x_empty = bar0 + 8u * (2 * kStages + 7);
-  const uint32_t mma_done = bar0 + 8u * (2 * kStages + 8);
-  const uint32_t xout_free = bar0 + 8u * (2 * kStages + 9);
-  const uint32_t xout_written = bar0 + 8u * (2 * kStages + 10);
-  const uint32_t xin_read = bar0 + 8u * (2 * kStages + 11);
+  const uint32_t q_ready = bar0 + 8u * (2 * kStages + 0);
+  const uint32_t s_full = bar0 + 8u * (2 * kStages + 1);
+  const uint32_t s_empty = bar0 + 8u * (2 * kStages + 2);
+  const uint32_t mma_done = bar0 + 8u * (2 * kStages + 3);
+  const uint32_t fin = bar0 + 8u * (2 * kStages + 4);
+  const uint32_t pside_done = bar0 + 8u * (2 * kStages + 5);  // P-side warps saw the last tile's statistics
+  // double-buffered barriers, index [tile parity]
+  enum {
+    X_FULL,         // received partial logits landed (armed here, bulk copy from the other CTA)
+    X_EMPTY,        // the other CTA has added our shipped partial (remote arrive)
+    XOUT_WRITTEN,   // ship warps staged the outgoing partial
+    XOUT_FREE,      // the outgoing bulk copy has read the staging buffer
+    XIN_READ,       // softmax warps have added the received partial
+    P_OWN_WRITTEN,  // softmax warps wrote their heads' P rows and statistics
+    PEER_P_FREE,    // the other CTA's P buffer is free (its PV two tiles back is done; remote arrive)
+    P_REMOTE_FULL,  // the other CTA's P rows and statistics landed (armed here, bulk copy)
+    PV_READY,       // all P rows present and every O row rescaled: PV may run
+    PV_DONE,        // PV of this buffer's last tile is done (tcgen05.commit)
+    RED_FULL        // both softmax warps of each head published their tile max
+  };
+  auto dbar = [&](int which, int b) { return bar0 + 8u * (2 * kStages + 6 + 2 * which + b); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = lane_id();
-  const uint32_t crank = cluster_rank();  // 0: latent columns [0, 256); 1: [256, 576)
+  const uint32_t crank = cluster_rank();  // 0: latent columns [0, 256), heads [0, 64); 1: [256, 576), [64, 128)
   const uint32_t peer = crank ^ 1u;
   const int a0 = crank == 0 ? 0 : kSplitCol / 64;  // first 64-column atom of this CTA
   const int natoms = crank == 0 ? kSplitCol / 64 : (kDqk - kSplitCol) / 64;
@@ -262,19 +335,29 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
       mbar_init(kv_full(i), 32 * kGatherWarps);
       mbar_init(kv_empty(i), 1);
     }
+    mbar_init(q_ready, 32 * kSoftWarps);
     mbar_init(s_full, 1);
-    mbar_init(s_empty, kSoftThreads);
-    mbar_init(p_full, kSoftThreads);
-    mbar_init(p_empty, 1);
-    mbar_init(o_done, 1);
-    mbar_init(q_ready, kSoftThreads);
-    mbar_init(x_full, 1);   // own arm (expect_tx) + the other CTA's bulk copy
-    mbar_init(x_empty, 1);  // arrived by the other CTA once it has read our partial
+    mbar_init(s_empty, 192);  // 128 softmax threads + 64 ship threads read S
     mbar_init(mma_done, 1);
-    mbar_init(xout_free, 1);
-    mbar_init(xout_written, kSoftThreads);
-    mbar_init(xin_read, kSoftThreads);
-    if (T > 0) mbar_arrive_expect_tx(x_full, kXBytes);  // armed for tile 0
+    mbar_init(fin, 128);
+    mbar_init(pside_done, 64);
+    for (int bb = 0; bb < 2; ++bb) {
+      mbar_init(dbar(X_FULL, bb), 1);
+      mbar_init(dbar(X_EMPTY, bb), 1);
+      mbar_init(dbar(XOUT_WRITTEN, bb), 64);
+      mbar_init(dbar(XOUT_FREE, bb), 1);
+      mbar_init(dbar(XIN_READ, bb), 128);
+      mbar_init(dbar(P_OWN_WRITTEN, bb), 128);
+      mbar_init(dbar(PEER_P_FREE, bb), 1);
+      mbar_init(dbar(P_REMOTE_FULL, bb), 1);
+      mbar_init(dbar(PV_READY, bb), 192);  // 128 softmax threads + 64 P-side threads
+      mbar_init(dbar(PV_DONE, bb), 1);
+      mbar_init(dbar(RED_FULL, bb), 128);
+      if (bb < T) {  // armed for tiles 0 and 1; later tiles re-arm one round ahead
+        mbar_arrive_expect_tx(dbar(X_FULL, bb), kXBytes);
+        mbar_arrive_expect_tx(dbar(P_REMOTE_FULL, bb), kPHalfBytes + kStatBytes);
+      }
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -285,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
-  cluster_sync_all();  // both CTAs' barriers exist before any remote arrival
+  cluster_sync_all();  // both CTAs' barriers exist (and are armed) before any remote arrival
   const uint32_t tmem = *tmem_slot;
 
   if (warp < kGatherWarps) {
@@ -325,17 +408,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
       uint64_t t0 = 0;
       uint32_t spins = 0;
       while (ok && np < T) {
-        // O += P(np) V(np) as soon as P is written (frees the tile's stage)
-        if (np < nq && mbar_test_wait(p_full, np & 1)) {
+        // O += P(np) V(np) once every P row is in place and O rows are rescaled
+        if (np < nq && mbar_test_wait(dbar(PV_READY, np & 1), (np >> 1) & 1)) {
           tc_fence_after_sync();
           const uint64_t st_off = static_cast<uint64_t>(((np % kStages) * kStageBytes) >> 4);
+          const uint64_t p_off = static_cast<uint64_t>(((np & 1) * kPBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < kRows / 16; ++kk)
-            tc_mma_f16(tmem, p_desc0 + ((kk * 32) >> 4), v_desc0 + st_off + ((kk * 16 * 128) >> 4), idesc_o,
+            tc_mma_f16(tmem, p_desc0 + p_off + ((kk * 32) >> 4), v_desc0 + st_off + ((kk * 16 * 128) >> 4), idesc_o,
                        (np > 0 || kk > 0) ? 1u : 0u);
           tc_commit(kv_empty(np % kStages));
-          tc_commit(p_empty);
-          tc_commit(o_done);
+          tc_commit(dbar(PV_DONE, np & 1));
           ++np;
           spins = 0;
           continue;
@@ -371,16 +454,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
       volatile int never = 0;
       mbar_wait(mma_done, 0, &never, P.err);
     }
+    __syncwarp();
   } else {
-    // ------------------------------------- Q to TMEM, softmax, output --
+    // ------------------------------------- Q to TMEM, then three roles --
     const int quarter = warp & 3;
-    const int h = quarter * 32 + lane;  // head == TMEM lane
+    const int sub = (warp - (kGatherWarps + 1)) >> 2;  // which of the quarter's two warps
+    const int h = quarter * 32 + lane;                 // head == TMEM lane
+    const int hl = h & (kHHalf - 1);                   // index among its CTA's 64 heads
+    const bool own = static_cast<uint32_t>(quarter >> 1) == crank;
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     {
       // this CTA's columns of q[r, h, :] as packed bf16 pairs (element 2i in
-      // the low half of column i)
+      // the low half of column i); the quarter's two warps take half each
       const uint4* qs = reinterpret_cast<const uint4*>(P.q + (static_cast<int64_t>(r) * kH + h) * kDqk + a0 * 64);
-      for (int c = 0; c < natoms * 64 / 32; ++c) {
+      for (int c = sub * natoms; c < (sub + 1) * natoms; ++c) {
         uint32_t u[16];
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
@@ -396,140 +483,246 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
       tc_fence_before_sync();
       mbar_arrive(q_ready);
     }
-    const uint32_t xin = sbase + kOffXin, xout = sbase + kOffXout;
-    const uint32_t xin_peer = map_peer(xin, peer);
-    const uint32_t x_full_peer = map_peer(x_full, peer);
-    const uint32_t x_empty_peer = map_peer(x_empty, peer);
-    const bool leader = (h == 0);  // issues the bulk copy and the cross-CTA signals
-    float m_run = -INFINITY, l_run = 0.f;
+    const uint32_t p0 = sbase + kOffP;
+    const uint32_t xin0 = sbase + kOffXin, xout0 = sbase + kOffXout;
+    const uint32_t sto0 = sbase + kOffStOut, sti0 = sbase + kOffStIn;
     bool ok = true;
-    int nx0 = (lane < nrows) ? __ldg(sel + lane) : -1;
-    int nx1 = (lane + 32 < nrows) ? __ldg(sel + lane + 32) : -1;
-    for (int j = 0; j < T; ++j) {
-      // which rows of this tile are real (indices fetched one tile ahead)
-      const uint32_t valid0 = __ballot_sync(0xffffffffu, nx0 >= 0 && nx0 < L);
-      const uint32_t valid1 = __ballot_sync(0xffffffffu, nx1 >= 0 && nx1 < L);
-      const int jn = (j + 1) * kRows + lane;
-      nx0 = (j + 1 < T && jn < nrows) ? __ldg(sel + jn) : -1;
-      nx1 = (j + 1 < T && jn + 32 < nrows) ? __ldg(sel + jn + 32) : -1;
-      if (!mbar_wait_warp(s_full, j & 1, abort_flag, P.err)) { ok = false; break; }
-      tc_fence_after_sync();
-      float s[kRows];
-      tmem_ld32(tl + kSCol, s);
-      tmem_ld32(tl + kSCol + 32, s + 32);
-      tc_fence_before_sync();
-      mbar_arrive(s_empty);
-      // swap partial logits with the other CTA: stage mine locally, one
-      // thread copies the 32 KB into the other CTA's receive buffer ...
-      if (leader && j >= 1) {
-        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // previous copy has read xout
-        mbar_arrive(xout_free);
+    float m_fin = -INFINITY, l_fin = 0.f;  // head h's final running max and sum
+    int c_lo = 0, c_hi = 0;                // this thread's O columns in the epilogue
+
+    if (own) {
+      // ---------------------- softmax of this CTA's heads, 32 columns a warp --
+      const int kh = sub;
+      const bool leader = (hl == 0 && kh == 0);  // ships P rows; re-arms and releases the receive buffer
+      float sreg[32], snext[32];
+      float m_run = -INFINITY, l_half = 0.f;
+      int ix = (kh * 32 + lane < nrows) ? __ldg(sel + kh * 32 + lane) : -1;
+      if (T > 0) {
+        if (!mbar_wait_warp(s_full, 0, abort_flag, P.err)) {
+          ok = false;
+        } else {
+          tc_fence_after_sync();
+          tmem_ld32(tl + kSCol + 32 * kh, sreg);
+          tc_fence_before_sync();
+          mbar_arrive(s_empty);
+        }
       }
-      if (!mbar_wait_warp(xout_free, (j & 1) ^ 1, abort_flag, P.err)) { ok = false; break; }
+      for (int j = 0; ok && j < T; ++j) {
+        const int bb = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        const uint32_t valid = __ballot_sync(0xffffffffu, ix >= 0 && ix < L);
+        const int jn = (j + 1) * kRows + kh * 32 + lane;
+        ix = (j + 1 < T && jn < nrows) ? __ldg(sel + jn) : -1;
+        // the next tile's logits first, so that its MMA runs under this softmax
+        if (j + 1 < T) {
+          if (!mbar_wait_warp(s_full, (j + 1) & 1, abort_flag, P.err)) { ok = false; break; }
+          tc_fence_after_sync();
+          tmem_ld32(tl + kSCol + 32 * kh, snext);
+          tc_fence_before_sync();
+          mbar_arrive(s_empty);
+        }
+        // S = S_0 + S_1: add the other CTA's partial for these heads
+        if (!mbar_wait_warp_cluster(dbar(X_FULL, bb), ph, abort_flag, P.err)) { ok = false; break; }
+        const uint32_t xb = xin0 + bb * kXBytes;
 #pragma unroll
-      for (int c = 0; c < kRows / 4; ++c)
-        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(xout + (c * kH + h) * 16), "f"(s[4 * c]),
-                     "f"(s[4 * c + 1]), "f"(s[4 * c + 2]), "f"(s[4 * c + 3])
-                     : "memory");
-      fence_proxy_async_smem();
-      mbar_arrive(xout_written);
-      if (leader) {
-        bool go = mbar_wait(xout_written, j & 1, abort_flag, P.err);
-        if (go && j >= 1) {
-          // the other CTA has read our previous partial
-          go = false;
-          const uint64_t t0 = global_timer_ns();
-          for (uint32_t it = 0; it < kWaitLimitPolls; ++it) {
-            if (mbar_try_wait_cluster(x_empty, (j - 1) & 1)) { go = true; break; }
-            if ((it & 63u) == 63u && (*abort_flag || global_timer_ns() - t0 > kWaitLimitNs)) break;
+        for (int c = 0; c < 8; ++c) {
+          const float4 v = ld_shared_v4f(xb + ((kh * 8 + c) * kHHalf + hl) * 16);
+          sreg[4 * c] += v.x;
+          sreg[4 * c + 1] += v.y;
+          sreg[4 * c + 2] += v.z;
+          sreg[4 * c + 3] += v.w;
+        }
+        mbar_arrive(dbar(XIN_READ, bb));
+        if (leader && mbar_wait(dbar(XIN_READ, bb), ph, abort_flag, P.err) && j + 2 < T) {
+          mbar_arrive_expect_tx(dbar(X_FULL, bb), kXBytes);  // armed for tile j + 2 ...
+          mbar_arrive_remote(map_peer(dbar(X_EMPTY, bb), peer));  // ... before the other CTA may send it
+        }
+        float mt = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const bool v = ((valid >> i) & 1u) != 0;
+          sreg[i] = v ? sreg[i] * P.scale_log2 : -INFINITY;
+          mt = fmaxf(mt, sreg[i]);
+        }
+        // tile max over all 64 columns: swap with the head's other warp
+        const uint32_t red = sbase + kOffRed + bb * (2 * kHHalf * 4);
+        st_shared_f32(red + (kh * kHHalf + hl) * 4, mt);
+        mbar_arrive(dbar(RED_FULL, bb));
+        if (!mbar_wait_warp(dbar(RED_FULL, bb), ph, abort_flag, P.err)) { ok = false; break; }
+        mt = fmaxf(mt, ld_shared_f32(red + ((kh ^ 1) * kHHalf + hl) * 4));
+        // move the running max only when the tile max exceeds it by > 8 (base 2)
+        const bool move = mt > m_run + 8.f;
+        const bool rescale_o = move && m_run != -INFINITY;
+        if (__any_sync(0xffffffffu, rescale_o)) {
+          // O must hold every previous tile before it is rescaled (PV of
+          // tile j - 3 was awaited one tile ago, so this parity is unambiguous)
+          if (j >= 1 && !mbar_wait_warp(dbar(PV_DONE, bb ^ 1), ((j - 1) >> 1) & 1, abort_flag, P.err)) {
+            ok = false;
+            break;
           }
-          if (!go && !*abort_flag) { *abort_flag = 1; raise_error(P.err, kErrTimeout); }
+          tc_fence_after_sync();
+          rescale_o_cols(tl, kh * 128, kh * 128 + 128, rescale_o ? exp2f(m_run - mt) : 1.f);
         }
-        if (go) {
-          asm volatile(
-              "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n\t"
-              "cp.async.bulk.commit_group;" ::"r"(xin_peer),
-              "r"(xout), "r"(kXBytes), "r"(x_full_peer)
-              : "memory");
+        if (move) {
+          if (m_run != -INFINITY) l_half *= exp2f(m_run - mt);
+          m_run = mt;
         }
-      }
-      // ... and the other CTA's partial arrives in ours: S = S_0 + S_1 on both sides
-      if (!mbar_wait_warp_cluster(x_full, j & 1, abort_flag, P.err)) { ok = false; break; }
+        // P = 2^(s - m) in bf16, 128-byte-swizzled K-major; the buffer is free
+        // once the PV two tiles back is done
+        if (j >= 2 && !mbar_wait_warp(dbar(PV_DONE, bb), ((j - 2) >> 1) & 1, abort_flag, P.err)) {
+          ok = false;
+          break;
+        }
+        const uint32_t pb = p0 + bb * kPBytes;
+        const uint32_t prow = pb + (h >> 3) * 1024 + (h & 7) * 128;
+        float psum = 0.f;
 #pragma unroll
-      for (int c = 0; c < kRows / 4; ++c) {
-        const float4 v = ld_shared_v4f(xin + (c * kH + h) * 16);
-        s[4 * c] += v.x;
-        s[4 * c + 1] += v.y;
-        s[4 * c + 2] += v.z;
-        s[4 * c + 3] += v.w;
-      }
-      mbar_arrive(xin_read);
-      if (leader) {
-        if (mbar_wait(xin_read, j & 1, abort_flag, P.err)) {
-          if (j + 1 < T) mbar_arrive_expect_tx(x_full, kXBytes);  // arm for the next tile
-          mbar_arrive_remote(x_empty_peer);
-        }
-      }
-      float mt = -INFINITY;
+        for (int c = 0; c < 4; ++c) {
+          float p[8];
 #pragma unroll
-      for (int i = 0; i < kRows; ++i) {
-        const bool v = ((i < 32 ? (valid0 >> i) : (valid1 >> (i - 32))) & 1u) != 0;
-        s[i] = v ? s[i] * P.scale_log2 : -INFINITY;
-        mt = fmaxf(mt, s[i]);
+          for (int e = 0; e < 8; ++e) {
+            p[e] = (m_run == -INFINITY) ? 0.f : fast_exp2(sreg[c * 8 + e] - m_run);
+            psum += p[e];
+          }
+          st_shared_v4(prow + (((kh * 4 + c) ^ (h & 7)) << 4), pack_bf16(p[0], p[1]), pack_bf16(p[2], p[3]),
+                       pack_bf16(p[4], p[5]), pack_bf16(p[6], p[7]));
+        }
+        l_half += psum;
+        // statistics for the other CTA: running max, and each warp's partial sum
+        const uint32_t so = sto0 + bb * kStatBytes;
+        if (kh == 0) st_shared_f32(so + hl * 4, m_run);
+        st_shared_f32(so + ((1 + kh) * kHHalf + hl) * 4, l_half);
+        fence_proxy_async_smem();
+        tc_fence_before_sync();
+        mbar_arrive(dbar(P_OWN_WRITTEN, bb));
+        mbar_arrive(dbar(PV_READY, bb));
+        if (leader) {
+          bool go = mbar_wait(dbar(P_OWN_WRITTEN, bb), ph, abort_flag, P.err);
+          if (go && j >= 2) go = mbar_wait_cluster1(dbar(PEER_P_FREE, bb), ((j - 2) >> 1) & 1, abort_flag, P.err);
+          if (go) {
+            bulk_wait_read<0>();  // earlier copies have read P and the statistics
+            const uint32_t pbar = map_peer(dbar(P_REMOTE_FULL, bb), peer);
+            const uint32_t mine = pb + crank * kPHalfBytes;
+            bulk_to_peer(map_peer(mine, peer), mine, kPHalfBytes, pbar);
+            bulk_to_peer(map_peer(sti0 + bb * kStatBytes, peer), so, kStatBytes, pbar);
+            bulk_commit();
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sreg[i] = snext[i];
       }
-      // move the running max only when the tile max exceeds it by > 8 (base 2)
-      const bool move = mt > m_run + 8.f;
-      const bool rescale_o = move && m_run != -INFINITY;
-      if (__any_sync(0xffffffffu, rescale_o)) {
-        // O must hold every previous tile before it is rescaled
-        if (j >= 1 && !mbar_wait_warp(o_done, (j - 1) & 1, abort_flag, P.err)) { ok = false; break; }
+      if (leader) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+      // both warps' partial sums of the last tile
+      if (ok && T > 0) {
+        mbar_arrive(fin);
+        ok = mbar_wait_warp(fin, 0, abort_flag, P.err);
+      }
+      if (ok && T > 0) {
+        const uint32_t so = sto0 + ((T - 1) & 1) * kStatBytes;
+        m_fin = m_run;
+        l_fin = ld_shared_f32(so + (kHHalf + hl) * 4) + ld_shared_f32(so + (2 * kHHalf + hl) * 4);
+      }
+      c_lo = kh * 128;
+      c_hi = c_lo + 128;
+    } else if (sub == 0) {
+      // ------------ ship: partial logits of the other CTA's heads, per tile --
+      const bool leader = (hl == 0);
+      for (int j = 0; ok && j < T; ++j) {
+        const int bb = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (!mbar_wait_warp(s_full, j & 1, abort_flag, P.err)) { ok = false; break; }
         tc_fence_after_sync();
-        const float f = rescale_o ? exp2f(m_run - mt) : 1.f;
-#pragma unroll 1
-        for (int c = 0; c < kDvHalf; c += 32) {
-          float o[32];
-          tmem_ld32(tl + c, o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= f;
-          tmem_st32f(tl + c, o);
+        float s[kRows];
+        tmem_ld32(tl + kSCol, s);
+        tmem_ld32(tl + kSCol + 32, s + 32);
+        tc_fence_before_sync();
+        mbar_arrive(s_empty);
+        if (j >= 2 && !mbar_wait_warp(dbar(XOUT_FREE, bb), ((j - 2) >> 1) & 1, abort_flag, P.err)) {
+          ok = false;
+          break;
         }
-        tmem_st_wait();
-      }
-      if (move) {
-        if (m_run != -INFINITY) l_run *= exp2f(m_run - mt);
-        m_run = mt;
-      }
-      // P = 2^(s - m) in bf16: one 128-byte row per head, 128-byte-swizzled K-major
-      if (j >= 1 && !mbar_wait_warp(p_empty, (j - 1) & 1, abort_flag, P.err)) { ok = false; break; }
-      const uint32_t prow = sbase + kOffP + (h >> 3) * 1024 + (h & 7) * 128;
-      float psum = 0.f;
+        const uint32_t xo = xout0 + bb * kXBytes;
 #pragma unroll
-      for (int c = 0; c < kRows / 8; ++c) {
-        float p[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          p[e] = (m_run == -INFINITY) ? 0.f : fast_exp2(s[c * 8 + e] - m_run);
-          psum += p[e];
+        for (int c = 0; c < kRows / 4; ++c)
+          asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(xo + (c * kHHalf + hl) * 16), "f"(s[4 * c]),
+                       "f"(s[4 * c + 1]), "f"(s[4 * c + 2]), "f"(s[4 * c + 3])
+                       : "memory");
+        fence_proxy_async_smem();
+        mbar_arrive(dbar(XOUT_WRITTEN, bb));
+        if (leader) {
+          bool go = mbar_wait(dbar(XOUT_WRITTEN, bb), ph, abort_flag, P.err);
+          if (go && j >= 2) go = mbar_wait_cluster1(dbar(X_EMPTY, bb), ((j - 2) >> 1) & 1, abort_flag, P.err);
+          if (go) {
+            bulk_to_peer(map_peer(xin0 + bb * kXBytes, peer), xo, kXBytes, map_peer(dbar(X_FULL, bb), peer));
+            bulk_commit();
+            if (j >= 1) {
+              bulk_wait_read<1>();  // the copy of tile j - 1 has read its staging buffer
+              mbar_arrive(dbar(XOUT_FREE, bb ^ 1));
+            }
+          }
         }
-        st_shared_v4(prow + ((c ^ (h & 7)) << 4), pack_bf16(p[0], p[1]), pack_bf16(p[2], p[3]),
-                     pack_bf16(p[4], p[5]), pack_bf16(p[6], p[7]));
       }
-      l_run += psum;
-      fence_proxy_async_smem();
-      tc_fence_before_sync();
-      mbar_arrive(p_full);
+      if (leader) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+      // the other CTA's statistics of these heads after the last tile, once
+      // the P-side warps (which waited on every tile's copy) have seen them
+      if (ok && T > 0) ok = mbar_wait_warp(pside_done, 0, abort_flag, P.err);
+      if (ok && T > 0) {
+        const uint32_t si = sti0 + ((T - 1) & 1) * kStatBytes;
+        m_fin = ld_shared_f32(si + hl * 4);
+        l_fin = ld_shared_f32(si + (kHHalf + hl) * 4) + ld_shared_f32(si + (2 * kHHalf + hl) * 4);
+      }
+      c_lo = 128;
+      c_hi = 256;
+    } else {
+      // -------- P side: the other CTA's P rows and statistics, O rescaling --
+      const bool leader = (hl == 0);
+      float m_prev = -INFINITY;
+      for (int j = 0; ok && j < T; ++j) {
+        const int bb = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (leader && j >= 2 && mbar_wait(dbar(PV_DONE, bb), ((j - 2) >> 1) & 1, abort_flag, P.err)) {
+          // P buffer bb is free again: arm it for tile j, then let the other CTA fill it
+          mbar_arrive_expect_tx(dbar(P_REMOTE_FULL, bb), kPHalfBytes + kStatBytes);
+          mbar_arrive_remote(map_peer(dbar(PEER_P_FREE, bb), peer));
+        }
+        if (!mbar_wait_warp_cluster(dbar(P_REMOTE_FULL, bb), ph, abort_flag, P.err)) { ok = false; break; }
+        const float m_new = ld_shared_f32(sti0 + bb * kStatBytes + hl * 4);
+        const bool rescale_o = m_new != m_prev && m_prev != -INFINITY;
+        if (__any_sync(0xffffffffu, rescale_o)) {
+          // (P_REMOTE_FULL of tile j implies PV of tile j - 2 is done)
+          if (j >= 1 && !mbar_wait_warp(dbar(PV_DONE, bb ^ 1), ((j - 1) >> 1) & 1, abort_flag, P.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          rescale_o_cols(tl, 0, kDvHalf, rescale_o ? exp2f(m_prev - m_new) : 1.f);
+        }
+        m_prev = m_new;
+        tc_fence_before_sync();
+        mbar_arrive(dbar(PV_READY, bb));
+      }
+      if (ok && T > 0) mbar_arrive(pside_done);
+      if (ok && T > 0) {
+        const uint32_t si = sti0 + ((T - 1) & 1) * kStatBytes;
+        m_fin = m_prev;
+        l_fin = ld_shared_f32(si + (kHHalf + hl) * 4) + ld_shared_f32(si + (2 * kHHalf + hl) * 4);
+      }
+      c_lo = 0;
+      c_hi = 128;
     }
-    if (leader) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     // ------------------------------------------------------------ output --
-    if (ok && T >= 1) ok = mbar_wait_warp(o_done, (T - 1) & 1, abort_flag, P.err);
+    // every role has seen PV of tile T - 3 complete (directly, or through the
+    // other CTA's P rows of tile T - 1), so this parity is unambiguous
+    if (ok && T >= 1) ok = mbar_wait_warp(dbar(PV_DONE, (T - 1) & 1), ((T - 1) >> 1) & 1, abort_flag, P.err);
     if (ok) {
       tc_fence_after_sync();
       const int64_t rh = static_cast<int64_t>(r) * kH + h;
+      const bool stats_writer = own ? (sub == 0) : (sub == 1);  // one thread per head
       if (P.splits == 1) {
-        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+        const float inv = l_fin > 0.f ? 1.f / l_fin : 0.f;
         __nv_bfloat16* dst = P.out + rh * kDv + crank * kDvHalf;
 #pragma unroll 1
-        for (int c = 0; c < kDvHalf; c += 32) {
+        for (int c = c_lo; c < c_hi; c += 32) {
           float o[32];
           if (T >= 1) tmem_ld32(tl + c, o);
           else
@@ -544,13 +737,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
             *reinterpret_cast<uint4*>(dst + c + q * 8) = v;
           }
         }
-        if (P.lse != nullptr && crank == 0)
-          P.lse[rh] = l_run > 0.f ? (m_run + log2f(l_run)) * 0.6931471805599453f : -INFINITY;
+        if (P.lse != nullptr && crank == 0 && stats_writer)
+          P.lse[rh] = l_fin > 0.f ? (m_fin + log2f(l_fin)) * 0.6931471805599453f : -INFINITY;
       } else {
         const int64_t it = (static_cast<int64_t>(r) * P.splits + sp) * 2 + crank;
         float* dst = P.part_o + (it * kH + h) * kDvHalf;
 #pragma unroll 1
-        for (int c = 0; c < kDvHalf; c += 32) {
+        for (int c = c_lo; c < c_hi; c += 32) {
           float o[32];
           if (T >= 1) tmem_ld32(tl + c, o);
           else
@@ -559,8 +752,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
           for (int q = 0; q < 8; ++q)
             *reinterpret_cast<float4*>(dst + c + q * 4) = make_float4(o[q * 4], o[q * 4 + 1], o[q * 4 + 2], o[q * 4 + 3]);
         }
-        P.part_ml[(it * 2 + 0) * kH + h] = m_run;
-        P.part_ml[(it * 2 + 1) * kH + h] = l_run;
+        if (own && stats_writer) {
+          const int64_t ms = static_cast<int64_t>(r) * P.splits + sp;
+          P.part_ml[(ms * 2 + 0) * kH + h] = m_fin;
+          P.part_ml[(ms * 2 + 1) * kH + h] = l_fin;
+        }
       }
     }
   }
@@ -596,14 +792,14 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
     const int h = h0 + tid;
     float M = -INFINITY;
     for (int i = 0; i < splits; ++i) {
-      const int64_t it = (static_cast<int64_t>(r) * splits + i) * 2;
+      const int64_t it = static_cast<int64_t>(r) * splits + i;
       const float m = part_ml[(it * 2 + 0) * kH + h];
       const float l = part_ml[(it * 2 + 1) * kH + h];
       if (l > 0.f) M = fmaxf(M, m);
     }
     float Ls = 0.f;
     for (int i = 0; i < splits; ++i) {
-      const int64_t it = (static_cast<int64_t>(r) * splits + i) * 2;
+      const int64_t it = static_cast<int64_t>(r) * splits + i;
       const float m = part_ml[(it * 2 + 0) * kH + h];
       const float l = part_ml[(it * 2 + 1) * kH + h];
       const float wgt = (l > 0.f) ? exp2f(m - M) : 0.f;
