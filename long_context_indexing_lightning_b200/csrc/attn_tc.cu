@@ -56,10 +56,12 @@ constexpr int kAtomsMax = 5;             // 64-column swizzle atoms per CTA (CTA
 constexpr int kAtomBytes = kRows * 128;  // one atom of one tile: 8 KB
 constexpr int kStageBytes = kAtomsMax * kAtomBytes;  // 40 KB
 constexpr int kStages = 3;
+constexpr int kPrefetchAhead = 6;        // tiles whose rows are pulled into L2 ahead of their gather
 constexpr int kGatherWarps = 4;
 constexpr int kMmaWarp = 4;
 constexpr int kSoftWarps = 8;
-constexpr int kThreads = 32 * (kGatherWarps + 1 + kSoftWarps);  // 416
+constexpr int kPrefetchWarp = kGatherWarps + 1 + kSoftWarps;    // 13
+constexpr int kThreads = 32 * (kPrefetchWarp + 1);               // 448
 // tensor memory: O half [0, 256), Q columns [256, 256 + 160), S [416, 480)
 constexpr int kTmemCols = 512;
 constexpr int kQCol = 256;
@@ -255,6 +257,10 @@ __device__ __forceinline__ void bulk_to_peer(uint32_t dst, uint32_t src, uint32_
                "r"(src), "r"(bytes), "r"(bar)
                : "memory");
 }
+// Pull the 128-byte line at p into L2 (a hint: no data returned, nothing to wait for).
+__device__ __forceinline__ void prefetch_l2_line(const void* p) {
+  asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p));
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until at most N of this thread's bulk groups still read their source.
 template <int N>
@@ -312,6 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
   auto dbar = [&](int which, int b) { return bar0 + 8u * (2 * kStages + 6 + 2 * which + b); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+  volatile int* gather_progress = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = lane_id();
@@ -359,6 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
       }
     }
     *abort_flag = 0;
+    *gather_progress = 0;
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -371,7 +379,35 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
   cluster_sync_all();  // both CTAs' barriers exist (and are armed) before any remote arrival
   const uint32_t tmem = *tmem_slot;
 
-  if (warp < kGatherWarps) {
+  if (warp == kPrefetchWarp) {
+    // ------------------------------------------- L2 prefetch of the rows --
+    // Row reads from HBM take microseconds while a ring stage is held; pull
+    // each tile's rows into L2 up to kPrefetchAhead tiles before its gather,
+    // so the gather into the ring reads L2.  Lane l covers rows l and l + 32.
+    const char* kv_b = reinterpret_cast<const char*>(P.kv) + static_cast<int64_t>(b) * P.s_max * kDqk * 2;
+    const uint64_t t0 = global_timer_ns();
+    for (int t = 1; t < T; ++t) {
+      // stay at most kPrefetchAhead tiles ahead of the issued gathers (bounded)
+      bool go = true;
+      for (uint32_t i = 0; *gather_progress + kPrefetchAhead < t; ++i) {
+        if ((i & 63u) == 63u && (*abort_flag || global_timer_ns() - t0 > kWaitLimitNs)) {
+          go = false;
+          break;
+        }
+        __nanosleep(200);
+      }
+      if (!__all_sync(0xffffffffu, go)) break;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int rr = t * kRows + hh * 32 + lane;
+        const int s = rr < nrows ? __ldg(sel + rr) : -1;
+        if (s >= 0 && s < L) {
+          const char* row = kv_b + (static_cast<int64_t>(s) * kDqk + a0 * 64) * 2;
+          for (int c = 0; c < natoms; ++c) prefetch_l2_line(row + c * 128);
+        }
+      }
+    }
+  } else if (warp < kGatherWarps) {
     // --------------------------------------------------- gather (cp.async) --
     const int tid = threadIdx.x;
     const char* kv_b = reinterpret_cast<const char*>(P.kv) + static_cast<int64_t>(b) * P.s_max * kDqk * 2;
@@ -391,6 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
       if (crank == 0) gather_tile<kSplitCol / 64>(dst0, kv_b, a0, cur0, cur1, tid);
       else gather_tile<(kDqk - kSplitCol) / 64>(dst0, kv_b, a0, cur0, cur1, tid);
       cp_async_arrive(kv_full(st));
+      if (tid == 0) *gather_progress = j + 1;  // tiles whose gather has been issued
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
     if (__any_sync(0xffffffffu, bad) && lane == 0) raise_error(P.err, kErrBadIndex);
@@ -496,31 +533,42 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
       const bool leader = (hl == 0 && kh == 0);  // ships P rows; re-arms and releases the receive buffer
       float sreg[32], snext[32];
       float m_run = -INFINITY, l_half = 0.f;
-      int ix = (kh * 32 + lane < nrows) ? __ldg(sel + kh * 32 + lane) : -1;
-      if (T > 0) {
-        if (!mbar_wait_warp(s_full, 0, abort_flag, P.err)) {
-          ok = false;
-        } else {
-          tc_fence_after_sync();
-          tmem_ld32(tl + kSCol + 32 * kh, sreg);
-          tc_fence_before_sync();
-          mbar_arrive(s_empty);
-        }
-      }
+      // validity of this lane's row in tiles [vbase, vbase + 32), loaded in
+      // batches so that no global load is pending inside the loop (the
+      // release-ordered remote arrivals below would wait for it)
+      uint32_t vbits = 0;
+      int vbase = -32;
+      auto read_s = [&](float* dst) {
+        tc_fence_after_sync();
+        tmem_ld32(tl + kSCol + 32 * kh, dst);
+        tc_fence_before_sync();
+        mbar_arrive(s_empty);
+      };
+      // S(t) complete, tested without waiting; the whole warp agrees
+      auto s_ready = [&](int t) { return __all_sync(0xffffffffu, mbar_test_wait(s_full, t & 1)); };
+      bool have = false;  // sreg already holds S(j)
       for (int j = 0; ok && j < T; ++j) {
         const int bb = j & 1;
         const uint32_t ph = (j >> 1) & 1;
-        const uint32_t valid = __ballot_sync(0xffffffffu, ix >= 0 && ix < L);
-        const int jn = (j + 1) * kRows + kh * 32 + lane;
-        ix = (j + 1 < T && jn < nrows) ? __ldg(sel + jn) : -1;
-        // the next tile's logits first, so that its MMA runs under this softmax
-        if (j + 1 < T) {
-          if (!mbar_wait_warp(s_full, (j + 1) & 1, abort_flag, P.err)) { ok = false; break; }
-          tc_fence_after_sync();
-          tmem_ld32(tl + kSCol + 32 * kh, snext);
-          tc_fence_before_sync();
-          mbar_arrive(s_empty);
+        if (j >= vbase + 32) {
+          vbase = j;
+          vbits = 0;
+          for (int t = 0; t < 32 && j + t < T; ++t) {
+            const int rr = (j + t) * kRows + kh * 32 + lane;
+            const int ix = rr < nrows ? __ldg(sel + rr) : -1;
+            vbits |= ((ix >= 0 && ix < L) ? 1u : 0u) << t;
+          }
         }
+        const uint32_t valid = __ballot_sync(0xffffffffu, ((vbits >> (j - vbase)) & 1u) != 0);
+        if (!have) {
+          if (!mbar_wait_warp(s_full, j & 1, abort_flag, P.err)) { ok = false; break; }
+          read_s(sreg);
+        }
+        // the next tile's logits too if they are already there: its MMA then
+        // runs under this tile's softmax (never wait for them here: they
+        // hang on the next gather)
+        have = j + 1 < T && s_ready(j + 1);
+        if (have) read_s(snext);
         // S = S_0 + S_1: add the other CTA's partial for these heads
         if (!mbar_wait_warp_cluster(dbar(X_FULL, bb), ph, abort_flag, P.err)) { ok = false; break; }
         const uint32_t xb = xin0 + bb * kXBytes;
@@ -608,8 +656,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
             bulk_commit();
           }
         }
+        if (!have && j + 1 < T && s_ready(j + 1)) {
+          read_s(snext);
+          have = true;
+        }
+        if (have) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) sreg[i] = snext[i];
+          for (int i = 0; i < 32; ++i) sreg[i] = snext[i];
+        }
       }
       if (leader) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
       // both warps' partial sums of the last tile
