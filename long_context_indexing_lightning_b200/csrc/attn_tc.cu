@@ -8,37 +8,31 @@
 // 576-wide latent row per token; the value is the row's first 512 columns.
 //
 // One thread-block cluster of two CTAs per (query row, split of its selected
-// list).  The 576 latent columns are cut at 256: CTA 0 owns columns [0, 256),
-// CTA 1 owns [256, 576); CTA c also owns the softmax of heads [64c, 64c + 64).
-// Per 64-row tile, each CTA
+// list).  CTA c owns latent columns [256c, 256c + 256) and rope columns
+// [512 + 32c, 544 + 32c).  Per 64-row tile, each CTA
 //   * gathers only its own columns of the selected rows (cp.async, 16 bytes a
-//     thread, into a 3-stage ring in the 128-byte-swizzled K-major layout the
-//     MMA reads; padding and out-of-range rows are zero filled),
+//     thread, into a 3-stage ring in the swizzled K-major layouts the MMA
+//     reads: 128-byte swizzle for the latent part, 64-byte for the rope part;
+//     padding and out-of-range rows are zero filled), helped by a warp that
+//     pulls the rows of the next tiles into L2 ahead of time,
 //   * computes its partial logits S_c = Q_c K_c^T for all 128 heads (M = 128,
 //     N = 64, Q_c held in tensor memory),
-//   * reduce-scatter: ships the partial logits of the other CTA's 64 heads
-//     (16 KB, one bulk copy into the other CTA's shared memory) and adds the
-//     partial it receives for its own 64 heads, so each CTA holds the full
-//     S = S_0 + S_1 for the heads whose softmax it runs,
-//   * runs the online softmax of its 64 heads (base 2; the running max only
-//     moves, and O is rescaled in TMEM, when a tile max exceeds it by more
-//     than 8) and writes their P rows in bf16,
-//   * all-gather: ships those P rows (8 KB) and the heads' running max and
-//     partial sums to the other CTA, which rescales its O rows of those heads
-//     when the max moved,
+//   * swaps partials with the other CTA (32 KB, one bulk copy into the other
+//     CTA's shared memory), so both hold the same S = S_0 + S_1 (fp32
+//     addition is commutative: the two sums are bit-identical) and run the
+//     same online softmax over all heads (base 2; the running max only moves,
+//     and O is rescaled in TMEM, when a tile max exceeds it by more than 8),
 //   * accumulates its 256-column half of the output, O_c += P V_c, in TMEM
 //     (V_0 = latent columns [0, 256), V_1 = [256, 512): each CTA's value half
 //     lies inside the columns it already gathered).
-// Exchange buffers, P and the row statistics are double buffered so that
-// tile j's exchange overlaps tile j-1's softmax, and the softmax warps read
-// tile j+1's logits before they wait for tile j's partial.
-// Warps: 0-3 gather, 4 issues tcgen05.mma, 5-12 (two per TMEM lane quarter,
-// thread = head = TMEM lane): in the quarters of this CTA's own heads both
-// warps run the softmax, 32 of the tile's 64 columns each; in the other
-// quarters one warp ships the partial logits and one applies the other CTA's
-// P statistics to this CTA's O rows.  Long selections are split across
-// clusters and merged by a small combine kernel (log-sum-exp weights).  Every
-// wait is bounded.
+// The swap of tile j+1 is issued before the softmax of tile j and lands in
+// the second of two receive buffers, so the copy overlaps the softmax; one
+// warp does the copies and the cross-CTA signals.
+// Warps: 0-3 gather, 4 issues tcgen05.mma, 5-12 softmax (two per TMEM lane
+// quarter, thread = head = TMEM lane, 32 of the tile's 64 columns each), 13
+// L2 prefetch, 14 copies.  Long selections are split across clusters and
+// merged by a small combine kernel (log-sum-exp weights).  Every wait is
+// bounded.
 #include "dsa_common.cuh"
 #include "dsa_internal.h"
 
@@ -46,48 +40,46 @@ namespace dsa {
 namespace {
 
 constexpr int kH = 128;                  // heads == MMA M
-constexpr int kHHalf = 64;               // heads whose softmax one CTA runs
 constexpr int kDqk = 576;                // latent 512 + rope 64
 constexpr int kDv = 512;
 constexpr int kDvHalf = 256;
 constexpr int kRows = 64;                // selected rows per tile (MMA N of S, K of PV)
-constexpr int kSplitCol = 256;           // CTA 0: columns [0, 256); CTA 1: [256, 576)
-constexpr int kAtomsMax = 5;             // 64-column swizzle atoms per CTA (CTA 0 uses 4)
-constexpr int kAtomBytes = kRows * 128;  // one atom of one tile: 8 KB
-constexpr int kStageBytes = kAtomsMax * kAtomBytes;  // 40 KB
+constexpr int kLatCols = 256;            // latent columns per CTA (also its value half)
+constexpr int kLatAtoms = kLatCols / 64; // 64-column, 128-byte-swizzled atoms per tile
+constexpr int kRopeCols = 32;            // rope columns per CTA
+constexpr int kAtomBytes = kRows * 128;  // one latent atom of one tile: 8 KB
+constexpr int kRopeBytes = kRows * 64;   // the rope piece of one tile (64-byte swizzle): 4 KB
+constexpr int kStageBytes = kLatAtoms * kAtomBytes + kRopeBytes;  // 36 KB
+constexpr int kQk = kLatCols + kRopeCols;  // 288 logit columns per CTA: 18 MMA K-steps
 constexpr int kStages = 3;
 constexpr int kPrefetchAhead = 6;        // tiles whose rows are pulled into L2 ahead of their gather
 constexpr int kGatherWarps = 4;
 constexpr int kMmaWarp = 4;
 constexpr int kSoftWarps = 8;
-constexpr int kPrefetchWarp = kGatherWarps + 1 + kSoftWarps;    // 13
-constexpr int kThreads = 32 * (kPrefetchWarp + 1);               // 448
-// tensor memory: O half [0, 256), Q columns [256, 256 + 160), S [416, 480)
+constexpr int kSoftThreads = 32 * kSoftWarps;
+constexpr int kPrefetchWarp = kGatherWarps + 1 + kSoftWarps;  // 13
+constexpr int kCommWarp = kPrefetchWarp + 1;                   // 14
+constexpr int kThreads = 32 * (kCommWarp + 1);                 // 480
+// tensor memory: O half [0, 256), Q columns [256, 256 + 144), S [400, 464)
 constexpr int kTmemCols = 512;
 constexpr int kQCol = 256;
-constexpr int kSCol = 416;
+constexpr int kSCol = kQCol + kQk / 2;
 
-// shared memory map (from a 1024-aligned base); [2] = double buffered by tile parity
-constexpr int kPBytes = kH * kRows * 2;      // P: 128 heads x 64 rows bf16, SW128 K-major
-constexpr int kPHalfBytes = kPBytes / 2;     // the 64 rows of one CTA's heads (contiguous)
-constexpr int kXBytes = kHHalf * kRows * 4;  // partial logits of 64 heads: [16 x 4 rows][64 heads] fp32
-constexpr int kStatBytes = 3 * kHHalf * 4;   // per head: running max, partial sum of each softmax warp
+// shared memory map (from a 1024-aligned base)
+constexpr int kPBytes = kH * kRows * 2;  // P: 128 heads x 64 rows bf16, SW128 K-major
+constexpr int kXBytes = kH * kRows * 4;  // partial logits: [16 x 4 rows][128 heads] fp32
 constexpr int kOffKV = 0;
 constexpr int kOffP = kOffKV + kStages * kStageBytes;
-constexpr int kOffXin = kOffP + 2 * kPBytes;      // partial logits received for this CTA's heads
-constexpr int kOffXout = kOffXin + 2 * kXBytes;   // partial logits of the other CTA's heads, to ship
-constexpr int kOffStOut = kOffXout + 2 * kXBytes; // statistics of this CTA's heads, to ship
-constexpr int kOffStIn = kOffStOut + 2 * kStatBytes;
-constexpr int kOffRed = kOffStIn + 2 * kStatBytes;  // tile max of each softmax warp: [2][2 warps][64]
-// barriers: kv_full[3], kv_empty[3], q_ready, s_full, s_empty, mma_done, fin,
-// pside_done, then 11 double-buffered ones (see the enum in the kernel)
-constexpr int kNumDBars = 11;
-constexpr int kNumBars = 2 * kStages + 6 + 2 * kNumDBars;
-constexpr int kOffBar = kOffRed + 2 * 2 * kHHalf * 4;
+constexpr int kOffXin = kOffP + kPBytes;         // the other CTA's partials, [tile parity]
+constexpr int kOffXout = kOffXin + 2 * kXBytes;  // this CTA's partial, for the bulk copy
+constexpr int kOffRed = kOffXout + kXBytes;  // tile max of each softmax warp: [2][2 warps][128]
+// barriers: kv_full[3], kv_empty[3], then the 17 named in the kernel
+constexpr int kNumBars = 2 * kStages + 17;
+constexpr int kOffBar = kOffRed + 2 * 2 * kH * 4;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory");
-static_assert(kOffP % 1024 == 0 && kPBytes % 1024 == 0, "P tiles must stay 1024-aligned");
+static_assert(kOffP % 1024 == 0 && kPBytes % 1024 == 0, "P tile must stay 1024-aligned");
 
 struct AttnParams {
   const uint16_t* q;        // [R][128][576] bf16
@@ -218,20 +210,22 @@ __device__ __forceinline__ float fast_exp2(float x) {
 
 
 // Gather this CTA's NA atoms (64 latent columns each) of the tile's 64 rows.
-// Lane l of each gather warp holds the global rows of tile rows l and l + 32.
+// Gather warp w covers tile rows [16w, 16w + 16); in group g its lane l moves
+// 16-byte chunk l % 8 of every atom of row 16w + 4g + l / 8, whose cache row
+// is rows[g] (-1: zero fill).  No per-copy shuffles or divisions.
 template <int NA>
-__device__ __forceinline__ void gather_tile(uint32_t dst0, const char* kv_b, int a0, int cur0, int cur1, int tid) {
-#pragma unroll 4
-  for (int i = 0; i < NA * 4; ++i) {
-    const int x = i * 128 + tid;
-    const int row = x / (NA * 8), cc = x % (NA * 8);
-    const int v0 = __shfl_sync(0xffffffffu, cur0, row & 31);
-    const int v1 = __shfl_sync(0xffffffffu, cur1, row & 31);
-    const int s = row < 32 ? v0 : v1;
-    const int kb = cc >> 3, c = cc & 7;
-    const uint32_t dst = dst0 + kb * kAtomBytes + row * 128 + ((c ^ (row & 7)) << 4);
-    const char* src = kv_b + (s >= 0 ? (static_cast<int64_t>(s) * kDqk + (a0 + kb) * 64) * 2 + c * 16 : 0);
-    cp_async16(dst, src, s >= 0 ? 16u : 0u);
+__device__ __forceinline__ void gather_tile(uint32_t dst0, const char* kv_b, int a0, const int* rows, int w, int lane) {
+  const int c = lane & 7;
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    const int row = w * 16 + g * 4 + (lane >> 3);
+    const int s = rows[g];
+    const char* src = kv_b + (s >= 0 ? (static_cast<int64_t>(s) * kDqk + a0 * 64) * 2 + c * 16 : 0);
+    const uint32_t dst = dst0 + row * 128 + ((c ^ (row & 7)) << 4);
+    const uint32_t nbytes = s >= 0 ? 16u : 0u;
+    const int step = s >= 0 ? 128 : 0;
+#pragma unroll
+    for (int a = 0; a < NA; ++a) cp_async16(dst + a * kAtomBytes, src + a * step, nbytes);
   }
 }
 
@@ -288,6 +282,25 @@ __device__ __forceinline__ void rescale_o_cols(uint32_t tl, int c0, int c1, floa
   tmem_st_wait();
 }
 
+// Gather this CTA's 32 rope columns of the tile's 64 rows into the piece at
+// dst0: 64-byte rows, 64-byte swizzle (16-byte chunk c of row r sits at chunk
+// c ^ ((r & 7) >> 1)).  Gather warp w covers rows [16w, 16w + 16); in group g
+// its lane l moves chunk l % 4 of row 16w + 8g + l / 4, whose cache row is
+// rows[g] (-1: zero fill).
+__device__ __forceinline__ void gather_rope(uint32_t dst0, const char* kv_b, int col0, const int* rows, int w,
+                                            int lane) {
+  const int c = lane & 3;
+#pragma unroll
+  for (int g = 0; g < 2; ++g) {
+    const int row = w * 16 + g * 8 + (lane >> 2);
+    const int s = rows[g];
+    const char* src = kv_b + (s >= 0 ? (static_cast<int64_t>(s) * kDqk + col0) * 2 + c * 16 : 0);
+    const uint32_t dst = dst0 + (row >> 3) * 512 + (row & 7) * 64 + ((c ^ ((row & 7) >> 1)) << 4);
+    cp_async16(dst, src, s >= 0 ? 16u : 0u);
+  }
+}
+constexpr uint32_t kLayoutSW64 = 4;
+
 __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -295,37 +308,31 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
   const uint32_t bar0 = sbase + kOffBar;
   auto kv_full = [&](int i) { return bar0 + 8u * i; };
   auto kv_empty = [&](int i) { return bar0 + 8u * (kStages + i); };
-  const uint32_t q_ready = bar0 + 8u * (2 * kStages + 0);
-  const uint32_t s_full = bar0 + 8u * (2 * kStages + 1);
-  const uint32_t s_empty = bar0 + 8u * (2 * kStages + 2);
-  const uint32_t mma_done = bar0 + 8u * (2 * kStages + 3);
-  const uint32_t fin = bar0 + 8u * (2 * kStages + 4);
-  const uint32_t pside_done = bar0 + 8u * (2 * kStages + 5);  // P-side warps saw the last tile's statistics
-  // double-buffered barriers, index [tile parity]
-  enum {
-    X_FULL,         // received partial logits landed (armed here, bulk copy from the other CTA)
-    X_EMPTY,        // the other CTA has added our shipped partial (remote arrive)
-    XOUT_WRITTEN,   // ship warps staged the outgoing partial
-    XOUT_FREE,      // the outgoing bulk copy has read the staging buffer
-    XIN_READ,       // softmax warps have added the received partial
-    P_OWN_WRITTEN,  // softmax warps wrote their heads' P rows and statistics
-    PEER_P_FREE,    // the other CTA's P buffer is free (its PV two tiles back is done; remote arrive)
-    P_REMOTE_FULL,  // the other CTA's P rows and statistics landed (armed here, bulk copy)
-    PV_READY,       // all P rows present and every O row rescaled: PV may run
-    PV_DONE,        // PV of this buffer's last tile is done (tcgen05.commit)
-    RED_FULL        // both softmax warps of each head published their tile max
-  };
-  auto dbar = [&](int which, int b) { return bar0 + 8u * (2 * kStages + 6 + 2 * which + b); };
+  const uint32_t nb0 = bar0 + 8u * (2 * kStages);
+  const uint32_t q_ready = nb0 + 0;
+  const uint32_t s_full = nb0 + 8;        // S(j) in TMEM (tcgen05.commit)
+  const uint32_t s_empty = nb0 + 16;      // every softmax thread has read S(j)
+  const uint32_t mma_done = nb0 + 24;
+  const uint32_t fin = nb0 + 32;          // final partial sums published
+  const uint32_t xout_written = nb0 + 40; // every softmax thread has written its partial of tile j
+  const uint32_t xout_free = nb0 + 48;    // the bulk copy of tile j has read xout
+  const uint32_t pv_ready = nb0 + 56;     // P of tile j written and O rescaled: PV may run
+  const uint32_t pv_done = nb0 + 64;      // PV of tile j done (tcgen05.commit)
+  // [tile parity]:
+  auto red_full = [&](int bb) { return nb0 + 72 + 8u * bb; };   // tile max published
+  auto x_full = [&](int bb) { return nb0 + 88 + 8u * bb; };     // the other CTA's partial landed in xin[bb] (tx)
+  auto x_empty = [&](int bb) { return nb0 + 104 + 8u * bb; };   // the other CTA has added what we sent to its xin[bb]
+  auto xin_read = [&](int bb) { return nb0 + 120 + 8u * bb; };  // every softmax thread has added xin[bb]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
   volatile int* gather_progress = reinterpret_cast<volatile int*>(smem + kOffMisc + 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = lane_id();
-  const uint32_t crank = cluster_rank();  // 0: latent columns [0, 256), heads [0, 64); 1: [256, 576), [64, 128)
+  const uint32_t crank = cluster_rank();  // latent columns [256c, 256c + 256), rope [512 + 32c, 544 + 32c)
   const uint32_t peer = crank ^ 1u;
-  const int a0 = crank == 0 ? 0 : kSplitCol / 64;  // first 64-column atom of this CTA
-  const int natoms = crank == 0 ? kSplitCol / 64 : (kDqk - kSplitCol) / 64;
+  const int a0 = crank * kLatAtoms;                       // first 64-column latent atom of this CTA
+  const int rope0 = kLatCols * 2 + crank * kRopeCols;     // first rope column of this CTA
   // work item of the cluster
   const int item = blockIdx.x >> 1;
   const int sp = item % P.splits;
@@ -336,35 +343,30 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
   const int nrows = max(0, min(P.rows_per_split, P.k - row0));
   const int T = (nrows + kRows - 1) / kRows;
   const int32_t* sel = P.idx + static_cast<int64_t>(r) * P.k + row0;
+  const char* kv_b = reinterpret_cast<const char*>(P.kv) + static_cast<int64_t>(b) * P.s_max * kDqk * 2;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(kv_full(i), 32 * kGatherWarps);
       mbar_init(kv_empty(i), 1);
     }
-    mbar_init(q_ready, 32 * kSoftWarps);
+    mbar_init(q_ready, kSoftThreads);
     mbar_init(s_full, 1);
-    mbar_init(s_empty, 192);  // 128 softmax threads + 64 ship threads read S
+    mbar_init(s_empty, kSoftThreads);
     mbar_init(mma_done, 1);
-    mbar_init(fin, 128);
-    mbar_init(pside_done, 64);
+    mbar_init(fin, kSoftThreads);
     for (int bb = 0; bb < 2; ++bb) {
-      mbar_init(dbar(X_FULL, bb), 1);
-      mbar_init(dbar(X_EMPTY, bb), 1);
-      mbar_init(dbar(XOUT_WRITTEN, bb), 64);
-      mbar_init(dbar(XOUT_FREE, bb), 1);
-      mbar_init(dbar(XIN_READ, bb), 128);
-      mbar_init(dbar(P_OWN_WRITTEN, bb), 128);
-      mbar_init(dbar(PEER_P_FREE, bb), 1);
-      mbar_init(dbar(P_REMOTE_FULL, bb), 1);
-      mbar_init(dbar(PV_READY, bb), 192);  // 128 softmax threads + 64 P-side threads
-      mbar_init(dbar(PV_DONE, bb), 1);
-      mbar_init(dbar(RED_FULL, bb), 128);
-      if (bb < T) {  // armed for tiles 0 and 1; later tiles re-arm one round ahead
-        mbar_arrive_expect_tx(dbar(X_FULL, bb), kXBytes);
-        mbar_arrive_expect_tx(dbar(P_REMOTE_FULL, bb), kPHalfBytes + kStatBytes);
-      }
+      mbar_init(x_full(bb), 1);
+      mbar_init(x_empty(bb), 1);
+      mbar_init(xin_read(bb), kSoftThreads);
+      if (bb < T) mbar_arrive_expect_tx(x_full(bb), kXBytes);  // armed for tiles 0, 1; later re-armed ahead
     }
+    mbar_init(xout_written, kSoftThreads);
+    mbar_init(xout_free, 1);
+    mbar_init(pv_ready, kSoftThreads);
+    mbar_init(pv_done, 1);
+    mbar_init(red_full(0), kSoftThreads);
+    mbar_init(red_full(1), kSoftThreads);
     *abort_flag = 0;
     *gather_progress = 0;
     fence_mbar_init();
@@ -379,12 +381,38 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
   cluster_sync_all();  // both CTAs' barriers exist (and are armed) before any remote arrival
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == kPrefetchWarp) {
+  if (warp == kCommWarp) {
+    // --------------------------------------- copies and cross-CTA signals --
+    // Lane 0 issues the bulk copies; lane 1, which has none in flight, sends
+    // the remote signals (a release-ordered arrive from a thread with a copy
+    // in flight waits for that copy).
+    if (lane == 0) {
+      for (int j = 0; j < T; ++j) {
+        const int bb = j & 1;
+        // this CTA's partial of tile j, once written and once the other CTA
+        // has added the one that last used its buffer (tile j - 2)
+        if (!mbar_wait(xout_written, j & 1, abort_flag, P.err)) break;
+        if (j >= 2 && !mbar_wait_cluster1(x_empty(bb), ((j - 2) >> 1) & 1, abort_flag, P.err)) break;
+        bulk_to_peer(map_peer(sbase + kOffXin + bb * kXBytes, peer), sbase + kOffXout, kXBytes,
+                     map_peer(x_full(bb), peer));
+        bulk_commit();
+        bulk_wait_read<0>();
+        mbar_arrive(xout_free);
+      }
+      asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    } else if (lane == 1) {
+      // our receive buffer [j & 1] is free once tile j's partial was added here
+      for (int j = 0; j + 2 < T; ++j) {
+        if (!mbar_wait(xin_read(j & 1), (j >> 1) & 1, abort_flag, P.err)) break;
+        mbar_arrive_remote(map_peer(x_empty(j & 1), peer));
+      }
+    }
+    __syncwarp();
+  } else if (warp == kPrefetchWarp) {
     // ------------------------------------------- L2 prefetch of the rows --
     // Row reads from HBM take microseconds while a ring stage is held; pull
     // each tile's rows into L2 up to kPrefetchAhead tiles before its gather,
     // so the gather into the ring reads L2.  Lane l covers rows l and l + 32.
-    const char* kv_b = reinterpret_cast<const char*>(P.kv) + static_cast<int64_t>(b) * P.s_max * kDqk * 2;
     const uint64_t t0 = global_timer_ns();
     for (int t = 1; t < T; ++t) {
       // stay at most kPrefetchAhead tiles ahead of the issued gathers (bounded)
@@ -402,32 +430,44 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
         const int rr = t * kRows + hh * 32 + lane;
         const int s = rr < nrows ? __ldg(sel + rr) : -1;
         if (s >= 0 && s < L) {
-          const char* row = kv_b + (static_cast<int64_t>(s) * kDqk + a0 * 64) * 2;
-          for (int c = 0; c < natoms; ++c) prefetch_l2_line(row + c * 128);
+          const char* row = kv_b + static_cast<int64_t>(s) * kDqk * 2;
+          for (int c = 0; c < kLatAtoms; ++c) prefetch_l2_line(row + (a0 + c) * 128);
+          prefetch_l2_line(row + kLatCols * 4);  // the line holding both CTAs' rope columns
         }
       }
     }
   } else if (warp < kGatherWarps) {
     // --------------------------------------------------- gather (cp.async) --
-    const int tid = threadIdx.x;
-    const char* kv_b = reinterpret_cast<const char*>(P.kv) + static_cast<int64_t>(b) * P.s_max * kDqk * 2;
     bool bad = false;
-    int nx0 = (lane < nrows) ? __ldg(sel + lane) : -1;
-    int nx1 = (lane + 32 < nrows) ? __ldg(sel + lane + 32) : -1;
+    const int myrow = warp * 16 + (lane >> 3);  // + 4 g: this lane's rows of each tile
+    const int myrope = warp * 16 + (lane >> 2);  // + 8 g: this lane's rope rows
+    int nx[4], rnx[2];
+#pragma unroll
+    for (int g = 0; g < 4; ++g) nx[g] = (myrow + 4 * g < nrows) ? __ldg(sel + myrow + 4 * g) : -1;
+#pragma unroll
+    for (int g = 0; g < 2; ++g) rnx[g] = (myrope + 8 * g < nrows) ? __ldg(sel + myrope + 8 * g) : -1;
     for (int j = 0; j < T; ++j) {
       const int st = j % kStages;
-      int cur0 = nx0, cur1 = nx1;
-      if (cur0 >= L) { bad = true; cur0 = -1; }
-      if (cur1 >= L) { bad = true; cur1 = -1; }
-      const int jn = (j + 1) * kRows + lane;
-      nx0 = (j + 1 < T && jn < nrows) ? __ldg(sel + jn) : -1;
-      nx1 = (j + 1 < T && jn + 32 < nrows) ? __ldg(sel + jn + 32) : -1;
+      int cur[4], rcur[2];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        cur[g] = nx[g];
+        if (cur[g] >= L) { bad = true; cur[g] = -1; }
+        const int rn = (j + 1) * kRows + myrow + 4 * g;
+        nx[g] = (j + 1 < T && rn < nrows) ? __ldg(sel + rn) : -1;
+      }
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {
+        rcur[g] = rnx[g] < L ? rnx[g] : -1;  // (out-of-range rows are flagged above)
+        const int rn = (j + 1) * kRows + myrope + 8 * g;
+        rnx[g] = (j + 1 < T && rn < nrows) ? __ldg(sel + rn) : -1;
+      }
       if (!mbar_wait_warp(kv_empty(st), ((j / kStages) & 1) ^ 1, abort_flag, P.err)) break;
       const uint32_t dst0 = sbase + kOffKV + st * kStageBytes;
-      if (crank == 0) gather_tile<kSplitCol / 64>(dst0, kv_b, a0, cur0, cur1, tid);
-      else gather_tile<(kDqk - kSplitCol) / 64>(dst0, kv_b, a0, cur0, cur1, tid);
+      gather_tile<kLatAtoms>(dst0, kv_b, a0, cur, warp, lane);
+      gather_rope(dst0 + kLatAtoms * kAtomBytes, kv_b, rope0, rcur, warp, lane);
       cp_async_arrive(kv_full(st));
-      if (tid == 0) *gather_progress = j + 1;  // tiles whose gather has been issued
+      if (threadIdx.x == 0) *gather_progress = j + 1;  // tiles whose gather has been issued
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
     if (__any_sync(0xffffffffu, bad) && lane == 0) raise_error(P.err, kErrBadIndex);
@@ -438,24 +478,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
       constexpr uint32_t idesc_o = idesc_bf16_f32_bmn(kH, kDvHalf);
       const uint64_t kv_desc0 = sdesc(sbase + kOffKV, 16, 1024, kLayoutSW128);      // K-major rows (logits)
       const uint64_t v_desc0 = sdesc(sbase + kOffKV, kAtomBytes, 1024, kLayoutSW128);  // MN-major columns (value)
-      const uint64_t p_desc0 = sdesc(sbase + kOffP, 16, 1024, kLayoutSW128);
+      const uint64_t p_desc = sdesc(sbase + kOffP, 16, 1024, kLayoutSW128);
+      const uint64_t rope_desc0 = sdesc(sbase + kOffKV + kLatAtoms * kAtomBytes, 16, 512, kLayoutSW64);  // K-major rope rows
       const uint32_t q_t = tmem + kQCol, s_t = tmem + kSCol;
       bool ok = mbar_wait(q_ready, 0, abort_flag, P.err);
       int nq = 0, np = 0;
       uint64_t t0 = 0;
       uint32_t spins = 0;
       while (ok && np < T) {
-        // O += P(np) V(np) once every P row is in place and O rows are rescaled
-        if (np < nq && mbar_test_wait(dbar(PV_READY, np & 1), (np >> 1) & 1)) {
+        // O += P(np) V(np) once P is written and O rescaled (frees the tile's stage)
+        if (np < nq && mbar_test_wait(pv_ready, np & 1)) {
           tc_fence_after_sync();
           const uint64_t st_off = static_cast<uint64_t>(((np % kStages) * kStageBytes) >> 4);
-          const uint64_t p_off = static_cast<uint64_t>(((np & 1) * kPBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < kRows / 16; ++kk)
-            tc_mma_f16(tmem, p_desc0 + p_off + ((kk * 32) >> 4), v_desc0 + st_off + ((kk * 16 * 128) >> 4), idesc_o,
+            tc_mma_f16(tmem, p_desc + ((kk * 32) >> 4), v_desc0 + st_off + ((kk * 16 * 128) >> 4), idesc_o,
                        (np > 0 || kk > 0) ? 1u : 0u);
           tc_commit(kv_empty(np % kStages));
-          tc_commit(dbar(PV_DONE, np & 1));
+          tc_commit(pv_done);
           ++np;
           spins = 0;
           continue;
@@ -466,16 +506,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
           fence_proxy_async_smem();  // cp.async (generic proxy) writes -> tensor-core reads
           tc_fence_after_sync();
           const uint64_t kvs = kv_desc0 + static_cast<uint64_t>(((nq % kStages) * kStageBytes) >> 4);
-          const int nk = natoms * 4;
-          for (int kk = 0; kk < nk; ++kk) {
+#pragma unroll
+          for (int kk = 0; kk < kLatAtoms * 4; ++kk) {
             const uint32_t b_off = (kk >> 2) * kAtomBytes + (kk & 3) * 32;
             tc_mma_f16_ts(s_t, q_t + kk * 8, kvs + (b_off >> 4), idesc_s, kk > 0 ? 1u : 0u);
           }
+          const uint64_t ropes = rope_desc0 + static_cast<uint64_t>(((nq % kStages) * kStageBytes) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < kRopeCols / 16; ++kk)
+            tc_mma_f16_ts(s_t, q_t + (kLatAtoms * 4 + kk) * 8, ropes + ((kk * 32) >> 4), idesc_s, 1u);
           tc_commit(s_full);
           ++nq;
           spins = 0;
           continue;
         }
+        // nothing to issue: back off so this lane does not take issue slots
+        // and shared-memory bandwidth from the gather and softmax warps
+        __nanosleep(32);
         if ((++spins & 63u) == 0u) {
           const uint64_t now = global_timer_ns();
           if (t0 == 0 || spins == 64) t0 = now;
@@ -493,22 +540,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
     }
     __syncwarp();
   } else {
-    // ------------------------------------- Q to TMEM, then three roles --
+    // ------------------------------------------- softmax (all 128 heads) --
     const int quarter = warp & 3;
-    const int sub = (warp - (kGatherWarps + 1)) >> 2;  // which of the quarter's two warps
-    const int h = quarter * 32 + lane;                 // head == TMEM lane
-    const int hl = h & (kHHalf - 1);                   // index among its CTA's 64 heads
-    const bool own = static_cast<uint32_t>(quarter >> 1) == crank;
+    const int kh = (warp - (kGatherWarps + 1)) >> 2;  // columns [32 kh, 32 kh + 32) of each tile
+    const int h = quarter * 32 + lane;                // head == TMEM lane
     const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    const bool leader = (h == 0 && kh == 0);          // re-arms the receive buffer
     {
       // this CTA's columns of q[r, h, :] as packed bf16 pairs (element 2i in
       // the low half of column i); the quarter's two warps take half each
-      const uint4* qs = reinterpret_cast<const uint4*>(P.q + (static_cast<int64_t>(r) * kH + h) * kDqk + a0 * 64);
-      for (int c = sub * natoms; c < (sub + 1) * natoms; ++c) {
+      const uint16_t* qrow = P.q + (static_cast<int64_t>(r) * kH + h) * kDqk;
+      constexpr int kChunks = kQk / 32;  // 32-column chunks: latent 0..7, rope 8
+      for (int c = kh == 0 ? 0 : (kChunks + 1) / 2; c < (kh == 0 ? (kChunks + 1) / 2 : kChunks); ++c) {
+        const uint4* qs = reinterpret_cast<const uint4*>(qrow + (c < kLatCols / 32 ? a0 * 64 + c * 32 : rope0));
         uint32_t u[16];
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
-          const uint4 x = __ldg(qs + c * 4 + v);
+          const uint4 x = __ldg(qs + v);
           u[4 * v + 0] = x.x;
           u[4 * v + 1] = x.y;
           u[4 * v + 2] = x.z;
@@ -520,258 +568,149 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
       tc_fence_before_sync();
       mbar_arrive(q_ready);
     }
-    const uint32_t p0 = sbase + kOffP;
-    const uint32_t xin0 = sbase + kOffXin, xout0 = sbase + kOffXout;
-    const uint32_t sto0 = sbase + kOffStOut, sti0 = sbase + kOffStIn;
+    const uint32_t xin = sbase + kOffXin, xout = sbase + kOffXout;
     bool ok = true;
-    float m_fin = -INFINITY, l_fin = 0.f;  // head h's final running max and sum
-    int c_lo = 0, c_hi = 0;                // this thread's O columns in the epilogue
-
-    if (own) {
-      // ---------------------- softmax of this CTA's heads, 32 columns a warp --
-      const int kh = sub;
-      const bool leader = (hl == 0 && kh == 0);  // ships P rows; re-arms and releases the receive buffer
-      float sreg[32], snext[32];
-      float m_run = -INFINITY, l_half = 0.f;
-      // validity of this lane's row in tiles [vbase, vbase + 32), loaded in
-      // batches so that no global load is pending inside the loop (the
-      // release-ordered remote arrivals below would wait for it)
-      uint32_t vbits = 0;
-      int vbase = -32;
-      auto read_s = [&](float* dst) {
-        tc_fence_after_sync();
-        tmem_ld32(tl + kSCol + 32 * kh, dst);
-        tc_fence_before_sync();
-        mbar_arrive(s_empty);
+    float sreg[32], snext[32];
+    float m_run = -INFINITY, l_half = 0.f;
+    // S(t): this thread's 32 columns, then S(t) may be overwritten
+    auto read_s = [&](float* dst) {
+      tc_fence_after_sync();
+      tmem_ld32(tl + kSCol + 32 * kh, dst);
+      tc_fence_before_sync();
+      mbar_arrive(s_empty);
+    };
+    // this thread's partial of the tile, chunk-major [16 x 4 rows][128 heads]
+    auto write_x = [&](const float* v) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(xout + ((kh * 8 + c) * kH + h) * 16),
+                     "f"(v[4 * c]), "f"(v[4 * c + 1]), "f"(v[4 * c + 2]), "f"(v[4 * c + 3])
+                     : "memory");
+      fence_proxy_async_smem();  // generic writes -> bulk-copy reads
+      mbar_arrive(xout_written);
+    };
+    // S(t) complete, tested without waiting; the whole warp agrees
+    auto s_ready = [&](int t) { return __all_sync(0xffffffffu, mbar_test_wait(s_full, t & 1)); };
+    // validity of this lane's row in tiles [vbase, vbase + 32), loaded in
+    // batches so that no global load is pending inside the loop
+    uint32_t vbits = 0;
+    int vbase = -32;
+    if (T > 0) {
+      if (!mbar_wait_warp(s_full, 0, abort_flag, P.err)) {
+        ok = false;
+      } else {
+        read_s(sreg);
+        write_x(sreg);
+      }
+    }
+    for (int j = 0; ok && j < T; ++j) {
+      const int bb = j & 1;
+      if (j >= vbase + 32) {
+        vbase = j;
+        vbits = 0;
+        for (int t = 0; t < 32 && j + t < T; ++t) {
+          const int rr = (j + t) * kRows + kh * 32 + lane;
+          const int ix = rr < nrows ? __ldg(sel + rr) : -1;
+          vbits |= ((ix >= 0 && ix < L) ? 1u : 0u) << t;
+        }
+      }
+      const uint32_t valid = __ballot_sync(0xffffffffu, ((vbits >> (j - vbase)) & 1u) != 0);
+      // S = S_0 + S_1
+      if (!mbar_wait_warp_cluster(x_full(bb), (j >> 1) & 1, abort_flag, P.err)) { ok = false; break; }
+      // arm for tile j + 2 (the other CTA sends it only after x_empty of tile j)
+      if (leader && j + 2 < T) mbar_arrive_expect_tx(x_full(bb), kXBytes);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float4 v = ld_shared_v4f(xin + bb * kXBytes + ((kh * 8 + c) * kH + h) * 16);
+        sreg[4 * c] += v.x;
+        sreg[4 * c + 1] += v.y;
+        sreg[4 * c + 2] += v.z;
+        sreg[4 * c + 3] += v.w;
+      }
+      mbar_arrive(xin_read(bb));
+      // tile j + 1's partial goes out now if its logits are ready, so the
+      // copy runs under this tile's softmax
+      bool shipped = false;
+      auto ship_next = [&]() -> bool {
+        read_s(snext);
+        // the copy of tile j has read xout
+        if (!mbar_wait_warp(xout_free, j & 1, abort_flag, P.err)) return false;
+        write_x(snext);
+        shipped = true;
+        return true;
       };
-      // S(t) complete, tested without waiting; the whole warp agrees
-      auto s_ready = [&](int t) { return __all_sync(0xffffffffu, mbar_test_wait(s_full, t & 1)); };
-      bool have = false;  // sreg already holds S(j)
-      for (int j = 0; ok && j < T; ++j) {
-        const int bb = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (j >= vbase + 32) {
-          vbase = j;
-          vbits = 0;
-          for (int t = 0; t < 32 && j + t < T; ++t) {
-            const int rr = (j + t) * kRows + kh * 32 + lane;
-            const int ix = rr < nrows ? __ldg(sel + rr) : -1;
-            vbits |= ((ix >= 0 && ix < L) ? 1u : 0u) << t;
-          }
-        }
-        const uint32_t valid = __ballot_sync(0xffffffffu, ((vbits >> (j - vbase)) & 1u) != 0);
-        if (!have) {
-          if (!mbar_wait_warp(s_full, j & 1, abort_flag, P.err)) { ok = false; break; }
-          read_s(sreg);
-        }
-        // the next tile's logits too if they are already there: its MMA then
-        // runs under this tile's softmax (never wait for them here: they
-        // hang on the next gather)
-        have = j + 1 < T && s_ready(j + 1);
-        if (have) read_s(snext);
-        // S = S_0 + S_1: add the other CTA's partial for these heads
-        if (!mbar_wait_warp_cluster(dbar(X_FULL, bb), ph, abort_flag, P.err)) { ok = false; break; }
-        const uint32_t xb = xin0 + bb * kXBytes;
+      if (j + 1 < T && s_ready(j + 1) && !ship_next()) { ok = false; break; }
+      float mt = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const float4 v = ld_shared_v4f(xb + ((kh * 8 + c) * kHHalf + hl) * 16);
-          sreg[4 * c] += v.x;
-          sreg[4 * c + 1] += v.y;
-          sreg[4 * c + 2] += v.z;
-          sreg[4 * c + 3] += v.w;
-        }
-        mbar_arrive(dbar(XIN_READ, bb));
-        if (leader && mbar_wait(dbar(XIN_READ, bb), ph, abort_flag, P.err) && j + 2 < T) {
-          mbar_arrive_expect_tx(dbar(X_FULL, bb), kXBytes);  // armed for tile j + 2 ...
-          mbar_arrive_remote(map_peer(dbar(X_EMPTY, bb), peer));  // ... before the other CTA may send it
-        }
-        float mt = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const bool v = ((valid >> i) & 1u) != 0;
-          sreg[i] = v ? sreg[i] * P.scale_log2 : -INFINITY;
-          mt = fmaxf(mt, sreg[i]);
-        }
-        // tile max over all 64 columns: swap with the head's other warp
-        const uint32_t red = sbase + kOffRed + bb * (2 * kHHalf * 4);
-        st_shared_f32(red + (kh * kHHalf + hl) * 4, mt);
-        mbar_arrive(dbar(RED_FULL, bb));
-        if (!mbar_wait_warp(dbar(RED_FULL, bb), ph, abort_flag, P.err)) { ok = false; break; }
-        mt = fmaxf(mt, ld_shared_f32(red + ((kh ^ 1) * kHHalf + hl) * 4));
-        // move the running max only when the tile max exceeds it by > 8 (base 2)
-        const bool move = mt > m_run + 8.f;
-        const bool rescale_o = move && m_run != -INFINITY;
-        if (__any_sync(0xffffffffu, rescale_o)) {
-          // O must hold every previous tile before it is rescaled (PV of
-          // tile j - 3 was awaited one tile ago, so this parity is unambiguous)
-          if (j >= 1 && !mbar_wait_warp(dbar(PV_DONE, bb ^ 1), ((j - 1) >> 1) & 1, abort_flag, P.err)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after_sync();
-          rescale_o_cols(tl, kh * 128, kh * 128 + 128, rescale_o ? exp2f(m_run - mt) : 1.f);
-        }
-        if (move) {
-          if (m_run != -INFINITY) l_half *= exp2f(m_run - mt);
-          m_run = mt;
-        }
-        // P = 2^(s - m) in bf16, 128-byte-swizzled K-major; the buffer is free
-        // once the PV two tiles back is done
-        if (j >= 2 && !mbar_wait_warp(dbar(PV_DONE, bb), ((j - 2) >> 1) & 1, abort_flag, P.err)) {
-          ok = false;
-          break;
-        }
-        const uint32_t pb = p0 + bb * kPBytes;
-        const uint32_t prow = pb + (h >> 3) * 1024 + (h & 7) * 128;
-        float psum = 0.f;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float p[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            p[e] = (m_run == -INFINITY) ? 0.f : fast_exp2(sreg[c * 8 + e] - m_run);
-            psum += p[e];
-          }
-          st_shared_v4(prow + (((kh * 4 + c) ^ (h & 7)) << 4), pack_bf16(p[0], p[1]), pack_bf16(p[2], p[3]),
-                       pack_bf16(p[4], p[5]), pack_bf16(p[6], p[7]));
-        }
-        l_half += psum;
-        // statistics for the other CTA: running max, and each warp's partial sum
-        const uint32_t so = sto0 + bb * kStatBytes;
-        if (kh == 0) st_shared_f32(so + hl * 4, m_run);
-        st_shared_f32(so + ((1 + kh) * kHHalf + hl) * 4, l_half);
-        fence_proxy_async_smem();
-        tc_fence_before_sync();
-        mbar_arrive(dbar(P_OWN_WRITTEN, bb));
-        mbar_arrive(dbar(PV_READY, bb));
-        if (leader) {
-          bool go = mbar_wait(dbar(P_OWN_WRITTEN, bb), ph, abort_flag, P.err);
-          if (go && j >= 2) go = mbar_wait_cluster1(dbar(PEER_P_FREE, bb), ((j - 2) >> 1) & 1, abort_flag, P.err);
-          if (go) {
-            bulk_wait_read<0>();  // earlier copies have read P and the statistics
-            const uint32_t pbar = map_peer(dbar(P_REMOTE_FULL, bb), peer);
-            const uint32_t mine = pb + crank * kPHalfBytes;
-            bulk_to_peer(map_peer(mine, peer), mine, kPHalfBytes, pbar);
-            bulk_to_peer(map_peer(sti0 + bb * kStatBytes, peer), so, kStatBytes, pbar);
-            bulk_commit();
-          }
-        }
-        if (!have && j + 1 < T && s_ready(j + 1)) {
-          read_s(snext);
-          have = true;
-        }
-        if (have) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) sreg[i] = snext[i];
-        }
+      for (int i = 0; i < 32; ++i) {
+        const bool v = ((valid >> i) & 1u) != 0;
+        sreg[i] = v ? sreg[i] * P.scale_log2 : -INFINITY;
+        mt = fmaxf(mt, sreg[i]);
       }
-      if (leader) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-      // both warps' partial sums of the last tile
-      if (ok && T > 0) {
-        mbar_arrive(fin);
-        ok = mbar_wait_warp(fin, 0, abort_flag, P.err);
-      }
-      if (ok && T > 0) {
-        const uint32_t so = sto0 + ((T - 1) & 1) * kStatBytes;
-        m_fin = m_run;
-        l_fin = ld_shared_f32(so + (kHHalf + hl) * 4) + ld_shared_f32(so + (2 * kHHalf + hl) * 4);
-      }
-      c_lo = kh * 128;
-      c_hi = c_lo + 128;
-    } else if (sub == 0) {
-      // ------------ ship: partial logits of the other CTA's heads, per tile --
-      const bool leader = (hl == 0);
-      for (int j = 0; ok && j < T; ++j) {
-        const int bb = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (!mbar_wait_warp(s_full, j & 1, abort_flag, P.err)) { ok = false; break; }
+      // tile max over all 64 columns: swap with the head's other warp
+      const uint32_t red = sbase + kOffRed + bb * (2 * kH * 4);
+      st_shared_f32(red + (kh * kH + h) * 4, mt);
+      mbar_arrive(red_full(bb));
+      if (!mbar_wait_warp(red_full(bb), (j >> 1) & 1, abort_flag, P.err)) { ok = false; break; }
+      mt = fmaxf(mt, ld_shared_f32(red + ((kh ^ 1) * kH + h) * 4));
+      // move the running max only when the tile max exceeds it by > 8 (base 2)
+      const bool move = mt > m_run + 8.f;
+      const bool rescale_o = move && m_run != -INFINITY;
+      // O (and the P buffer) hold tile j - 1's PV once it is done (PV of
+      // tile j - 2 was awaited one tile ago, so the parity is unambiguous)
+      if (j >= 1 && !mbar_wait_warp(pv_done, (j - 1) & 1, abort_flag, P.err)) { ok = false; break; }
+      if (__any_sync(0xffffffffu, rescale_o)) {
         tc_fence_after_sync();
-        float s[kRows];
-        tmem_ld32(tl + kSCol, s);
-        tmem_ld32(tl + kSCol + 32, s + 32);
-        tc_fence_before_sync();
-        mbar_arrive(s_empty);
-        if (j >= 2 && !mbar_wait_warp(dbar(XOUT_FREE, bb), ((j - 2) >> 1) & 1, abort_flag, P.err)) {
-          ok = false;
-          break;
-        }
-        const uint32_t xo = xout0 + bb * kXBytes;
+        rescale_o_cols(tl, kh * 128, kh * 128 + 128, rescale_o ? exp2f(m_run - mt) : 1.f);
+      }
+      if (move) {
+        if (m_run != -INFINITY) l_half *= exp2f(m_run - mt);
+        m_run = mt;
+      }
+      // P = 2^(s - m) in bf16, 128-byte-swizzled K-major
+      const uint32_t prow = sbase + kOffP + (h >> 3) * 1024 + (h & 7) * 128;
+      float psum = 0.f;
 #pragma unroll
-        for (int c = 0; c < kRows / 4; ++c)
-          asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(xo + (c * kHHalf + hl) * 16), "f"(s[4 * c]),
-                       "f"(s[4 * c + 1]), "f"(s[4 * c + 2]), "f"(s[4 * c + 3])
-                       : "memory");
-        fence_proxy_async_smem();
-        mbar_arrive(dbar(XOUT_WRITTEN, bb));
-        if (leader) {
-          bool go = mbar_wait(dbar(XOUT_WRITTEN, bb), ph, abort_flag, P.err);
-          if (go && j >= 2) go = mbar_wait_cluster1(dbar(X_EMPTY, bb), ((j - 2) >> 1) & 1, abort_flag, P.err);
-          if (go) {
-            bulk_to_peer(map_peer(xin0 + bb * kXBytes, peer), xo, kXBytes, map_peer(dbar(X_FULL, bb), peer));
-            bulk_commit();
-            if (j >= 1) {
-              bulk_wait_read<1>();  // the copy of tile j - 1 has read its staging buffer
-              mbar_arrive(dbar(XOUT_FREE, bb ^ 1));
-            }
-          }
+      for (int c = 0; c < 4; ++c) {
+        float p[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          p[e] = (m_run == -INFINITY) ? 0.f : fast_exp2(sreg[c * 8 + e] - m_run);
+          psum += p[e];
         }
+        st_shared_v4(prow + (((kh * 4 + c) ^ (h & 7)) << 4), pack_bf16(p[0], p[1]), pack_bf16(p[2], p[3]),
+                     pack_bf16(p[4], p[5]), pack_bf16(p[6], p[7]));
       }
-      if (leader) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-      // the other CTA's statistics of these heads after the last tile, once
-      // the P-side warps (which waited on every tile's copy) have seen them
-      if (ok && T > 0) ok = mbar_wait_warp(pside_done, 0, abort_flag, P.err);
-      if (ok && T > 0) {
-        const uint32_t si = sti0 + ((T - 1) & 1) * kStatBytes;
-        m_fin = ld_shared_f32(si + hl * 4);
-        l_fin = ld_shared_f32(si + (kHHalf + hl) * 4) + ld_shared_f32(si + (2 * kHHalf + hl) * 4);
+      l_half += psum;
+      fence_proxy_async_smem();
+      tc_fence_before_sync();
+      mbar_arrive(pv_ready);
+      if (j + 1 < T && !shipped) {
+        if (!mbar_wait_warp(s_full, (j + 1) & 1, abort_flag, P.err)) { ok = false; break; }
+        if (!ship_next()) { ok = false; break; }
       }
-      c_lo = 128;
-      c_hi = 256;
-    } else {
-      // -------- P side: the other CTA's P rows and statistics, O rescaling --
-      const bool leader = (hl == 0);
-      float m_prev = -INFINITY;
-      for (int j = 0; ok && j < T; ++j) {
-        const int bb = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (leader && j >= 2 && mbar_wait(dbar(PV_DONE, bb), ((j - 2) >> 1) & 1, abort_flag, P.err)) {
-          // P buffer bb is free again: arm it for tile j, then let the other CTA fill it
-          mbar_arrive_expect_tx(dbar(P_REMOTE_FULL, bb), kPHalfBytes + kStatBytes);
-          mbar_arrive_remote(map_peer(dbar(PEER_P_FREE, bb), peer));
-        }
-        if (!mbar_wait_warp_cluster(dbar(P_REMOTE_FULL, bb), ph, abort_flag, P.err)) { ok = false; break; }
-        const float m_new = ld_shared_f32(sti0 + bb * kStatBytes + hl * 4);
-        const bool rescale_o = m_new != m_prev && m_prev != -INFINITY;
-        if (__any_sync(0xffffffffu, rescale_o)) {
-          // (P_REMOTE_FULL of tile j implies PV of tile j - 2 is done)
-          if (j >= 1 && !mbar_wait_warp(dbar(PV_DONE, bb ^ 1), ((j - 1) >> 1) & 1, abort_flag, P.err)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after_sync();
-          rescale_o_cols(tl, 0, kDvHalf, rescale_o ? exp2f(m_prev - m_new) : 1.f);
-        }
-        m_prev = m_new;
-        tc_fence_before_sync();
-        mbar_arrive(dbar(PV_READY, bb));
+#pragma unroll
+      for (int i = 0; i < 32; ++i) sreg[i] = snext[i];
+    }
+    // final sum of head h: both warps' partial sums
+    float m_fin = -INFINITY, l_fin = 0.f;
+    if (ok && T > 0) {
+      const uint32_t red_fin = sbase + kOffRed + (T & 1) * (2 * kH * 4);  // unused since tile T - 2
+      st_shared_f32(red_fin + (kh * kH + h) * 4, l_half);
+      mbar_arrive(fin);
+      ok = mbar_wait_warp(fin, 0, abort_flag, P.err);
+      if (ok) {
+        m_fin = m_run;
+        l_fin = l_half + ld_shared_f32(red_fin + ((kh ^ 1) * kH + h) * 4);
       }
-      if (ok && T > 0) mbar_arrive(pside_done);
-      if (ok && T > 0) {
-        const uint32_t si = sti0 + ((T - 1) & 1) * kStatBytes;
-        m_fin = m_prev;
-        l_fin = ld_shared_f32(si + (kHHalf + hl) * 4) + ld_shared_f32(si + (2 * kHHalf + hl) * 4);
-      }
-      c_lo = 0;
-      c_hi = 128;
     }
     // ------------------------------------------------------------ output --
-    // every role has seen PV of tile T - 3 complete (directly, or through the
-    // other CTA's P rows of tile T - 1), so this parity is unambiguous
-    if (ok && T >= 1) ok = mbar_wait_warp(dbar(PV_DONE, (T - 1) & 1), ((T - 1) >> 1) & 1, abort_flag, P.err);
+    // (PV of tile T - 2 was awaited at tile T - 1: this parity is unambiguous)
+    if (ok && T >= 1) ok = mbar_wait_warp(pv_done, (T - 1) & 1, abort_flag, P.err);
     if (ok) {
       tc_fence_after_sync();
       const int64_t rh = static_cast<int64_t>(r) * kH + h;
-      const bool stats_writer = own ? (sub == 0) : (sub == 1);  // one thread per head
+      const int c_lo = kh * 128, c_hi = c_lo + 128;
       if (P.splits == 1) {
         const float inv = l_fin > 0.f ? 1.f / l_fin : 0.f;
         __nv_bfloat16* dst = P.out + rh * kDv + crank * kDvHalf;
@@ -791,7 +730,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
             *reinterpret_cast<uint4*>(dst + c + q * 8) = v;
           }
         }
-        if (P.lse != nullptr && crank == 0 && stats_writer)
+        if (P.lse != nullptr && crank == 0 && kh == 0)
           P.lse[rh] = l_fin > 0.f ? (m_fin + log2f(l_fin)) * 0.6931471805599453f : -INFINITY;
       } else {
         const int64_t it = (static_cast<int64_t>(r) * P.splits + sp) * 2 + crank;
@@ -806,7 +745,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
           for (int q = 0; q < 8; ++q)
             *reinterpret_cast<float4*>(dst + c + q * 4) = make_float4(o[q * 4], o[q * 4 + 1], o[q * 4 + 2], o[q * 4 + 3]);
         }
-        if (own && stats_writer) {
+        if (crank == 0 && kh == 0) {
           const int64_t ms = static_cast<int64_t>(r) * P.splits + sp;
           P.part_ml[(ms * 2 + 0) * kH + h] = m_fin;
           P.part_ml[(ms * 2 + 1) * kH + h] = l_fin;
