@@ -6,10 +6,12 @@
 // split over a thread-block cluster of C CTAs (C = 1..16); each thread keeps
 // its PER consecutive keys in registers for the whole selection:
 //   * three histogram passes (digits of 11, 11 and 10 bits, most significant
-//     first) into shared memory; the C partial histograms are summed through
-//     distributed shared memory and every CTA finds the same digit of the
-//     k-th largest key, so after three passes all CTAs know the exact key T of
-//     the k-th largest score and how many keys equal to T to keep;
+//     first) into shared memory.  Each CTA also totals its histogram in 32
+//     groups of 64 bins; through distributed shared memory every CTA sums the
+//     C CTAs' group totals, finds the group holding the k-th largest key, then
+//     sums only that group's 64 bins over the C CTAs and finds the digit (all
+//     CTAs reach the same digit).  After three passes all CTAs know the exact
+//     key T of the k-th largest score and how many keys equal to T to keep;
 //   * one ordered compaction: per-thread counts of keys > T and == T, a block
 //     prefix sum (warp shuffles), CTA totals exchanged across the cluster,
 //     then every kept index is written at its final position -- keys > T plus
@@ -26,6 +28,8 @@ namespace dsa {
 namespace {
 
 constexpr int kBins = 2048;
+constexpr int kGroupBins = 64;                    // bins per group total
+constexpr int kGroups = kBins / kGroupBins;       // 32
 constexpr int kMaxWarps = 32;
 constexpr int kMaxCluster = 16;
 
@@ -67,7 +71,10 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads)
                         const int32_t* __restrict__ q_pos0, int t_off, int n_q, int s_max, int k,
                         int32_t* __restrict__ idx) {
   __shared__ uint32_t hist[3][kBins];
-  __shared__ uint32_t merged[kBins];
+  __shared__ uint32_t gtot[3][kGroups];   // this CTA's group totals, read by the peers
+  __shared__ uint32_t mgroup[kGroups];    // group totals over the cluster
+  __shared__ uint32_t mbin[kGroupBins];   // the target group's bins over the cluster
+  __shared__ uint32_t s_group, s_gabove;
   __shared__ uint32_t wsum[kMaxWarps + 1];
   __shared__ uint32_t s_digit, s_above;
   __shared__ uint32_t s_tot[2];
@@ -121,36 +128,63 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads)
 #pragma unroll
     for (int e = 0; e < PER; ++e)
       if (((vmask >> e) & 1u) && (key[e] & pmask) == prefix) atomicAdd(&hist[pass][(key[e] >> shift) & dmask], 1u);
-    cluster.sync();  // every CTA's histogram of this pass is complete
-    for (int i = tid; i < kBins; i += kThreads) {
-      uint32_t v = 0;
-      for (int q = 0; q < C; ++q) v += cluster.map_shared_rank(&hist[pass][0], q)[i];
-      merged[i] = v;
-    }
     __syncthreads();
     {
-      // bins from the top, kBins / kThreads per thread; a block prefix sum
-      // finds the bin holding the remaining-th largest key
+      // group totals: kBins / kThreads consecutive bins a thread, 64 a group
       constexpr int kPerT = kBins / kThreads;
-      const int btop = kBins - 1 - kPerT * tid;
-      uint32_t cnt[kPerT];
-      uint32_t mine = 0;
+      constexpr int kLanesPerGroup = kGroupBins / kPerT;
+      uint32_t v = 0;
 #pragma unroll
-      for (int q = 0; q < kPerT; ++q) {
-        cnt[q] = merged[btop - q];
-        mine += cnt[q];
+      for (int q = 0; q < kPerT; ++q) v += hist[pass][tid * kPerT + q];
+#pragma unroll
+      for (int off = 1; off < kLanesPerGroup; off <<= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+      if ((tid & (kLanesPerGroup - 1)) == 0) gtot[pass][tid / kLanesPerGroup] = v;
+    }
+    cluster.sync();  // every CTA's histogram and group totals of this pass are complete
+    static_assert(kThreads == kGroups * kMaxCluster, "one thread per (group, cluster rank)");
+    {
+      // sum the C CTAs' group totals: thread = (group, rank), reduced over 16 lanes
+      const int g = tid / kMaxCluster, q = tid % kMaxCluster;
+      uint32_t v = q < C ? cluster.map_shared_rank(&gtot[pass][0], q)[g] : 0u;
+#pragma unroll
+      for (int off = 1; off < kMaxCluster; off <<= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+      if (q == 0) mgroup[g] = v;
+    }
+    __syncthreads();
+    if (tid < 32) {
+      // the group holding the remaining-th largest key, scanning from the top
+      const uint32_t cnt = mgroup[kGroups - 1 - tid];
+      const uint32_t incl = warp_incl_scan(cnt);
+      if (incl - cnt < remaining && remaining <= incl) {
+        s_group = static_cast<uint32_t>(kGroups - 1 - tid);
+        s_gabove = incl - cnt;
       }
-      uint32_t tot;
-      const uint32_t excl = block_excl_scan<kThreads>(mine, wsum, &tot);
-      if (excl < remaining && remaining <= excl + mine) {
-        uint32_t cum = excl;
+    }
+    __syncthreads();
+    const uint32_t G = s_group;
 #pragma unroll
-        for (int q = 0; q < kPerT; ++q) {
-          if (cum < remaining && remaining <= cum + cnt[q]) {
-            s_digit = static_cast<uint32_t>(btop - q);
-            s_above = cum;
-          }
-          cum += cnt[q];
+    for (int hb = 0; hb < kGroupBins / (kThreads / kMaxCluster); ++hb) {
+      // that group's bins summed over the C CTAs: thread = (bin, rank)
+      const int bl = hb * (kThreads / kMaxCluster) + tid / kMaxCluster, q = tid % kMaxCluster;
+      uint32_t v = q < C ? cluster.map_shared_rank(&hist[pass][0], q)[G * kGroupBins + bl] : 0u;
+#pragma unroll
+      for (int off = 1; off < kMaxCluster; off <<= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+      if (q == 0) mbin[bl] = v;
+    }
+    __syncthreads();
+    if (tid < 32) {
+      // the bin within the group, two bins a lane from the top
+      const uint32_t rem = remaining - s_gabove;
+      const uint32_t hi = mbin[kGroupBins - 1 - 2 * tid], lo = mbin[kGroupBins - 2 - 2 * tid];
+      const uint32_t incl = warp_incl_scan(hi + lo);
+      const uint32_t excl = incl - hi - lo;
+      if (excl < rem && rem <= incl) {
+        if (rem <= excl + hi) {
+          s_digit = G * kGroupBins + kGroupBins - 1 - 2 * tid;
+          s_above = s_gabove + excl;
+        } else {
+          s_digit = G * kGroupBins + kGroupBins - 2 - 2 * tid;
+          s_above = s_gabove + excl + hi;
         }
       }
     }
