@@ -302,6 +302,7 @@ __device__ __forceinline__ void gather_rope(uint32_t dst0, const char* kv_b, int
 constexpr uint32_t kLayoutSW64 = 4;
 
 __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) {
+  pdl_wait();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
@@ -589,8 +590,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
       fence_proxy_async_smem();  // generic writes -> bulk-copy reads
       mbar_arrive(xout_written);
     };
-    // S(t) complete, tested without waiting; the whole warp agrees
-    auto s_ready = [&](int t) { return __all_sync(0xffffffffu, mbar_test_wait(s_full, t & 1)); };
     // validity of this lane's row in tiles [vbase, vbase + 32), loaded in
     // batches so that no global load is pending inside the loop
     uint32_t vbits = 0;
@@ -628,18 +627,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
         sreg[4 * c + 3] += v.w;
       }
       mbar_arrive(xin_read(bb));
-      // tile j + 1's partial goes out now if its logits are ready, so the
-      // copy runs under this tile's softmax
-      bool shipped = false;
-      auto ship_next = [&]() -> bool {
+      // tile j + 1's partial goes out before this tile's softmax, from every
+      // warp at the same point, so the copy runs under the softmax
+      if (j + 1 < T) {
+        if (!mbar_wait_warp(s_full, (j + 1) & 1, abort_flag, P.err)) { ok = false; break; }
         read_s(snext);
         // the copy of tile j has read xout
-        if (!mbar_wait_warp(xout_free, j & 1, abort_flag, P.err)) return false;
+        if (!mbar_wait_warp(xout_free, j & 1, abort_flag, P.err)) { ok = false; break; }
         write_x(snext);
-        shipped = true;
-        return true;
-      };
-      if (j + 1 < T && s_ready(j + 1) && !ship_next()) { ok = false; break; }
+      }
       float mt = -INFINITY;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
@@ -685,10 +681,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
       fence_proxy_async_smem();
       tc_fence_before_sync();
       mbar_arrive(pv_ready);
-      if (j + 1 < T && !shipped) {
-        if (!mbar_wait_warp(s_full, (j + 1) & 1, abort_flag, P.err)) { ok = false; break; }
-        if (!ship_next()) { ok = false; break; }
-      }
 #pragma unroll
       for (int i = 0; i < 32; ++i) sreg[i] = snext[i];
     }
@@ -705,6 +697,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
       }
     }
     // ------------------------------------------------------------ output --
+    pdl_trigger();
     // (PV of tile T - 2 was awaited at tile T - 1: this parity is unambiguous)
     if (ok && T >= 1) ok = mbar_wait_warp(pv_done, (T - 1) & 1, abort_flag, P.err);
     if (ok) {
@@ -777,6 +770,7 @@ constexpr int kCombineHeads = 8;  // heads per combine block
 __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restrict__ part_o,
                                                            const float* __restrict__ part_ml, int splits,
                                                            __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+  pdl_wait();
   __shared__ float coef[kMaxSplits][kCombineHeads];
   const int r = blockIdx.x;
   const int h0 = blockIdx.y * kCombineHeads;
@@ -915,18 +909,26 @@ dsa_status_t attn_tc(const AttnArgs& a) {
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = a.stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1] = pdl_attribute();
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   if (cudaLaunchKernelEx(&cfg, attn_mla_tc_kernel, P) != cudaSuccess) return DSA_ERR_CUDA;
   if (p.splits > 1) {
-    attn_combine_kernel<<<dim3(static_cast<unsigned>(R), kH / kCombineHeads), 256, 0, a.stream>>>(
-        P.part_o, P.part_ml, p.splits, P.out, a.lse);
-    if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+    cudaLaunchConfig_t cc = {};
+    cc.gridDim = dim3(static_cast<unsigned>(R), kH / kCombineHeads, 1);
+    cc.blockDim = dim3(256, 1, 1);
+    cc.stream = a.stream;
+    cudaLaunchAttribute cattr[1] = {pdl_attribute()};
+    cc.attrs = cattr;
+    cc.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cc, attn_combine_kernel, static_cast<const float*>(P.part_o),
+                           static_cast<const float*>(P.part_ml), p.splits, P.out, a.lse) != cudaSuccess)
+      return DSA_ERR_CUDA;
   }
   return DSA_OK;
 }

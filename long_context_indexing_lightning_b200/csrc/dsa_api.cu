@@ -241,6 +241,26 @@ dsa_status_t check_attn_inputs(const dsa_shape_t* s, const void* q, const void* 
 
 int device_sm_count(int dev) { return (dev >= 0 && dev < kMaxDevices) ? g_sm_count[dev] : 0; }
 
+// The host-buffer entry point copies the attention queries on a second stream
+// of the library's own, so that the copy overlaps the indexer and top-k.
+// Created once per device on first use, with two events to join the streams.
+cudaStream_t g_copy_stream[kMaxDevices] = {};
+cudaEvent_t g_ev_start[kMaxDevices] = {}, g_ev_q[kMaxDevices] = {};
+bool ensure_copy_stream(int dev) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_copy_stream[dev] != nullptr) return true;
+  cudaStream_t s = nullptr;
+  cudaEvent_t a = nullptr, b = nullptr;
+  if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) return false;
+  if (cudaEventCreateWithFlags(&a, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&b, cudaEventDisableTiming) != cudaSuccess)
+    return false;
+  g_ev_start[dev] = a;
+  g_ev_q[dev] = b;
+  g_copy_stream[dev] = s;
+  return true;
+}
+
 uint32_t* device_error_word(int dev) { return (dev >= 0 && dev < kMaxDevices) ? g_err_ptr[dev] : nullptr; }
 
 bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem_bytes, uint64_t inner,
@@ -354,7 +374,7 @@ static dsa_status_t forward_impl(const dsa_shape_t* s, int dev, cudaStream_t st,
                                  const float* q_scale, const void* k_idx, const float* k_scale, const float* w,
                                  const void* q, const void* kv, const void* v, const int32_t* ctx_len,
                                  const int32_t* q_pos0, void* out, float* lse, int32_t* idx_out, uint8_t* ws,
-                                 const FwdLayout& L) {
+                                 const FwdLayout& L, cudaEvent_t q_ready = nullptr) {
   const int B = s->batch, n_q = s->n_q;
   if (B == 0 || n_q == 0) return DSA_OK;
   dsa_status_t rc;
@@ -378,6 +398,7 @@ static dsa_status_t forward_impl(const dsa_shape_t* s, int dev, cudaStream_t st,
     if (rc != DSA_OK) return rc;
     rc = run_topk(&si, dev, st, B, n_q, 0, scores, L.ld, ctx_len, q_pos0, idx, ws + L.off_topk, L.topk_bytes);
     if (rc != DSA_OK) return rc;
+    if (q_ready != nullptr && cudaStreamWaitEvent(st, q_ready, 0) != cudaSuccess) return DSA_ERR_CUDA;
     return run_attn(&si, dev, st, B, n_q, q, kv, v, idx, ctx_len, out, lse, ws + L.off_attn, L.attn_bytes);
   }
   // Rounds of `chunk` queries, one sequence at a time (positions shift by t0).
@@ -403,6 +424,8 @@ static dsa_status_t forward_impl(const dsa_shape_t* s, int dev, cudaStream_t st,
       rc = run_topk(&si, dev, st, 1, c, t0, scores, L.ld, ctx_len + b, q_pos0 + b, idx_b, ws + L.off_topk,
                     L.topk_bytes);
       if (rc != DSA_OK) return rc;
+      if (q_ready != nullptr && b == 0 && t0 == 0 && cudaStreamWaitEvent(st, q_ready, 0) != cudaSuccess)
+        return DSA_ERR_CUDA;
       rc = run_attn(&si, dev, st, 1, c, q_b, kv_b, v_b, idx_b, ctx_len + b, out_b, lse_b, ws + L.off_attn,
                     L.attn_bytes);
       if (rc != DSA_OK) return rc;
@@ -468,9 +491,16 @@ dsa_status_t dsa_forward_host(const dsa_shape_t* shape, const void* h_q_idx, con
   const size_t n_q_b = static_cast<size_t>(B) * n_q * shape->heads * shape->d_qk * aa;
   const size_t n_out = static_cast<size_t>(B) * n_q * shape->heads * shape->d_v * aa;
   const size_t n_lse = static_cast<size_t>(B) * n_q * shape->heads * 4;
+  // the attention queries (the bulk of the input) travel on the copy stream,
+  // under the indexer and top-k; the stream waits for them before attention
+  if (!ensure_copy_stream(dev)) return DSA_ERR_CUDA;
+  const cudaStream_t xs = g_copy_stream[dev];
+  if (cudaEventRecord(g_ev_start[dev], cs) != cudaSuccess || cudaStreamWaitEvent(xs, g_ev_start[dev], 0) != cudaSuccess ||
+      cudaMemcpyAsync(ws + L.off_h_q, h_q, n_q_b, cudaMemcpyHostToDevice, xs) != cudaSuccess ||
+      cudaEventRecord(g_ev_q[dev], xs) != cudaSuccess)
+    return DSA_ERR_CUDA;
   if (cudaMemcpyAsync(ws + L.off_h_qidx, h_q_idx, n_qidx, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
       cudaMemcpyAsync(ws + L.off_h_w, h_w, n_w, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
-      cudaMemcpyAsync(ws + L.off_h_q, h_q, n_q_b, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
       cudaMemcpyAsync(ws + L.off_h_ctx, h_ctx_len, static_cast<size_t>(B) * 4, cudaMemcpyHostToDevice, cs) !=
           cudaSuccess ||
       cudaMemcpyAsync(ws + L.off_h_pos, h_q_pos0, static_cast<size_t>(B) * 4, cudaMemcpyHostToDevice, cs) !=
@@ -480,7 +510,10 @@ dsa_status_t dsa_forward_host(const dsa_shape_t* shape, const void* h_q_idx, con
   st = forward_impl(&s2, dev, cs, ws + L.off_h_qidx, nullptr, k_idx, k_scale, reinterpret_cast<float*>(ws + L.off_h_w),
                     ws + L.off_h_q, kv, v, reinterpret_cast<int32_t*>(ws + L.off_h_ctx),
                     reinterpret_cast<int32_t*>(ws + L.off_h_pos), ws + L.off_h_out,
-                    h_lse ? reinterpret_cast<float*>(ws + L.off_h_lse) : nullptr, nullptr, ws, L);
+                    h_lse ? reinterpret_cast<float*>(ws + L.off_h_lse) : nullptr, nullptr, ws, L, g_ev_q[dev]);
+  // (already waited before attention; again here so that no copy into the
+  // workspace is left in flight on any path)
+  if (cudaStreamWaitEvent(cs, g_ev_q[dev], 0) != cudaSuccess && st == DSA_OK) st = DSA_ERR_CUDA;
   if (st != DSA_OK) return st;
   if (cudaMemcpyAsync(h_out, ws + L.off_h_out, n_out, cudaMemcpyDeviceToHost, cs) != cudaSuccess) return DSA_ERR_CUDA;
   if (h_lse && cudaMemcpyAsync(h_lse, ws + L.off_h_lse, n_lse, cudaMemcpyDeviceToHost, cs) != cudaSuccess)

@@ -24,6 +24,16 @@ __device__ __forceinline__ void raise_error(uint32_t* err, uint32_t bit) {
   if (err != nullptr) atomicOr(err, bit);
 }
 
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream-serialization attribute may start while the previous kernel of the
+// stream is still finishing.  pdl_wait() (first statement of every such
+// kernel, before any global memory access) returns once that kernel has
+// completed and its writes are visible; pdl_trigger() lets the next kernel be
+// scheduled once every CTA of this grid has called it or exited.  Both are
+// no-ops when the kernel was launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

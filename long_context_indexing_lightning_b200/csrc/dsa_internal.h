@@ -55,6 +55,14 @@ struct TopkArgs {
   uint32_t* err;
 };
 
+// Launch attribute for programmatic dependent launch (see pdl_wait()).
+inline cudaLaunchAttribute pdl_attribute() {
+  cudaLaunchAttribute a;
+  a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a.val.programmaticStreamSerializationAllowed = 1;
+  return a;
+}
+
 struct AttnArgs {
   int device;
   cudaStream_t stream;

@@ -138,6 +138,7 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
                       const int32_t* __restrict__ q_pos0, float* __restrict__ scores, int64_t ld,
                       float idx_scale, Sched S, uint32_t* err) {
   using C = IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQBufs>;
+  pdl_wait();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
@@ -389,6 +390,7 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
     }
   }
 
+  pdl_trigger();
   tc_fence_before_sync();
   __syncthreads();
   if (warp == 1) {
@@ -442,9 +444,17 @@ dsa_status_t launch_indexer_tc(const IndexerArgs& a) {
       return DSA_ERR_CUDA;
     attr_done[dev] = true;
   }
-  kern<<<grid, C::kThreads, C::kSmemBytes, a.stream>>>(tmk, tmq, a.w, a.q_scale, a.k_scale, a.ctx_len, a.q_pos0,
-                                                         a.scores, a.ld, a.idx_scale, S, a.err);
-  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = a.stream;
+  cudaLaunchAttribute attr[1] = {pdl_attribute()};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tmk, tmq, a.w, a.q_scale, a.k_scale, a.ctx_len, a.q_pos0,
+                                           a.scores, a.ld, a.idx_scale, S, a.err);
+  return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 }  // namespace

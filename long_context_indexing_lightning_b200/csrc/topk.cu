@@ -70,6 +70,7 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads)
     topk_cluster_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ ctx_len,
                         const int32_t* __restrict__ q_pos0, int t_off, int n_q, int s_max, int k,
                         int32_t* __restrict__ idx) {
+  pdl_wait();
   __shared__ uint32_t hist[3][kBins];
   __shared__ uint32_t gtot[3][kGroups];   // this CTA's group totals, read by the peers
   __shared__ uint32_t mgroup[kGroups];    // group totals over the cluster
@@ -197,6 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads)
   const uint32_t T = prefix;
   const uint32_t take_eq = remaining;  // keys == T to keep, lowest index first
 
+  pdl_trigger();  // the selection is fixed; only the writes remain
   uint32_t gt = 0, eq = 0;
 #pragma unroll
   for (int e = 0; e < PER; ++e) {
@@ -245,13 +247,14 @@ dsa_status_t launch_topk(const TopkArgs& a, int C) {
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = a.stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = C;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1] = pdl_attribute();
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a.scores, a.ld, a.ctx_len, a.q_pos0, a.t_off, a.n_q, a.s_max,
                                            a.k, a.idx);
   return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
