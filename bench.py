@@ -154,8 +154,8 @@ def _attn_extra_launches(wl, dsa, shape):
 # keyed by workload and by the SHA-256 of the indexer source the counters were taken on;
 # a changed kernel reports null.  Filled in from profiles/indexer_tc_decode128k.md.
 TRAFFIC = {
-    # B=8 capture (268,691,456 read + 6,685,184 written) scaled by 4 to B=32: traffic grows with the key tiles
-    "decode128k": ("b767673a70a4e371", 4 * (268691456 + 6685184)),
+    # B=8 capture (268,705,280 read + 6,302,976 written) scaled by 4 to B=32: traffic grows with the key tiles
+    "decode128k": ("60292bbc0f4e9c9d", 4 * (268705280 + 6302976)),
 }
 
 
