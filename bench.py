@@ -410,6 +410,73 @@ def run_reference(args, wl):
     return line
 
 
+def run_append(args):
+    """Cache append of one prefill chunk (the update before the step scores):
+    `--append-tokens` new tokens of one sequence written into a 65536-row cache,
+    index keys copied (bf16) or rotated + quantised (e4m3), latent rows copied.
+    HBM-bound: per token the key (256 B) and latent row (1152 B) are read and
+    written (the e4m3 key as 128 B of codes + a 4-byte scale)."""
+    import long_context_indexing_lightning_b200 as dsa
+
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    n, s_max = args.append_tokens, 65536
+    g = torch.Generator(device=dev).manual_seed(0)
+    k_new = (torch.randn(1, n, 128, generator=g, device=dev) / 11.3).to(torch.bfloat16)
+    kv_new = torch.randn(1, n, 576, generator=g, device=dev).to(torch.bfloat16)
+    kv_cache = torch.zeros(1, s_max, 576, dtype=torch.bfloat16, device=dev)
+    caches = {"bf16": (torch.zeros(1, s_max, 128, dtype=torch.bfloat16, device=dev), None),
+              "e4m3": (torch.zeros(1, s_max, 128, dtype=torch.uint8, device=dev),
+                       torch.zeros(1, s_max, dtype=torch.float32, device=dev))}
+    pos = torch.zeros(1, dtype=torch.int32, device=dev)
+    res = {}
+    for name, (k_cache, k_scale) in caches.items():
+        shape = dsa.make_shape(1, 1, s_max, idx_dtype=dsa.DSA_E4M3 if name == "e4m3" else dsa.DSA_BF16)
+        call = lambda: dsa.cache_append(shape, k_new, kv_new, pos, k_cache, kv_cache, k_scale=k_scale,
+                                        stream=stream)
+        for _ in range(args.warmup):
+            call()
+        torch.cuda.synchronize(dev)
+        clocks = ClockSampler(local)
+        clocks.start()
+        time.sleep(0.3)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(args.steps):
+            call()
+        e.record()
+        torch.cuda.synchronize(dev)
+        clk = clocks.stop()
+        ms = max_over_ranks(s.elapsed_time(e) / args.steps, dev)
+        key_out = 128 + 4 if name == "e4m3" else 256
+        res[name] = (ms, n * (256 + 1152 + key_out + 1152), clk)
+    rc, word = dsa.get_error(clear=True)
+    if rc != 0:
+        raise RuntimeError(f"device error word {word:#x}")
+    if rank != 0:
+        return None
+    hbm, _, _, src = _peaks()
+    ms, nbytes, clk = res["bf16"]
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    ms8, nbytes8, _ = res["e4m3"]
+    return {
+        "metric": f"cache append tokens/s ({n}-token prefill chunk)",
+        "value": n * ws / (ms * 1e-3), "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded gaussian, bf16)",
+        "config": {"workload": f"append: B=1, {n} new tokens into a 65536-row cache, index key 128 + latent 576",
+                   "l2": "inputs + outputs larger than L2"},
+        "roofline": {"kernel": "cache_append", "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "peak_source": f"{src} hbm_gbs (of {src})", "traffic": None,
+                     "algorithmic_bytes": nbytes},
+        "e4m3": {"ms_per_step": ms8, "tokens_per_s": n / (ms8 * 1e-3),
+                 "achieved_gbs": nbytes8 / (ms8 * 1e-3) / 1e9, "frac": nbytes8 / (ms8 * 1e-3) / 1e9 / hbm},
+        "gpu_launches": args.steps, "clocks": clk,
+    }
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -420,10 +487,18 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling runs)")
     ap.add_argument("--q-chunk", type=int, default=4096, help="prefill: queries per indexer/top-k/attention round")
+    ap.add_argument("--op", default="step", choices=["step", "append"],
+                    help="step: the layer step (default); append: the cache append of one prefill chunk")
+    ap.add_argument("--append-tokens", type=int, default=65536)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     wl = workloads.get(args.workload, **({"batch": args.batch} if args.batch else {}))
+    if args.op == "append" and args.impl == "ours":
+        line = run_append(args)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
     if args.impl == "reference":
         line = run_reference(args, wl)
         if line is not None:

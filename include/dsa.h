@@ -173,6 +173,34 @@ dsa_status_t dsa_hadamard_quant_fp8(const void *x, int32_t x_dtype, int64_t rows
                                     uint8_t *x_fp8, float *scale, void *stream);
 
 /*
+ * Cache append, the update before the step scores (DeepSeek-V3.2 model doc,
+ * section "DeepSeek Sparse Attention (DSA)": the indexer keeps its own small
+ * per-token key cache -- single head, index_head_dim wide -- beside the main
+ * K/V cache, updated through update_indexer(); the reference indexer runs in
+ * FP8 after the Hadamard rotation).  New token i of sequence b goes to cache
+ * row pos[b] + i:
+ *   k_new   [B][n_new][idx_dim] in idx_dtype (F32/BF16), or BF16 when
+ *           idx_dtype is E4M3;
+ *   kv_new  [B][n_new][kv_heads][d_qk] attn_dtype; v_new [B][n_new][kv_heads][d_v]
+ *           for the separate-V form, else NULL;
+ *   pos     [B] int32, DEVICE: the first cache row of each sequence's new tokens;
+ *   k_cache the indexer key cache as read by dsa_indexer_scores: the row is
+ *           copied (F32/BF16), or (E4M3, idx_dim 128) rotated by the 128-point
+ *           Hadamard and quantised exactly as dsa_hadamard_quant_fp8 does, codes
+ *           into k_cache [B][s_max][128] and the row scale into k_scale [B][s_max];
+ *   kv_cache, v_cache as read by dsa_sparse_mla_attn (v_cache NULL iff v_new is).
+ * All pointers are DEVICE pointers, 4-byte aligned; the caller owns them and
+ * advances its own ctx_len.  Rows that fall outside [0, s_max) are skipped
+ * and set DSA_ERR_BAD_INDEX in the device error word.  Nothing is allocated;
+ * the work is enqueued on `stream`.
+ */
+dsa_status_t dsa_cache_append(const dsa_shape_t *shape, int32_t n_new,
+                              const void *k_new, const void *kv_new, const void *v_new,
+                              const int32_t *pos,
+                              void *k_cache, float *k_scale, void *kv_cache, void *v_cache,
+                              void *stream);
+
+/*
  * The whole layer step: indexer scores -> top-k -> sparse attention, in
  * rounds of shape->q_chunk queries per sequence (scores of one round live in
  * the workspace).  Inputs as in the calls above, except with

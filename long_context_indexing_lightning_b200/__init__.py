@@ -25,7 +25,8 @@ STATUS = {
 }
 
 EXPORTS = (
-    "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_hadamard_quant_fp8", "dsa_forward",
+    "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_hadamard_quant_fp8", "dsa_cache_append",
+    "dsa_forward",
     "dsa_forward_host", "dsa_workspace_bytes", "dsa_get_error", "dsa_status_string", "dsa_version",
     "dsa_sparse_mla_attn_static", "dsa_selftest_wait_timeout",
 )
@@ -71,6 +72,7 @@ def lib():
         L.dsa_topk.argtypes = [S, P, i64, P, P, P, P, sz, P]
         L.dsa_sparse_mla_attn.argtypes = [S, P, P, P, P, P, P, P, P, sz, P]
         L.dsa_hadamard_quant_fp8.argtypes = [P, i32, i64, i32, P, P, P]
+        L.dsa_cache_append.argtypes = [S, i32, P, P, P, P, P, P, P, P, P]
         L.dsa_sparse_mla_attn_static.argtypes = [S, P, P, P, P, P, P, P, P]
         L.dsa_selftest_wait_timeout.argtypes = [P]
         L.dsa_forward.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
@@ -195,6 +197,18 @@ def hadamard_quant_fp8(x, x8=None, scale=None, stream=None):
     _check(lib().dsa_hadamard_quant_fp8(_p(x), _dtype_code(x.dtype), rows, dim, _p(x8), _p(scale),
                                         _stream(stream)), "dsa_hadamard_quant_fp8")
     return x8, scale
+
+
+def cache_append(shape, k_new, kv_new, pos, k_cache, kv_cache, k_scale=None, v_new=None, v_cache=None,
+                 stream=None):
+    """Write new tokens into the caches at rows pos[b] + i (see dsa_cache_append).
+
+    k_new [B, n_new, idx_dim], kv_new [B, n_new, ...]; with idx_dtype E4M3 the
+    keys are rotated + quantised into k_cache (uint8) and k_scale."""
+    n_new = k_new.shape[1] if k_new.dim() > 1 else 0
+    _check(lib().dsa_cache_append(ctypes.byref(shape), n_new, _p(k_new), _p(kv_new), _p(v_new), _p(pos),
+                                  _p(k_cache), _p(k_scale), _p(kv_cache), _p(v_cache), _stream(stream)),
+           "dsa_cache_append")
 
 
 def forward(shape, q_idx, k_idx, w, q, kv, ctx_len, q_pos0, out=None, v=None, q_scale=None, k_scale=None,

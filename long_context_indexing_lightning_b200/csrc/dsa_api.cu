@@ -340,6 +340,46 @@ dsa_status_t dsa_sparse_mla_attn(const dsa_shape_t* shape, const void* q, const 
                   out, lse, workspace, workspace_bytes);
 }
 
+dsa_status_t dsa_cache_append(const dsa_shape_t* shape, int32_t n_new, const void* k_new, const void* kv_new,
+                              const void* v_new, const int32_t* pos, void* k_cache, float* k_scale, void* kv_cache,
+                              void* v_cache, void* stream) {
+  dsa_status_t st = check_shape(shape);
+  if (st != DSA_OK) return st;
+  if (n_new < 0) return DSA_ERR_INVALID_ARG;
+  if (!k_new || !kv_new || !pos || !k_cache || !kv_cache) return DSA_ERR_INVALID_ARG;
+  if ((v_new == nullptr) != (v_cache == nullptr)) return DSA_ERR_INVALID_ARG;
+  const bool fp8 = shape->idx_dtype == DSA_E4M3;
+  if (shape->attn_dtype != DSA_F32 && shape->attn_dtype != DSA_BF16) return DSA_ERR_INVALID_ARG;
+  if (fp8 && k_scale == nullptr) return DSA_ERR_INVALID_ARG;
+  if (fp8 && shape->idx_dim != 128) return DSA_ERR_UNSUPPORTED;
+  const size_t ea = elem_size(shape->attn_dtype);
+  AppendArgs a;
+  a.k_new = k_new;
+  a.kv_new = kv_new;
+  a.v_new = v_new;
+  a.pos = pos;
+  a.k_cache = k_cache;
+  a.k_scale = k_scale;
+  a.kv_cache = kv_cache;
+  a.v_cache = v_cache;
+  a.B = shape->batch;
+  a.n_new = n_new;
+  a.s_max = shape->s_max;
+  a.k_row_bytes = fp8 ? 128 : static_cast<int64_t>(shape->idx_dim) * elem_size(shape->idx_dtype);
+  a.kv_row_bytes = static_cast<int64_t>(shape->kv_heads) * shape->d_qk * ea;
+  a.v_row_bytes = v_new ? static_cast<int64_t>(shape->kv_heads) * shape->d_v * ea : 0;
+  // rows are copied in 4-byte words (16-byte chunks when aligned)
+  if ((a.k_row_bytes | a.kv_row_bytes | a.v_row_bytes) & 3) return DSA_ERR_UNSUPPORTED;
+  const uintptr_t ptrs = reinterpret_cast<uintptr_t>(k_new) | reinterpret_cast<uintptr_t>(kv_new) |
+                         reinterpret_cast<uintptr_t>(v_new) | reinterpret_cast<uintptr_t>(k_cache) |
+                         reinterpret_cast<uintptr_t>(kv_cache) | reinterpret_cast<uintptr_t>(v_cache) |
+                         reinterpret_cast<uintptr_t>(k_scale);
+  if (ptrs & 3u) return DSA_ERR_INVALID_ARG;
+  DSA_SETUP(dev);
+  a.err = g_err_ptr[dev];
+  return cache_append(a, fp8, DSA_BF16, static_cast<cudaStream_t>(stream));
+}
+
 dsa_status_t dsa_hadamard_quant_fp8(const void* x, int32_t x_dtype, int64_t rows, int32_t dim, uint8_t* x_fp8,
                                     float* scale, void* stream) {
   if (rows < 0 || dim <= 0) return DSA_ERR_INVALID_ARG;

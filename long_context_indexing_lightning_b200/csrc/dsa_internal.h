@@ -55,6 +55,22 @@ struct TopkArgs {
   uint32_t* err;
 };
 
+// Cache append (csrc/cache_append.cu): token (b, i) -> cache row pos[b] + i.
+struct AppendArgs {
+  const void* k_new;   // [B][n_new][idx_dim]
+  const void* kv_new;  // [B][n_new] rows of kv_row_bytes
+  const void* v_new;   // [B][n_new] rows of v_row_bytes, or null
+  const int32_t* pos;  // [B]
+  void* k_cache;       // [B][s_max] rows of k_row_bytes (E4M3: 128 codes)
+  float* k_scale;      // [B][s_max] (E4M3 only)
+  void* kv_cache;
+  void* v_cache;
+  int B, n_new, s_max;
+  int64_t k_row_bytes, kv_row_bytes, v_row_bytes;
+  uint32_t* err;
+};
+dsa_status_t cache_append(const AppendArgs& a, bool fp8, int k_new_dtype, cudaStream_t stream);
+
 // Launch attribute for programmatic dependent launch (see pdl_wait()).
 inline cudaLaunchAttribute pdl_attribute() {
   cudaLaunchAttribute a;

@@ -1,20 +1,9 @@
-// Hadamard rotation + FP8 (E4M3) quantisation of 128-element rows.
-//
-// DeepSeek-V3.2 model doc (Transformers), section "DeepSeek Sparse Attention
-// (DSA)", item 1: the reference indexer runs in FP8 after the orthogonal
-// Hadamard transform `rotate_activation` (Hq.Hk = q.k).  Here: y = H x with
-// the orthonormal 128-point Sylvester-Hadamard matrix, one scale per row
-// sigma = max|y| / 448, codes e4m3(y / sigma) rounded to nearest even with
-// saturation.
-//
-// One warp per row; lane l holds elements 4l..4l+3.  The fast transform is
-// the butterfly network: strides 1 and 2 inside a lane, 4..64 across lanes
-// with shuffles.  HBM-bound: reads 2 (or 4) bytes and writes 1 byte per
-// element plus 4 bytes of scale per row.
-#include <cuda_fp8.h>
-
+// Hadamard rotation + FP8 (E4M3) quantisation of 128-element rows (the
+// arithmetic is in fp8_rows.cuh).  One warp per row, HBM-bound: reads 2 (or
+// 4) bytes and writes 1 byte per element plus 4 bytes of scale per row.
 #include "dsa_common.cuh"
 #include "dsa_internal.h"
+#include "fp8_rows.cuh"
 
 namespace dsa {
 namespace {
@@ -31,39 +20,8 @@ __global__ void __launch_bounds__(256) hadamard_quant_kernel(const T* __restrict
   const T* xr = x + r * kDim + 4 * lane;
 #pragma unroll
   for (int c = 0; c < 4; ++c) v[c] = to_f32(xr[c]);
-  // stride 1 and 2 (inside the lane)
-  {
-    const float a0 = v[0] + v[1], a1 = v[0] - v[1], a2 = v[2] + v[3], a3 = v[2] - v[3];
-    v[0] = a0 + a2;
-    v[1] = a1 + a3;
-    v[2] = a0 - a2;
-    v[3] = a1 - a3;
-  }
-  // strides 4 .. 64 (lane masks 1 .. 16)
-#pragma unroll
-  for (int m = 1; m < 32; m <<= 1) {
-    const bool upper = (lane & m) != 0;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const float o = __shfl_xor_sync(0xffffffffu, v[c], m);
-      v[c] = upper ? (o - v[c]) : (v[c] + o);
-    }
-  }
-  const float inv_sqrt = 0.08838834764831845f;  // 1/sqrt(128)
-  float amax = 0.f;
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    v[c] *= inv_sqrt;
-    amax = fmaxf(amax, fabsf(v[c]));
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-  const float sigma = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
-  const __nv_fp8x2_storage_t lo =
-      __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(v[0], sigma), __fdiv_rn(v[1], sigma)), __NV_SATFINITE, __NV_E4M3);
-  const __nv_fp8x2_storage_t hi =
-      __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(v[2], sigma), __fdiv_rn(v[3], sigma)), __NV_SATFINITE, __NV_E4M3);
-  const uint32_t packed = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+  float sigma;
+  const uint32_t packed = rotate_quant_e4m3(v, &sigma);
   *reinterpret_cast<uint32_t*>(x8 + r * kDim + 4 * lane) = packed;
   if (lane == 0) scale[r] = sigma;
 }

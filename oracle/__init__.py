@@ -143,6 +143,43 @@ def hadamard_quant(x):
     return code, sigma, quot
 
 
+def cache_append(k_cache, kv_cache, k_new, kv_new, pos, k_scale=None, v_cache=None, v_new=None):
+    """Cache append (section DSA: the indexer keeps its own per-token key
+    cache, single head, beside the K/V cache, updated through
+    update_indexer(); the reference indexer runs in FP8 after the Hadamard
+    rotation, item 1).
+
+    New token i of sequence b lands in cache row pos[b] + i; rows outside
+    [0, s_max) are skipped.  k_cache in a stored type (fp32, bf16 bits) gets
+    the key copied; a uint8 (e4m3) k_cache gets the rotated, quantised codes
+    and k_scale the row scale, as hadamard_quant computes them.  kv / v rows
+    are copied.  Returns updated copies (k_cache, k_scale, kv_cache, v_cache).
+    """
+    k_cache = np.array(k_cache, copy=True)
+    kv_cache = np.array(kv_cache, copy=True)
+    k_scale = None if k_scale is None else np.array(k_scale, copy=True)
+    v_cache = None if v_cache is None else np.array(v_cache, copy=True)
+    fp8 = k_cache.dtype == np.uint8
+    if fp8:
+        codes, sigma, _ = hadamard_quant(k_new)
+    B, n = k_new.shape[0], k_new.shape[1]
+    s_max = k_cache.shape[1]
+    for b in range(B):
+        for i in range(n):
+            r = int(pos[b]) + i
+            if r < 0 or r >= s_max:
+                continue
+            if fp8:
+                k_cache[b, r] = codes[b, i]
+                k_scale[b, r] = sigma[b, i]
+            else:
+                k_cache[b, r] = k_new[b, i]
+            kv_cache[b, r] = kv_new[b, i]
+            if v_cache is not None:
+                v_cache[b, r] = v_new[b, i]
+    return k_cache, k_scale, kv_cache, v_cache
+
+
 def e4m3_encode(x):
     x = np.ascontiguousarray(x, dtype=np.float64)
     out = np.empty(x.shape, dtype=np.uint8)

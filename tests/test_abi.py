@@ -65,6 +65,15 @@ def test_argument_errors_need_no_gpu(L):
     odd = s.replace(idx_dim=96)
     assert L.dsa_indexer_scores(ctypes.byref(odd), 16, None, 16, None, 16, 16, 16, 16, 1024, None) == 2
     assert L.dsa_hadamard_quant_fp8(16, dsa.DSA_BF16, 4, 64, 16, 16, None) == 2
+    # cache append: null buffers, one-sided v, missing FP8 scales, odd rows
+    assert L.dsa_cache_append(ctypes.byref(s), 1, None, 16, None, 16, 16, None, 16, None, None) == 1
+    assert L.dsa_cache_append(ctypes.byref(s), -1, 16, 16, None, 16, 16, None, 16, None, None) == 1
+    assert L.dsa_cache_append(ctypes.byref(s), 1, 16, 16, 16, 16, 16, None, 16, None, None) == 1
+    e4 = s.replace(idx_dtype=dsa.DSA_E4M3)
+    assert L.dsa_cache_append(ctypes.byref(e4), 1, 16, 16, None, 16, 16, None, 16, None, None) == 1
+    assert L.dsa_cache_append(ctypes.byref(e4.replace(idx_dim=64)), 1, 16, 16, None, 16, 16, 16, 16, None, None) == 2
+    assert L.dsa_cache_append(ctypes.byref(s.replace(d_qk=575)), 1, 16, 16, None, 16, 16, None, 16, None, None) == 2
+    assert L.dsa_cache_append(ctypes.byref(s), 1, 18, 16, None, 16, 16, None, 16, None, None) == 1
 
 
 def test_workspace_arithmetic(L):

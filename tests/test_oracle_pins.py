@@ -430,3 +430,83 @@ def test_tiny_workload_end_to_end_on_oracle():
     out = oracle.sparse_attn(n["q"], n["kv"], idx, wl.sm_scale, v=n["v"])
     de = oracle.dense_masked_attn(n["q"], n["kv"], idx, n["q_pos0"], wl.sm_scale, v=n["v"])
     np.testing.assert_allclose(out, de, rtol=1e-12, atol=1e-13)
+
+
+# ------------------------------------------------------------- cache append --
+
+def _append_case(seed, B=3, s_max=16, n=5, D=128, Dkv=40):
+    g = np.random.default_rng(seed)
+    k_cache = g.integers(0, 2**16, size=(B, s_max, D)).astype(np.uint16)
+    kv_cache = g.integers(0, 2**16, size=(B, s_max, Dkv)).astype(np.uint16)
+    k_new = _bf16_bits(torch.from_numpy(g.standard_normal((B, n, D)).astype(np.float32) / 8))
+    kv_new = g.integers(0, 2**16, size=(B, n, Dkv)).astype(np.uint16)
+    return k_cache, kv_cache, k_new, kv_new
+
+
+def test_cache_append_places_rows_and_leaves_the_rest():
+    """Token i of sequence b lands in row pos[b] + i; every other row, and
+    tokens whose row falls outside [0, s_max), change nothing."""
+    k_cache, kv_cache, k_new, kv_new = _append_case(1)
+    pos = np.array([3, 0, 13], np.int32)  # sequence 2: rows 13..17, only 13..15 exist
+    kc, _, kvc, _ = oracle.cache_append(k_cache, kv_cache, k_new, kv_new, pos)
+    for b in range(3):
+        for r in range(16):
+            i = r - pos[b]
+            if 0 <= i < 5:
+                np.testing.assert_array_equal(kc[b, r], k_new[b, i])
+                np.testing.assert_array_equal(kvc[b, r], kv_new[b, i])
+            else:
+                np.testing.assert_array_equal(kc[b, r], k_cache[b, r])
+                np.testing.assert_array_equal(kvc[b, r], kv_cache[b, r])
+    neg = np.array([-2, 0, 0], np.int32)  # rows -2, -1 skipped, 0..2 written
+    kc, _, _, _ = oracle.cache_append(k_cache, kv_cache, k_new, kv_new, neg)
+    np.testing.assert_array_equal(kc[0, :3], k_new[0, 2:])
+    np.testing.assert_array_equal(kc[0, 3:], k_cache[0, 3:])
+
+
+def test_cache_append_fp8_round_trip_within_e4m3_bound():
+    """E4M3 cache: decoding the codes, scaling and rotating back (H is its own
+    inverse) recovers each key within the quantisation bound: every rotated
+    element within 2^-4 relative or 2^-10 sigma absolute."""
+    k_cache, kv_cache, k_new, kv_new = _append_case(2)
+    codes0 = np.zeros(k_cache.shape, np.uint8)
+    sc0 = np.zeros(k_cache.shape[:2], np.float32)
+    pos = np.array([0, 4, 9], np.int32)
+    kc, ks, _, _ = oracle.cache_append(codes0, kv_cache, k_new, kv_new, pos, k_scale=sc0)
+    kf = torch.from_numpy(k_new.view(np.int16)).view(torch.bfloat16).float().numpy().astype(np.float64)
+    for b in range(3):
+        for i in range(5):
+            r = pos[b] + i
+            y = oracle.hadamard(kf[b, i])
+            yq = oracle.e4m3_decode(kc[b, r]) * np.float64(ks[b, r])
+            assert np.all(np.abs(yq - y) <= 2.0**-4 * np.abs(y) + 2.0**-10 * ks[b, r] + 1e-12)
+            back = oracle.hadamard(yq)
+            assert np.linalg.norm(back - kf[b, i]) <= 2.0**-4 * np.linalg.norm(kf[b, i]) + 1e-6
+            assert ks[b, r] == np.float32(np.abs(y).max() / 448.0)
+
+
+def test_cache_append_then_score_equals_scoring_the_full_keys():
+    """Appending a sequence's keys one step at a time and scoring gives the
+    scores of the whole key array (bf16 path, bit for bit), and the FP8 cache
+    equals quantising the whole key array at once."""
+    g = np.random.default_rng(3)
+    B, S, H, D = 2, 24, 4, 128
+    k_full = _bf16_bits(torch.from_numpy(g.standard_normal((B, S, D)).astype(np.float32) / 11))
+    q = _bf16_bits(torch.from_numpy(g.standard_normal((B, 1, H, D)).astype(np.float32) / 11))
+    w = g.standard_normal((B, 1, H)).astype(np.float32)
+    k_cache = np.zeros((B, S, D), np.uint16)
+    kv_cache = np.zeros((B, S, 8), np.uint16)
+    c8 = np.zeros((B, S, D), np.uint8)
+    s8 = np.zeros((B, S), np.float32)
+    for t0, n in ((0, 10), (10, 1), (11, 13)):  # a prefill chunk, a decode step, the rest
+        kn = np.ascontiguousarray(k_full[:, t0:t0 + n])
+        kvn = np.zeros((B, n, 8), np.uint16)
+        pos = np.full(B, t0, np.int32)
+        k_cache, _, kv_cache, _ = oracle.cache_append(k_cache, kv_cache, kn, kvn, pos)
+        c8, s8, _, _ = oracle.cache_append(c8, kv_cache, kn, kvn, pos, k_scale=s8)
+    ctx, pos0 = [S, S], [S - 1, S - 1]
+    np.testing.assert_array_equal(oracle.indexer_scores(q, k_cache, w, ctx, pos0),
+                                  oracle.indexer_scores(q, k_full, w, ctx, pos0))
+    cf, sf, _ = oracle.hadamard_quant(k_full)
+    np.testing.assert_array_equal(c8, cf)
+    np.testing.assert_array_equal(s8, sf)
