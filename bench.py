@@ -477,6 +477,66 @@ def run_append(args):
     }
 
 
+def run_topk_structures(args):
+    """Top-k alone at the 128K decode shape (32 rows x 131072 fp32 scores,
+    k = 2048) on rows of four structures: gaussian, a planted recent window
+    (the last 2048 keys above the rest), one exponent bucket (all in [1, 2))
+    and all-equal scores.  Reports each case's launch time and the
+    score-read rate against HBM."""
+    import long_context_indexing_lightning_b200 as dsa
+
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    B, S, k = 32, 131072, 2048
+    g = torch.Generator(device=dev).manual_seed(0)
+    cases = {
+        "gaussian": torch.randn(B, 1, S, generator=g, device=dev),
+        "recent_window": torch.randn(B, 1, S, generator=g, device=dev),
+        "one_exponent_bucket": 1.0 + torch.rand(B, 1, S, generator=g, device=dev),
+        "all_equal": torch.full((B, 1, S), 0.75, device=dev),
+    }
+    cases["recent_window"][:, :, S - 2048:] = 4.0 + torch.rand(B, 1, 2048, generator=g, device=dev)
+    ctx = torch.full((B,), S, dtype=torch.int32, device=dev)
+    pos0 = ctx - 1
+    idx = torch.empty(B, 1, k, dtype=torch.int32, device=dev)
+    shape = dsa.make_shape(B, 1, S, topk=k)
+    ws_t = torch.empty(max(1, dsa.workspace_bytes(shape, dsa.WS_TOPK)), dtype=torch.uint8, device=dev)
+    hbm, _, _, src = _peaks()
+    out = {}
+    for name, sc in cases.items():
+        call = lambda: dsa.topk(shape, sc, ctx, pos0, idx=idx, workspace=ws_t)
+        for _ in range(args.warmup):
+            call()
+        torch.cuda.synchronize(dev)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(args.steps):
+            call()
+        e.record()
+        torch.cuda.synchronize(dev)
+        ms = max_over_ranks(s.elapsed_time(e) / args.steps, dev)
+        nbytes = B * S * 4 + B * k * 4
+        out[name] = {"us": ms * 1e3, "rows_per_s": B / (ms * 1e-3),
+                     "frac_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm}
+    rc, word = dsa.get_error(clear=True)
+    if rc != 0:
+        raise RuntimeError(f"device error word {word:#x}")
+    if rank != 0:
+        return None
+    gms = out["gaussian"]["us"] * 1e-3
+    return {"metric": "top-k rows/s at 128K (gaussian rows)", "value": B * ws / (gms * 1e-3), "unit": "rows/s",
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": gms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32",
+            "data": "synthetic (seeded)", "config": {"workload": "top-k: B=32 rows x 131072 scores, k=2048",
+                                                      "l2": "scores resident in L2 (16.8 MB) between launches"},
+            "roofline": {"kernel": "topk_cluster", "bound": "hbm", "peak": hbm, "unit": "GB/s",
+                         "achieved": (B * S * 4 + B * k * 4) / (gms * 1e-3) / 1e9,
+                         "frac": out["gaussian"]["frac_hbm"], "peak_source": f"{src} hbm_gbs (of {src})",
+                         "traffic": None},
+            "cases": out, "gpu_launches": args.steps * len(cases)}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -487,15 +547,16 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling runs)")
     ap.add_argument("--q-chunk", type=int, default=4096, help="prefill: queries per indexer/top-k/attention round")
-    ap.add_argument("--op", default="step", choices=["step", "append"],
-                    help="step: the layer step (default); append: the cache append of one prefill chunk")
+    ap.add_argument("--op", default="step", choices=["step", "append", "topk"],
+                    help="step: the layer step (default); append: the cache append of one prefill chunk; "
+                         "topk: top-k alone on structured 128K rows")
     ap.add_argument("--append-tokens", type=int, default=65536)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     wl = workloads.get(args.workload, **({"batch": args.batch} if args.batch else {}))
-    if args.op == "append" and args.impl == "ours":
-        line = run_append(args)
+    if args.op in ("append", "topk") and args.impl == "ours":
+        line = run_append(args) if args.op == "append" else run_topk_structures(args)
         if line is not None:
             print(json.dumps(line), flush=True)
         return

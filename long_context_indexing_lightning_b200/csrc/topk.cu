@@ -219,6 +219,10 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads)
     gt_off += pt[0];
     eq_off += pt[1];
   }
+  // every remote read of this CTA is done: arrive now, wait only before
+  // leaving (peers may still be reading this CTA's totals), so the index
+  // writes below overlap the barrier
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
   uint32_t eq_rank = eq_off + (pre & 0xFFFFu);
   uint32_t pos = gt_off + (pre >> 16) + min(eq_rank, take_eq);
 #pragma unroll
@@ -231,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads)
       ++eq_rank;
     }
   }
-  cluster.sync();  // peers may still be reading this CTA's shared memory
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");  // peers are done with this CTA
 }
 
 template <int PER, int kThreads>

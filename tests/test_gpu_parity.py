@@ -187,6 +187,26 @@ def test_topk_ties_and_zeros_full_length(seed):
     _topk_case(B, 1, S, k, ctx, pos0, sc)
 
 
+def _structured_rows(g, B, S):
+    """Rows radix select finds hardest (the pages print no score
+    distribution): a planted recent window (the last 2048 keys score above
+    the rest), every score inside one exponent bucket [1, 2), and equal
+    scores; the remaining rows gaussian."""
+    sc = g.standard_normal((B, 1, S)).astype(np.float32)
+    sc[0, 0, S - 2048:] = 4.0 + g.random(2048).astype(np.float32)
+    sc[1, 0] = (1.0 + g.random(S)).astype(np.float32)
+    sc[2, 0] = np.float32(0.75)
+    return sc
+
+
+def test_topk_structured_rows_decode128k():
+    """Exact against the oracle at the 128K shape on the structured rows."""
+    g = np.random.default_rng(11)
+    B, S, k = 4, 131072, 2048
+    sc = _structured_rows(g, B, S)
+    _topk_case(B, 1, S, k, [S] * B, [S - 1] * B, sc)
+
+
 def test_topk_prefill_rows_all_positions():
     """Every query position of a short prefill, including rows with fewer
     than k candidates and rows around the 2048 boundary."""
