@@ -24,12 +24,26 @@ namespace {
 constexpr int kThreadsPerBlock = 256;
 
 // Warp copy of `bytes` (a multiple of 4): 16-byte chunks when both ends and
-// the size allow, else 4-byte words.
+// the size allow, else 4-byte words.  Each lane issues all of its loads of a
+// 2 KB span (16-byte case) before its stores, so a warp keeps several
+// requests in flight instead of one.
 __device__ __forceinline__ void warp_copy(char* dst, const char* src, int64_t bytes, int lane) {
   if (((reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(src) | static_cast<uintptr_t>(bytes)) & 15u) ==
       0) {
-    for (int64_t o = lane * 16; o < bytes; o += 32 * 16)
-      *reinterpret_cast<uint4*>(dst + o) = __ldg(reinterpret_cast<const uint4*>(src + o));
+    constexpr int kU = 4;  // chunks per lane per span: 4 x 32 x 16 B = 2 KB
+    for (int64_t base = 0; base < bytes; base += kU * 32 * 16) {
+      uint4 v[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int64_t o = base + (u * 32 + lane) * 16;
+        if (o < bytes) v[u] = __ldg(reinterpret_cast<const uint4*>(src + o));
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int64_t o = base + (u * 32 + lane) * 16;
+        if (o < bytes) *reinterpret_cast<uint4*>(dst + o) = v[u];
+      }
+    }
   } else {
     for (int64_t o = lane * 4; o < bytes; o += 32 * 4)
       *reinterpret_cast<uint32_t*>(dst + o) = __ldg(reinterpret_cast<const uint32_t*>(src + o));
@@ -49,24 +63,38 @@ __global__ void __launch_bounds__(kThreadsPerBlock) cache_append_kernel(AppendAr
     return;
   }
   const int64_t dst = static_cast<int64_t>(b) * P.s_max + row;
+  // this lane's part of the index key, loaded ahead of the row copies so
+  // that all of the warp's loads are in flight together
+  char* kdst = static_cast<char*>(P.k_cache) + dst * P.k_row_bytes;
+  const char* ksrc = static_cast<const char*>(P.k_new) + tok * (kFP8 ? 128 * sizeof(TK) : P.k_row_bytes);
+  const bool key16 = !kFP8 && P.k_row_bytes <= 32 * 16 &&
+                     ((reinterpret_cast<uintptr_t>(kdst) | reinterpret_cast<uintptr_t>(ksrc) |
+                       static_cast<uintptr_t>(P.k_row_bytes)) & 15u) == 0;
+  float kv4[4];
+  uint4 kchunk = make_uint4(0u, 0u, 0u, 0u);
   if (kFP8) {
-    const TK* kr = static_cast<const TK*>(P.k_new) + tok * 128 + 4 * lane;
-    float v[4];
+    const TK* kr = reinterpret_cast<const TK*>(ksrc) + 4 * lane;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) v[c] = to_f32(kr[c]);
-    float sigma;
-    const uint32_t packed = rotate_quant_e4m3(v, &sigma);
-    reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(P.k_cache) + dst * 128)[lane] = packed;
-    if (lane == 0) P.k_scale[dst] = sigma;
-  } else {
-    warp_copy(static_cast<char*>(P.k_cache) + dst * P.k_row_bytes,
-              static_cast<const char*>(P.k_new) + tok * P.k_row_bytes, P.k_row_bytes, lane);
+    for (int c = 0; c < 4; ++c) kv4[c] = to_f32(kr[c]);
+  } else if (key16 && lane * 16 < P.k_row_bytes) {
+    kchunk = __ldg(reinterpret_cast<const uint4*>(ksrc + lane * 16));
   }
+  // the attention rows (the larger part)
   warp_copy(static_cast<char*>(P.kv_cache) + dst * P.kv_row_bytes,
             static_cast<const char*>(P.kv_new) + tok * P.kv_row_bytes, P.kv_row_bytes, lane);
   if (P.v_new != nullptr)
     warp_copy(static_cast<char*>(P.v_cache) + dst * P.v_row_bytes,
               static_cast<const char*>(P.v_new) + tok * P.v_row_bytes, P.v_row_bytes, lane);
+  if (kFP8) {
+    float sigma;
+    const uint32_t packed = rotate_quant_e4m3(kv4, &sigma);
+    reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(P.k_cache) + dst * 128)[lane] = packed;
+    if (lane == 0) P.k_scale[dst] = sigma;
+  } else if (key16) {
+    if (lane * 16 < P.k_row_bytes) *reinterpret_cast<uint4*>(kdst + lane * 16) = kchunk;
+  } else {
+    warp_copy(kdst, ksrc, P.k_row_bytes, lane);
+  }
 }
 
 }  // namespace
