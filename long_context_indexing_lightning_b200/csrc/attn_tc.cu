@@ -60,17 +60,18 @@ constexpr int kSoftThreads = 32 * kSoftWarps;
 constexpr int kPrefetchWarp = kGatherWarps + 1 + kSoftWarps;  // 13
 constexpr int kCommWarp = kPrefetchWarp + 1;                   // 14
 constexpr int kThreads = 32 * (kCommWarp + 1);                 // 480
-// tensor memory: O half [0, 256), Q columns [256, 256 + 144), S [400, 464)
+// tensor memory: O half [0, 256), Q columns [256, 400), S [400, 464), P [464, 496)
+// (P as bf16 pairs: the A operand of the value MMA)
 constexpr int kTmemCols = 512;
 constexpr int kQCol = 256;
 constexpr int kSCol = kQCol + kQk / 2;
+constexpr int kPCol = kSCol + kRows;
+static_assert(kPCol + kRows / 2 <= kTmemCols, "tensor memory");
 
 // shared memory map (from a 1024-aligned base)
-constexpr int kPBytes = kH * kRows * 2;  // P: 128 heads x 64 rows bf16, SW128 K-major
 constexpr int kXBytes = kH * kRows * 4;  // partial logits: [16 x 4 rows][128 heads] fp32
 constexpr int kOffKV = 0;
-constexpr int kOffP = kOffKV + kStages * kStageBytes;
-constexpr int kOffXin = kOffP + kPBytes;         // the other CTA's partials, [tile parity]
+constexpr int kOffXin = kOffKV + kStages * kStageBytes;  // the other CTA's partials, [tile parity]
 constexpr int kOffXout = kOffXin + 2 * kXBytes;  // this CTA's partial, for the bulk copy
 constexpr int kOffRed = kOffXout + kXBytes;  // tile max of each softmax warp: [2][2 warps][128]
 // barriers: kv_full[3], kv_empty[3], then the 17 named in the kernel
@@ -79,7 +80,7 @@ constexpr int kOffBar = kOffRed + 2 * 2 * kH * 4;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory");
-static_assert(kOffP % 1024 == 0 && kPBytes % 1024 == 0, "P tile must stay 1024-aligned");
+static_assert(kStageBytes % 1024 == 0, "ring stages must stay 1024-aligned");
 
 struct AttnParams {
   const uint16_t* q;        // [R][128][576] bf16
@@ -121,9 +122,6 @@ __device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
 }
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 __device__ __forceinline__ float4 ld_shared_v4f(uint32_t addr) {
   float4 v;
@@ -479,9 +477,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
       constexpr uint32_t idesc_o = idesc_bf16_f32_bmn(kH, kDvHalf);
       const uint64_t kv_desc0 = sdesc(sbase + kOffKV, 16, 1024, kLayoutSW128);      // K-major rows (logits)
       const uint64_t v_desc0 = sdesc(sbase + kOffKV, kAtomBytes, 1024, kLayoutSW128);  // MN-major columns (value)
-      const uint64_t p_desc = sdesc(sbase + kOffP, 16, 1024, kLayoutSW128);
       const uint64_t rope_desc0 = sdesc(sbase + kOffKV + kLatAtoms * kAtomBytes, 16, 512, kLayoutSW64);  // K-major rope rows
-      const uint32_t q_t = tmem + kQCol, s_t = tmem + kSCol;
+      const uint32_t q_t = tmem + kQCol, s_t = tmem + kSCol, p_t = tmem + kPCol;
       bool ok = mbar_wait(q_ready, 0, abort_flag, P.err);
       int nq = 0, np = 0;
       uint64_t t0 = 0;
@@ -493,8 +490,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
           const uint64_t st_off = static_cast<uint64_t>(((np % kStages) * kStageBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < kRows / 16; ++kk)
-            tc_mma_f16(tmem, p_desc + ((kk * 32) >> 4), v_desc0 + st_off + ((kk * 16 * 128) >> 4), idesc_o,
-                       (np > 0 || kk > 0) ? 1u : 0u);
+            tc_mma_f16_ts(tmem, p_t + kk * 8, v_desc0 + st_off + ((kk * 16 * 128) >> 4), idesc_o,
+                          (np > 0 || kk > 0) ? 1u : 0u);
           tc_commit(kv_empty(np % kStages));
           tc_commit(pv_done);
           ++np;
@@ -652,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
       // move the running max only when the tile max exceeds it by > 8 (base 2)
       const bool move = mt > m_run + 8.f;
       const bool rescale_o = move && m_run != -INFINITY;
-      // O (and the P buffer) hold tile j - 1's PV once it is done (PV of
+      // O (and P in TMEM) hold tile j - 1's PV once it is done (PV of
       // tile j - 2 was awaited one tile ago, so the parity is unambiguous)
       if (j >= 1 && !mbar_wait_warp(pv_done, (j - 1) & 1, abort_flag, P.err)) { ok = false; break; }
       if (__any_sync(0xffffffffu, rescale_o)) {
@@ -663,22 +660,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
         if (m_run != -INFINITY) l_half *= exp2f(m_run - mt);
         m_run = mt;
       }
-      // P = 2^(s - m) in bf16, 128-byte-swizzled K-major
-      const uint32_t prow = sbase + kOffP + (h >> 3) * 1024 + (h & 7) * 128;
+      // P = 2^(s - m) in bf16 into TMEM (lane = head, column i = rows 2i, 2i+1
+      // of this tile): the A operand of the value MMA
       float psum = 0.f;
+      uint32_t pu[16];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        float p[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          p[e] = (m_run == -INFINITY) ? 0.f : fast_exp2(sreg[c * 8 + e] - m_run);
-          psum += p[e];
-        }
-        st_shared_v4(prow + (((kh * 4 + c) ^ (h & 7)) << 4), pack_bf16(p[0], p[1]), pack_bf16(p[2], p[3]),
-                     pack_bf16(p[4], p[5]), pack_bf16(p[6], p[7]));
+      for (int c = 0; c < 16; ++c) {
+        const float p0 = (m_run == -INFINITY) ? 0.f : fast_exp2(sreg[2 * c] - m_run);
+        const float p1 = (m_run == -INFINITY) ? 0.f : fast_exp2(sreg[2 * c + 1] - m_run);
+        psum += p0 + p1;
+        pu[c] = pack_bf16(p0, p1);
       }
+      tmem_st16(tl + kPCol + 16 * kh, pu);
+      tmem_st_wait();
       l_half += psum;
-      fence_proxy_async_smem();
       tc_fence_before_sync();
       mbar_arrive(pv_ready);
 #pragma unroll
