@@ -63,8 +63,23 @@ __global__ void __launch_bounds__(kThreadsPerBlock) cache_append_kernel(AppendAr
     return;
   }
   const int64_t dst = static_cast<int64_t>(b) * P.s_max + row;
-  // this lane's part of the index key, loaded ahead of the row copies so
-  // that all of the warp's loads are in flight together
+  // All of this lane's loads first (the latent row in up to 4 x 16 bytes, the
+  // key part), then the key's rotation, then the stores: every request of the
+  // warp is in flight at once.  Rows over 2 KB, unaligned rows and the
+  // separate-V form take the general copy.
+  const char* kvs = static_cast<const char*>(P.kv_new) + tok * P.kv_row_bytes;
+  char* kvd = static_cast<char*>(P.kv_cache) + dst * P.kv_row_bytes;
+  const bool kv_fast = P.v_new == nullptr && P.kv_row_bytes <= 4 * 32 * 16 &&
+                       ((reinterpret_cast<uintptr_t>(kvs) | reinterpret_cast<uintptr_t>(kvd) |
+                         static_cast<uintptr_t>(P.kv_row_bytes)) & 15u) == 0;
+  uint4 kvr[4];
+  if (kv_fast) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t o = (u * 32 + lane) * 16;
+      if (o < P.kv_row_bytes) kvr[u] = __ldg(reinterpret_cast<const uint4*>(kvs + o));
+    }
+  }
   char* kdst = static_cast<char*>(P.k_cache) + dst * P.k_row_bytes;
   const char* ksrc = static_cast<const char*>(P.k_new) + tok * (kFP8 ? 128 * sizeof(TK) : P.k_row_bytes);
   const bool key16 = !kFP8 && P.k_row_bytes <= 32 * 16 &&
@@ -79,15 +94,23 @@ __global__ void __launch_bounds__(kThreadsPerBlock) cache_append_kernel(AppendAr
   } else if (key16 && lane * 16 < P.k_row_bytes) {
     kchunk = __ldg(reinterpret_cast<const uint4*>(ksrc + lane * 16));
   }
-  // the attention rows (the larger part)
-  warp_copy(static_cast<char*>(P.kv_cache) + dst * P.kv_row_bytes,
-            static_cast<const char*>(P.kv_new) + tok * P.kv_row_bytes, P.kv_row_bytes, lane);
-  if (P.v_new != nullptr)
-    warp_copy(static_cast<char*>(P.v_cache) + dst * P.v_row_bytes,
-              static_cast<const char*>(P.v_new) + tok * P.v_row_bytes, P.v_row_bytes, lane);
+  if (!kv_fast) {
+    warp_copy(kvd, kvs, P.kv_row_bytes, lane);
+    if (P.v_new != nullptr)
+      warp_copy(static_cast<char*>(P.v_cache) + dst * P.v_row_bytes,
+                static_cast<const char*>(P.v_new) + tok * P.v_row_bytes, P.v_row_bytes, lane);
+  }
+  uint32_t packed = 0;
+  float sigma = 0.f;
+  if (kFP8) packed = rotate_quant_e4m3(kv4, &sigma);
+  if (kv_fast) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t o = (u * 32 + lane) * 16;
+      if (o < P.kv_row_bytes) *reinterpret_cast<uint4*>(kvd + o) = kvr[u];
+    }
+  }
   if (kFP8) {
-    float sigma;
-    const uint32_t packed = rotate_quant_e4m3(kv4, &sigma);
     reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(P.k_cache) + dst * 128)[lane] = packed;
     if (lane == 0) P.k_scale[dst] = sigma;
   } else if (key16) {
