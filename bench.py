@@ -154,8 +154,8 @@ def _attn_extra_launches(wl, dsa, shape):
 # keyed by workload and by the SHA-256 of the indexer source the counters were taken on;
 # a changed kernel reports null.  Filled in from profiles/indexer_tc_decode128k.md.
 TRAFFIC = {
-    # B=8 capture (268,705,280 read + 6,302,976 written) scaled by 4 to B=32: traffic grows with the key tiles
-    "decode128k": ("60292bbc0f4e9c9d", 4 * (268705280 + 6302976)),
+    # B=8 capture (268,701,440 read + 6,647,552 written) scaled by 4 to B=32: traffic grows with the key tiles
+    "decode128k": ("9ff323b1295512fe", 4 * (268701440 + 6647552)),
 }
 
 

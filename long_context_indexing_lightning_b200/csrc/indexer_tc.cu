@@ -330,13 +330,32 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
         }
       }
       const float* wd = w_s + wb * kQG * kHI;
+      // FP8 key scales run four tiles ahead of the accumulators: a scale
+      // loaded after the accumulator wait would put one DRAM latency on
+      // every tile's critical path.
+      const float* ks_row = kFP8 ? k_scale + static_cast<int64_t>(U.b) * S.s_max + row : nullptr;
+      auto load_ks = [&](int t) -> float {
+        return (t < U.kt_comp && t * kTileKeys + row < U.L) ? __ldg(ks_row + t * kTileKeys) : 1.f;
+      };
+      float ks0 = 1.f, ks1 = 1.f, ks2 = 1.f, ks3 = 1.f;
+      if (kFP8) {
+        ks0 = load_ks(U.kt0);
+        ks1 = load_ks(U.kt0 + 1);
+        ks2 = load_ks(U.kt0 + 2);
+        ks3 = load_ks(U.kt0 + 3);
+      }
       bool ok = true;
       for (int kt = U.kt0; kt < U.kt_comp; ++kt) {
+        const float ks = ks0;
+        if (kFP8) {
+          ks0 = ks1;
+          ks1 = ks2;
+          ks2 = ks3;
+          ks3 = load_ks(kt + 4);
+        }
         if (!mbar_wait_warp(acc_full(ab), aph, abort_flag, err)) { ok = false; break; }
         tc_fence_after_sync();
         const int s = kt * kTileKeys + row;
-        float ks = 1.f;
-        if (kFP8 && s < U.L) ks = __ldg(k_scale + static_cast<int64_t>(U.b) * S.s_max + s);
         const uint32_t tl = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(ab * C::N);
         if constexpr (kQG == 1 && kHI == 64) {
           float v0[32], v1[32];

@@ -79,6 +79,7 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads)
   __shared__ uint32_t wsum[kMaxWarps + 1];
   __shared__ uint32_t s_digit, s_above;
   __shared__ uint32_t s_tot[2];
+  __shared__ uint32_t s_off[2];
 
   cg::cluster_group cluster = cg::this_cluster();
   const int C = static_cast<int>(cluster.num_blocks());
@@ -213,16 +214,31 @@ __global__ void __launch_bounds__(kThreads, 1024 / kThreads)
     s_tot[1] = total & 0xFFFFu;
   }
   cluster.sync();  // CTA totals visible across the cluster
-  uint32_t gt_off = 0, eq_off = 0;
-  for (int q = 0; q < c; ++q) {
-    const uint32_t* pt = cluster.map_shared_rank(&s_tot[0], q);
-    gt_off += pt[0];
-    eq_off += pt[1];
+  if (tid < 32) {
+    // offsets of this CTA: the totals of the lower-ranked CTAs, one remote
+    // read per lane, summed across the warp
+    uint32_t g = 0, e = 0;
+    if (tid < c) {
+      const uint32_t* pt = cluster.map_shared_rank(&s_tot[0], tid);
+      g = pt[0];
+      e = pt[1];
+    }
+#pragma unroll
+    for (int off = 1; off < kMaxCluster; off <<= 1) {
+      g += __shfl_xor_sync(0xffffffffu, g, off);
+      e += __shfl_xor_sync(0xffffffffu, e, off);
+    }
+    if (tid == 0) {
+      s_off[0] = g;
+      s_off[1] = e;
+    }
   }
   // every remote read of this CTA is done: arrive now, wait only before
   // leaving (peers may still be reading this CTA's totals), so the index
   // writes below overlap the barrier
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  __syncthreads();
+  const uint32_t gt_off = s_off[0], eq_off = s_off[1];
   uint32_t eq_rank = eq_off + (pre & 0xFFFFu);
   uint32_t pos = gt_off + (pre >> 16) + min(eq_rank, take_eq);
 #pragma unroll
