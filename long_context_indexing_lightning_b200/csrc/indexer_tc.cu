@@ -57,7 +57,12 @@ struct IdxCfg {
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
   static_assert(N % 16 == 0 && N >= 16 && N <= 256, "MMA N");
   static_assert(kHI % 16 == 0, "heads per query");
-  static_assert(kEpiWarps == 4 || (kEpiWarps == 8 && kQG % 2 == 0), "epilogue split");
+  // 8 epilogue warps: two groups of four split the query block (kQG even),
+  // or take alternate key tiles (one query a tile)
+  static constexpr bool kAltTiles = (kEpiWarps == 8 && kQG == 1);
+  static constexpr int kAccArrivals = kAltTiles ? 128 : kEpiThreads;
+  static_assert(kEpiWarps == 4 || (kEpiWarps == 8 && (kQG % 2 == 0 || kQG == 1)), "epilogue split");
+  static_assert(!kAltTiles || kNumAcc % 2 == 0, "alternate tiles need an even accumulator count");
   static_assert(kKTile % 1024 == 0 && kQTile % 1024 == 0, "swizzle atom alignment");
 };
 
@@ -160,7 +165,7 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) { mbar_init(k_full(i), 1); mbar_init(k_empty(i), 1); }
     for (int i = 0; i < kQBufs; ++i) { mbar_init(q_full(i), 1); mbar_init(q_empty(i), 1); }
-    for (int i = 0; i < C::kNumAcc; ++i) { mbar_init(acc_full(i), 1); mbar_init(acc_empty(i), C::kEpiThreads); }
+    for (int i = 0; i < C::kNumAcc; ++i) { mbar_init(acc_full(i), 1); mbar_init(acc_empty(i), C::kAccArrivals); }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -282,10 +287,15 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
     const int e = warp - 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;  // key within the tile == TMEM lane
-    const int jbeg = (kEpiWarps == 8) ? (e >> 2) * (kQG / 2) : 0;
-    const int jend = (kEpiWarps == 8) ? jbeg + kQG / 2 : kQG;
+    const int grp = e >> 2;  // warp group
+    const int jbeg = (kEpiWarps == 8 && !C::kAltTiles) ? grp * (kQG / 2) : 0;
+    const int jend = (kEpiWarps == 8 && !C::kAltTiles) ? jbeg + kQG / 2 : kQG;
+    // alternate tiles: group g takes the CTA's computed tiles n = g, g + 2, ...
+    // (accumulator n % kNumAcc, phase (n / kNumAcc) & 1)
+    constexpr int kStep = C::kAltTiles ? 2 : 1;
+    int ncomp = 0;  // tiles the CTA computed in earlier units
     const int tid_e = threadIdx.x - 64;
-    int ab = 0, wb = 0;
+    int ab = C::kAltTiles ? grp : 0, wb = 0;
     uint32_t aph = 0;
     int last_bg = -1;
     float wreg[kQG == 1 ? kHI : 1];
@@ -337,21 +347,23 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
       auto load_ks = [&](int t) -> float {
         return (t < U.kt_comp && t * kTileKeys + row < U.L) ? __ldg(ks_row + t * kTileKeys) : 1.f;
       };
+      const int kt_first = C::kAltTiles ? U.kt0 + ((grp - ncomp) & 1) : U.kt0;
+      if (C::kAltTiles && U.kt_comp > U.kt0) ncomp += U.kt_comp - U.kt0;
       float ks0 = 1.f, ks1 = 1.f, ks2 = 1.f, ks3 = 1.f;
       if (kFP8) {
-        ks0 = load_ks(U.kt0);
-        ks1 = load_ks(U.kt0 + 1);
-        ks2 = load_ks(U.kt0 + 2);
-        ks3 = load_ks(U.kt0 + 3);
+        ks0 = load_ks(kt_first);
+        ks1 = load_ks(kt_first + kStep);
+        ks2 = load_ks(kt_first + 2 * kStep);
+        ks3 = load_ks(kt_first + 3 * kStep);
       }
       bool ok = true;
-      for (int kt = U.kt0; kt < U.kt_comp; ++kt) {
+      for (int kt = kt_first; kt < U.kt_comp; kt += kStep) {
         const float ks = ks0;
         if (kFP8) {
           ks0 = ks1;
           ks1 = ks2;
           ks2 = ks3;
-          ks3 = load_ks(kt + 4);
+          ks3 = load_ks(kt + 4 * kStep);
         }
         if (!mbar_wait_warp(acc_full(ab), aph, abort_flag, err)) { ok = false; break; }
         tc_fence_after_sync();
@@ -396,11 +408,12 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
         }
         tc_fence_before_sync();
         mbar_arrive(acc_empty(ab));
-        if (++ab == C::kNumAcc) { ab = 0; aph ^= 1; }
+        ab += kStep;
+        if (ab >= C::kNumAcc) { ab -= C::kNumAcc; aph ^= 1; }
       }
       if (!ok) break;
       // key tiles entirely after every query of the block: -inf only
-      for (int kt = U.kt_comp; kt < U.kt_end; ++kt) {
+      for (int kt = U.kt_comp + (C::kAltTiles ? grp : 0); kt < U.kt_end; kt += kStep) {
         const int s = kt * kTileKeys + row;
         if (s < U.L)
           for (int j = jbeg; j < min(jend, U.nq); ++j)
@@ -485,7 +498,7 @@ dsa_status_t indexer_tc(const IndexerArgs& a) {
   const bool one = (a.n_q == 1);
 #define DSA_IDX_CASE(HI, QGP)                                                              \
   if (a.H == HI) {                                                                         \
-    if (one) return fp8 ? launch_indexer_tc<true, 1, HI, 4, 12, 2>(a)                       \
+    if (one) return fp8 ? launch_indexer_tc<true, 1, HI, 8, 12, 2>(a)                       \
                         : launch_indexer_tc<false, 1, HI, 4, 5, 2>(a);                     \
     return fp8 ? launch_indexer_tc<true, QGP, HI, ((QGP) % 2 == 0 ? 8 : 4), 6, 1>(a)       \
                : launch_indexer_tc<false, QGP, HI, ((QGP) % 2 == 0 ? 8 : 4), 4, 1>(a);     \
