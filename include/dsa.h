@@ -227,7 +227,14 @@ dsa_status_t dsa_forward(const dsa_shape_t *shape,
  * k_idx, k_scale, kv, v stay on the device as the layer's resident state.
  * The call copies the inputs in (one cudaMemcpyAsync each), runs the step,
  * copies the outputs back and synchronises `stream` before returning.
- * workspace: dsa_workspace_bytes(shape, DSA_WS_FORWARD_HOST) bytes.
+ * workspace: dsa_workspace_bytes(shape, DSA_WS_FORWARD_HOST) bytes: the
+ * scratch of dsa_forward, two input staging slots (consecutive host-buffer
+ * calls on a device alternate between them) and the output staging.  The
+ * inputs are copied on a stream of the library's own, which waits for the
+ * last call that used the same slot; it waits for `stream` too when the
+ * workspace address differs from the previous host-buffer call's.  So
+ * between two host-buffer calls with the same workspace, the caller must
+ * not use that memory for anything else.
  */
 dsa_status_t dsa_forward_host(const dsa_shape_t *shape,
                               const void *h_q_idx, const float *h_w, const void *h_q,
@@ -237,6 +244,41 @@ dsa_status_t dsa_forward_host(const dsa_shape_t *shape,
                               void *h_out, float *h_lse,
                               void *workspace, size_t workspace_bytes,
                               void *stream);
+
+/*
+ * dsa_forward_host for a loop of steps whose copies overlap one another's
+ * compute (the pages have no counterpart; it is the serving-loop form of the
+ * call above).  Arguments as in dsa_forward_host, plus:
+ *   done_event  a cudaEvent_t (passed as void*) created by the caller on the
+ *               same device, or NULL.  It is recorded once this call's
+ *               outputs are in h_out / h_lse.
+ * The call returns once the work is enqueued; it does not synchronise.
+ *   - The inputs are copied in on a stream of the library's own into the
+ *     call's staging slot (as in dsa_forward_host): the indexer waits for
+ *     its inputs, the attention for the queries, and the copies need not
+ *     wait for the previous call's compute, only for the call before it
+ *     (the last one that used the slot) to finish its attention.
+ *   - The outputs are copied back on a second stream of the library's own
+ *     after the step's attention, so that the copy runs under the next
+ *     call's indexer and top-k.  The next host-buffer call on the device
+ *     (either form) waits for that copy before its attention rewrites the
+ *     device output, so one workspace serves consecutive calls.
+ *   - Host buffers: the inputs must stay unchanged, and h_out / h_lse must
+ *     not be read, until done_event has completed (or the device has been
+ *     synchronised).
+ *   - Errors: argument errors return before anything is enqueued; device
+ *     errors are read with dsa_get_error.  Calls on one device are
+ *     serialised by the caller (the library's streams and events are per
+ *     device).
+ */
+dsa_status_t dsa_forward_host_async(const dsa_shape_t *shape,
+                                    const void *h_q_idx, const float *h_w, const void *h_q,
+                                    const int32_t *h_ctx_len, const int32_t *h_q_pos0,
+                                    const void *k_idx, const float *k_scale,
+                                    const void *kv, const void *v,
+                                    void *h_out, float *h_lse,
+                                    void *workspace, size_t workspace_bytes,
+                                    void *done_event, void *stream);
 
 /*
  * dsa_sparse_mla_attn without a workspace argument: the scratch memory that

@@ -27,7 +27,7 @@ STATUS = {
 EXPORTS = (
     "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_attn", "dsa_hadamard_quant_fp8", "dsa_cache_append",
     "dsa_forward",
-    "dsa_forward_host", "dsa_workspace_bytes", "dsa_get_error", "dsa_status_string", "dsa_version",
+    "dsa_forward_host", "dsa_forward_host_async", "dsa_workspace_bytes", "dsa_get_error", "dsa_status_string", "dsa_version",
     "dsa_sparse_mla_attn_static", "dsa_selftest_wait_timeout",
 )
 
@@ -77,6 +77,7 @@ def lib():
         L.dsa_selftest_wait_timeout.argtypes = [P]
         L.dsa_forward.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
         L.dsa_forward_host.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, sz, P]
+        L.dsa_forward_host_async.argtypes = [S, P, P, P, P, P, P, P, P, P, P, P, P, sz, P, P]
         L.dsa_workspace_bytes.argtypes = [S, i32]
         L.dsa_workspace_bytes.restype = sz
         L.dsa_get_error.argtypes = [i32, ctypes.POINTER(ctypes.c_uint32)]
@@ -230,6 +231,23 @@ def forward_host(shape, h_q_idx, h_w, h_q, h_ctx_len, h_q_pos0, k_idx, kv, h_out
     _check(lib().dsa_forward_host(ctypes.byref(shape), _p(h_q_idx), _p(h_w), _p(h_q), _p(h_ctx_len), _p(h_q_pos0),
                                   _p(k_idx), _p(k_scale), _p(kv), _p(v), _p(h_out), _p(h_lse), _p(ws), n,
                                   _stream(stream)), "dsa_forward_host")
+    return h_out
+
+
+def forward_host_async(shape, h_q_idx, h_w, h_q, h_ctx_len, h_q_pos0, k_idx, kv, h_out, done=None, v=None,
+                       k_scale=None, h_lse=None, workspace=None, stream=None):
+    """The host-buffer step, returning once enqueued (see dsa_forward_host_async).
+    `done`: a torch.cuda.Event recorded once h_out / h_lse hold this call's
+    outputs (or None)."""
+    ws, n = _workspace(shape, WS_FORWARD_HOST, workspace, k_idx.device)
+    ev = None
+    if done is not None:
+        if not done.cuda_event:  # torch creates the event on its first record
+            done.record(torch.cuda.current_stream(k_idx.device))
+        ev = done.cuda_event
+    _check(lib().dsa_forward_host_async(ctypes.byref(shape), _p(h_q_idx), _p(h_w), _p(h_q), _p(h_ctx_len),
+                                        _p(h_q_pos0), _p(k_idx), _p(k_scale), _p(kv), _p(v), _p(h_out), _p(h_lse),
+                                        _p(ws), n, ev, _stream(stream)), "dsa_forward_host_async")
     return h_out
 
 

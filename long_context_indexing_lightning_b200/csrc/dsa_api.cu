@@ -158,8 +158,12 @@ struct FwdLayout {
   size_t off_scores, off_idx, off_q8, off_qs, off_topk, off_attn;
   size_t topk_bytes, attn_bytes;
   size_t total;
-  // host-variant staging
-  size_t off_h_qidx, off_h_w, off_h_q, off_h_ctx, off_h_pos, off_h_out, off_h_lse;
+  // host-variant staging: two input slots (consecutive calls alternate, so a
+  // call's inputs can be copied in while the previous call still reads its
+  // own), offsets of each input within a slot, one output area
+  size_t off_h_in[2];
+  size_t off_h_qidx, off_h_w, off_h_q, off_h_ctx, off_h_pos;
+  size_t off_h_out, off_h_lse;
   size_t total_host;
 };
 
@@ -190,16 +194,20 @@ FwdLayout forward_layout(const dsa_shape_t* s) {
   // staging for dsa_forward_host
   const size_t ai = elem_size(s->idx_dtype == DSA_E4M3 ? DSA_BF16 : s->idx_dtype);
   const size_t aa = elem_size(s->attn_dtype);
-  L.off_h_qidx = off;
-  off = align_up(off + static_cast<size_t>(B) * s->n_q * s->idx_heads * s->idx_dim * ai, 256);
-  L.off_h_w = off;
-  off = align_up(off + static_cast<size_t>(B) * s->n_q * s->idx_heads * 4, 256);
-  L.off_h_q = off;
-  off = align_up(off + static_cast<size_t>(B) * s->n_q * s->heads * s->d_qk * aa, 256);
-  L.off_h_ctx = off;
-  off = align_up(off + static_cast<size_t>(B) * 4, 256);
-  L.off_h_pos = off;
-  off = align_up(off + static_cast<size_t>(B) * 4, 256);
+  size_t in = 0;
+  L.off_h_qidx = in;
+  in = align_up(in + static_cast<size_t>(B) * s->n_q * s->idx_heads * s->idx_dim * ai, 256);
+  L.off_h_w = in;
+  in = align_up(in + static_cast<size_t>(B) * s->n_q * s->idx_heads * 4, 256);
+  L.off_h_q = in;
+  in = align_up(in + static_cast<size_t>(B) * s->n_q * s->heads * s->d_qk * aa, 256);
+  L.off_h_ctx = in;
+  in = align_up(in + static_cast<size_t>(B) * 4, 256);
+  L.off_h_pos = in;
+  in = align_up(in + static_cast<size_t>(B) * 4, 256);
+  L.off_h_in[0] = off;
+  L.off_h_in[1] = off + in;
+  off += 2 * in;
   L.off_h_out = off;
   off = align_up(off + static_cast<size_t>(B) * s->n_q * s->heads * s->d_v * aa, 256);
   L.off_h_lse = off;
@@ -241,22 +249,46 @@ dsa_status_t check_attn_inputs(const dsa_shape_t* s, const void* q, const void* 
 
 int device_sm_count(int dev) { return (dev >= 0 && dev < kMaxDevices) ? g_sm_count[dev] : 0; }
 
-// The host-buffer entry point copies the attention queries on a second stream
-// of the library's own, so that the copy overlaps the indexer and top-k.
-// Created once per device on first use, with two events to join the streams.
-cudaStream_t g_copy_stream[kMaxDevices] = {};
-cudaEvent_t g_ev_start[kMaxDevices] = {}, g_ev_q[kMaxDevices] = {};
+// The host-buffer entry points copy their inputs in on a stream of the
+// library's own, into one of two staging slots of the workspace (consecutive
+// calls alternate), so that a call's copies run while the previous call
+// computes; the asynchronous one also copies the output back on a third
+// stream, under the next call's indexer and top-k.  Created once per device
+// on first use, with the events that join the streams:
+//   g_ev_free[p]  the attention of the last call that used slot p is done
+//                 (the next copy into slot p waits for it),
+//   g_ev_in       the indexer inputs of a call are in its slot,
+//   g_ev_q        the attention queries of a call are in its slot,
+//   g_ev_attn     the attention of the last asynchronous call is done,
+//   g_ev_out      the output copy of the last asynchronous call is done (the
+//                 next call's attention, which rewrites the output, waits),
+//   g_ev_join     the compute stream reached a call with a workspace other
+//                 than the last one: the copy stream starts after it, since
+//                 memory just handed out by a stream-ordered allocator may
+//                 still be in use by earlier work on that stream.
+cudaStream_t g_copy_stream[kMaxDevices] = {}, g_out_stream[kMaxDevices] = {};
+cudaEvent_t g_ev_free[kMaxDevices][2] = {}, g_ev_in[kMaxDevices] = {}, g_ev_q[kMaxDevices] = {};
+cudaEvent_t g_ev_attn[kMaxDevices] = {}, g_ev_out[kMaxDevices] = {}, g_ev_join[kMaxDevices] = {};
+int g_slot[kMaxDevices] = {};
+const void* g_last_ws[kMaxDevices] = {};
 bool ensure_copy_stream(int dev) {
   std::lock_guard<std::mutex> lock(g_mutex);
   if (g_copy_stream[dev] != nullptr) return true;
-  cudaStream_t s = nullptr;
-  cudaEvent_t a = nullptr, b = nullptr;
-  if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) return false;
-  if (cudaEventCreateWithFlags(&a, cudaEventDisableTiming) != cudaSuccess ||
-      cudaEventCreateWithFlags(&b, cudaEventDisableTiming) != cudaSuccess)
+  cudaStream_t s = nullptr, so = nullptr;
+  cudaEvent_t ev[7] = {};
+  if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaStreamCreateWithFlags(&so, cudaStreamNonBlocking) != cudaSuccess)
     return false;
-  g_ev_start[dev] = a;
-  g_ev_q[dev] = b;
+  for (cudaEvent_t& e : ev)
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return false;
+  g_ev_free[dev][0] = ev[0];
+  g_ev_free[dev][1] = ev[1];
+  g_ev_in[dev] = ev[2];
+  g_ev_q[dev] = ev[3];
+  g_ev_attn[dev] = ev[4];
+  g_ev_out[dev] = ev[5];
+  g_ev_join[dev] = ev[6];
+  g_out_stream[dev] = so;
   g_copy_stream[dev] = s;
   return true;
 }
@@ -414,7 +446,8 @@ static dsa_status_t forward_impl(const dsa_shape_t* s, int dev, cudaStream_t st,
                                  const float* q_scale, const void* k_idx, const float* k_scale, const float* w,
                                  const void* q, const void* kv, const void* v, const int32_t* ctx_len,
                                  const int32_t* q_pos0, void* out, float* lse, int32_t* idx_out, uint8_t* ws,
-                                 const FwdLayout& L, cudaEvent_t q_ready = nullptr) {
+                                 const FwdLayout& L, cudaEvent_t q_ready = nullptr,
+                                 cudaEvent_t out_free = nullptr) {
   const int B = s->batch, n_q = s->n_q;
   if (B == 0 || n_q == 0) return DSA_OK;
   dsa_status_t rc;
@@ -439,6 +472,7 @@ static dsa_status_t forward_impl(const dsa_shape_t* s, int dev, cudaStream_t st,
     rc = run_topk(&si, dev, st, B, n_q, 0, scores, L.ld, ctx_len, q_pos0, idx, ws + L.off_topk, L.topk_bytes);
     if (rc != DSA_OK) return rc;
     if (q_ready != nullptr && cudaStreamWaitEvent(st, q_ready, 0) != cudaSuccess) return DSA_ERR_CUDA;
+    if (out_free != nullptr && cudaStreamWaitEvent(st, out_free, 0) != cudaSuccess) return DSA_ERR_CUDA;
     return run_attn(&si, dev, st, B, n_q, q, kv, v, idx, ctx_len, out, lse, ws + L.off_attn, L.attn_bytes);
   }
   // Rounds of `chunk` queries, one sequence at a time (positions shift by t0).
@@ -464,8 +498,10 @@ static dsa_status_t forward_impl(const dsa_shape_t* s, int dev, cudaStream_t st,
       rc = run_topk(&si, dev, st, 1, c, t0, scores, L.ld, ctx_len + b, q_pos0 + b, idx_b, ws + L.off_topk,
                     L.topk_bytes);
       if (rc != DSA_OK) return rc;
-      if (q_ready != nullptr && b == 0 && t0 == 0 && cudaStreamWaitEvent(st, q_ready, 0) != cudaSuccess)
-        return DSA_ERR_CUDA;
+      if (b == 0 && t0 == 0) {
+        if (q_ready != nullptr && cudaStreamWaitEvent(st, q_ready, 0) != cudaSuccess) return DSA_ERR_CUDA;
+        if (out_free != nullptr && cudaStreamWaitEvent(st, out_free, 0) != cudaSuccess) return DSA_ERR_CUDA;
+      }
       rc = run_attn(&si, dev, st, 1, c, q_b, kv_b, v_b, idx_b, ctx_len + b, out_b, lse_b, ws + L.off_attn,
                     L.attn_bytes);
       if (rc != DSA_OK) return rc;
@@ -511,10 +547,17 @@ dsa_status_t dsa_forward(const dsa_shape_t* shape, const void* q_idx, const floa
                       ctx_len, q_pos0, out, lse, idx_out, static_cast<uint8_t*>(workspace), L);
 }
 
-dsa_status_t dsa_forward_host(const dsa_shape_t* shape, const void* h_q_idx, const float* h_w, const void* h_q,
-                              const int32_t* h_ctx_len, const int32_t* h_q_pos0, const void* k_idx,
-                              const float* k_scale, const void* kv, const void* v, void* h_out, float* h_lse,
-                              void* workspace, size_t workspace_bytes, void* stream) {
+// The step with host-memory inputs and outputs.  Synchronous: the output is
+// copied back on the compute stream and the call returns after it.
+// Asynchronous: the output is copied back on the library's output stream
+// after the attention, `done` (if given) is recorded after that copy, and the
+// call returns once everything is enqueued; the next call's attention waits
+// for the copy before it rewrites the device output.
+static dsa_status_t forward_host_impl(const dsa_shape_t* shape, const void* h_q_idx, const float* h_w,
+                                      const void* h_q, const int32_t* h_ctx_len, const int32_t* h_q_pos0,
+                                      const void* k_idx, const float* k_scale, const void* kv, const void* v,
+                                      void* h_out, float* h_lse, void* workspace, size_t workspace_bytes,
+                                      void* stream, bool async, cudaEvent_t done) {
   dsa_status_t st = check_forward(shape, h_q_idx, nullptr, k_idx, k_scale, h_w, h_q, kv, v, h_ctx_len, h_q_pos0,
                                   h_out, true);
   if (st != DSA_OK) return st;
@@ -531,34 +574,72 @@ dsa_status_t dsa_forward_host(const dsa_shape_t* shape, const void* h_q_idx, con
   const size_t n_q_b = static_cast<size_t>(B) * n_q * shape->heads * shape->d_qk * aa;
   const size_t n_out = static_cast<size_t>(B) * n_q * shape->heads * shape->d_v * aa;
   const size_t n_lse = static_cast<size_t>(B) * n_q * shape->heads * 4;
-  // the attention queries (the bulk of the input) travel on the copy stream,
-  // under the indexer and top-k; the stream waits for them before attention
+  // inputs travel on the copy stream into this call's slot, once the last
+  // call that used the slot has finished its attention: the indexer inputs
+  // first (the compute stream waits for them), then the attention queries
+  // (the bulk of the input: waited for just before attention, so that they
+  // land under the indexer and top-k)
   if (!ensure_copy_stream(dev)) return DSA_ERR_CUDA;
   const cudaStream_t xs = g_copy_stream[dev];
-  if (cudaEventRecord(g_ev_start[dev], cs) != cudaSuccess || cudaStreamWaitEvent(xs, g_ev_start[dev], 0) != cudaSuccess ||
-      cudaMemcpyAsync(ws + L.off_h_q, h_q, n_q_b, cudaMemcpyHostToDevice, xs) != cudaSuccess ||
-      cudaEventRecord(g_ev_q[dev], xs) != cudaSuccess)
-    return DSA_ERR_CUDA;
-  if (cudaMemcpyAsync(ws + L.off_h_qidx, h_q_idx, n_qidx, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
-      cudaMemcpyAsync(ws + L.off_h_w, h_w, n_w, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
-      cudaMemcpyAsync(ws + L.off_h_ctx, h_ctx_len, static_cast<size_t>(B) * 4, cudaMemcpyHostToDevice, cs) !=
+  const int slot = g_slot[dev];
+  g_slot[dev] ^= 1;
+  uint8_t* in = ws + L.off_h_in[slot];
+  if (g_last_ws[dev] != workspace) {
+    if (cudaEventRecord(g_ev_join[dev], cs) != cudaSuccess || cudaStreamWaitEvent(xs, g_ev_join[dev], 0) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    g_last_ws[dev] = workspace;
+  }
+  if (cudaStreamWaitEvent(xs, g_ev_free[dev][slot], 0) != cudaSuccess ||
+      cudaMemcpyAsync(in + L.off_h_qidx, h_q_idx, n_qidx, cudaMemcpyHostToDevice, xs) != cudaSuccess ||
+      cudaMemcpyAsync(in + L.off_h_w, h_w, n_w, cudaMemcpyHostToDevice, xs) != cudaSuccess ||
+      cudaMemcpyAsync(in + L.off_h_ctx, h_ctx_len, static_cast<size_t>(B) * 4, cudaMemcpyHostToDevice, xs) !=
           cudaSuccess ||
-      cudaMemcpyAsync(ws + L.off_h_pos, h_q_pos0, static_cast<size_t>(B) * 4, cudaMemcpyHostToDevice, cs) !=
-          cudaSuccess)
+      cudaMemcpyAsync(in + L.off_h_pos, h_q_pos0, static_cast<size_t>(B) * 4, cudaMemcpyHostToDevice, xs) !=
+          cudaSuccess ||
+      cudaEventRecord(g_ev_in[dev], xs) != cudaSuccess ||
+      cudaMemcpyAsync(in + L.off_h_q, h_q, n_q_b, cudaMemcpyHostToDevice, xs) != cudaSuccess ||
+      cudaEventRecord(g_ev_q[dev], xs) != cudaSuccess || cudaStreamWaitEvent(cs, g_ev_in[dev], 0) != cudaSuccess)
     return DSA_ERR_CUDA;
   dsa_shape_t s2 = *shape;
-  st = forward_impl(&s2, dev, cs, ws + L.off_h_qidx, nullptr, k_idx, k_scale, reinterpret_cast<float*>(ws + L.off_h_w),
-                    ws + L.off_h_q, kv, v, reinterpret_cast<int32_t*>(ws + L.off_h_ctx),
-                    reinterpret_cast<int32_t*>(ws + L.off_h_pos), ws + L.off_h_out,
-                    h_lse ? reinterpret_cast<float*>(ws + L.off_h_lse) : nullptr, nullptr, ws, L, g_ev_q[dev]);
+  st = forward_impl(&s2, dev, cs, in + L.off_h_qidx, nullptr, k_idx, k_scale, reinterpret_cast<float*>(in + L.off_h_w),
+                    in + L.off_h_q, kv, v, reinterpret_cast<int32_t*>(in + L.off_h_ctx),
+                    reinterpret_cast<int32_t*>(in + L.off_h_pos), ws + L.off_h_out,
+                    h_lse ? reinterpret_cast<float*>(ws + L.off_h_lse) : nullptr, nullptr, ws, L, g_ev_q[dev],
+                    g_ev_out[dev]);
   // (already waited before attention; again here so that no copy into the
   // workspace is left in flight on any path)
   if (cudaStreamWaitEvent(cs, g_ev_q[dev], 0) != cudaSuccess && st == DSA_OK) st = DSA_ERR_CUDA;
+  if (cudaStreamWaitEvent(cs, g_ev_out[dev], 0) != cudaSuccess && st == DSA_OK) st = DSA_ERR_CUDA;
   if (st != DSA_OK) return st;
-  if (cudaMemcpyAsync(h_out, ws + L.off_h_out, n_out, cudaMemcpyDeviceToHost, cs) != cudaSuccess) return DSA_ERR_CUDA;
-  if (h_lse && cudaMemcpyAsync(h_lse, ws + L.off_h_lse, n_lse, cudaMemcpyDeviceToHost, cs) != cudaSuccess)
+  if (cudaEventRecord(g_ev_free[dev][slot], cs) != cudaSuccess) return DSA_ERR_CUDA;  // the slot is read
+  const cudaStream_t os = async ? g_out_stream[dev] : cs;
+  if (async && (cudaEventRecord(g_ev_attn[dev], cs) != cudaSuccess ||
+                cudaStreamWaitEvent(os, g_ev_attn[dev], 0) != cudaSuccess))
     return DSA_ERR_CUDA;
-  return cudaStreamSynchronize(cs) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  if (cudaMemcpyAsync(h_out, ws + L.off_h_out, n_out, cudaMemcpyDeviceToHost, os) != cudaSuccess) return DSA_ERR_CUDA;
+  if (h_lse && cudaMemcpyAsync(h_lse, ws + L.off_h_lse, n_lse, cudaMemcpyDeviceToHost, os) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  if (!async) return cudaStreamSynchronize(cs) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  if (cudaEventRecord(g_ev_out[dev], os) != cudaSuccess) return DSA_ERR_CUDA;
+  if (done != nullptr && cudaEventRecord(done, os) != cudaSuccess) return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
+dsa_status_t dsa_forward_host(const dsa_shape_t* shape, const void* h_q_idx, const float* h_w, const void* h_q,
+                              const int32_t* h_ctx_len, const int32_t* h_q_pos0, const void* k_idx,
+                              const float* k_scale, const void* kv, const void* v, void* h_out, float* h_lse,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  return forward_host_impl(shape, h_q_idx, h_w, h_q, h_ctx_len, h_q_pos0, k_idx, k_scale, kv, v, h_out, h_lse,
+                           workspace, workspace_bytes, stream, false, nullptr);
+}
+
+dsa_status_t dsa_forward_host_async(const dsa_shape_t* shape, const void* h_q_idx, const float* h_w,
+                                    const void* h_q, const int32_t* h_ctx_len, const int32_t* h_q_pos0,
+                                    const void* k_idx, const float* k_scale, const void* kv, const void* v,
+                                    void* h_out, float* h_lse, void* workspace, size_t workspace_bytes,
+                                    void* done_event, void* stream) {
+  return forward_host_impl(shape, h_q_idx, h_w, h_q, h_ctx_len, h_q_pos0, k_idx, k_scale, kv, v, h_out, h_lse,
+                           workspace, workspace_bytes, stream, true, static_cast<cudaEvent_t>(done_event));
 }
 
 dsa_status_t dsa_get_error(int32_t clear, uint32_t* detail) {

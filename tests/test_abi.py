@@ -74,6 +74,11 @@ def test_argument_errors_need_no_gpu(L):
     assert L.dsa_cache_append(ctypes.byref(e4.replace(idx_dim=64)), 1, 16, 16, None, 16, 16, 16, 16, None, None) == 2
     assert L.dsa_cache_append(ctypes.byref(s.replace(d_qk=575)), 1, 16, 16, None, 16, 16, None, 16, None, None) == 2
     assert L.dsa_cache_append(ctypes.byref(s), 1, 18, 16, None, 16, 16, None, 16, None, None) == 1
+    # host-buffer step, asynchronous form: null inputs, a workspace too small
+    assert L.dsa_forward_host_async(ctypes.byref(s), None, None, None, None, None, 16, None, 16, None, 16, None,
+                                    16, 1 << 30, None, None) == 1
+    assert L.dsa_forward_host_async(ctypes.byref(s), 16, 16, 16, 16, 16, 16, None, 16, None, 16, None,
+                                    16, 16, None, None) == 3
 
 
 def test_workspace_arithmetic(L):

@@ -368,6 +368,34 @@ def test_forward_host_buffers_match_device_call():
     assert np.abs(h_out.float().numpy().reshape(4, wl.heads, wl.d_v) - o).max() <= ATTN_ATOL_BF16
 
 
+def test_forward_host_async_calls_in_flight_share_one_workspace():
+    """Three asynchronous host-buffer steps on different inputs, enqueued back
+    to back on one workspace (each output copy runs under the next step), then
+    a synchronous one: every output equals the device-buffer call's."""
+    wl = _custom("decode32k", batch=4, s_max=8192)
+    shape = dsa.shape_from_workload(wl)
+    ins = [workloads.make_inputs(wl, DEV, seed=20 + i) for i in range(3)]
+    want = [dsa.forward(shape, t["q_idx"], t["k_idx"], t["w"], t["q"], t["kv"], t["ctx_len"], t["q_pos0"]).cpu()
+            for t in ins]
+    pin = lambda x: x.cpu().pin_memory()
+    hin = [{k: pin(t[k]) for k in ("q_idx", "w", "q", "ctx_len", "q_pos0")} for t in ins]
+    ws = torch.empty(dsa.workspace_bytes(shape, dsa.WS_FORWARD_HOST), dtype=torch.uint8, device=DEV)
+    h_out = [torch.empty(want[0].shape, dtype=want[0].dtype).pin_memory() for _ in range(4)]
+    done = [torch.cuda.Event() for _ in range(3)]
+    torch.cuda.synchronize()
+    for i, (t, h) in enumerate(zip(ins, hin)):
+        dsa.forward_host_async(shape, h["q_idx"], h["w"], h["q"], h["ctx_len"], h["q_pos0"], t["k_idx"], t["kv"],
+                               h_out[i], done=done[i], workspace=ws)
+    h = hin[0]
+    dsa.forward_host(shape, h["q_idx"], h["w"], h["q"], h["ctx_len"], h["q_pos0"], ins[0]["k_idx"], ins[0]["kv"],
+                     h_out[3], workspace=ws)
+    for i in range(3):
+        done[i].synchronize()
+        torch.testing.assert_close(h_out[i], want[i], rtol=0, atol=0)
+    torch.testing.assert_close(h_out[3], want[0], rtol=0, atol=0)
+    assert dsa.get_error()[0] == 0
+
+
 # --------------------------------------------------------------------- FP8 --
 
 def _codes_ok(g_code, o_code, quot):
