@@ -154,8 +154,8 @@ def _attn_extra_launches(wl, dsa, shape):
 # keyed by workload and by the SHA-256 of the indexer source the counters were taken on;
 # a changed kernel reports null.  Filled in from profiles/indexer_tc_decode128k.md.
 TRAFFIC = {
-    # B=8 capture (268,701,440 read + 6,647,552 written) scaled by 4 to B=32: traffic grows with the key tiles
-    "decode128k": ("9ff323b1295512fe", 4 * (268701440 + 6647552)),
+    # B=8 capture (268,703,488 read + 7,743,744 written) scaled by 4 to B=32: traffic grows with the key tiles
+    "decode128k": ("bfd6d9283dfdb902", 4 * (268703488 + 7743744)),
 }
 
 
