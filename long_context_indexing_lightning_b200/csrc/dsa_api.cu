@@ -610,8 +610,10 @@ static dsa_status_t forward_host_impl(const dsa_shape_t* shape, const void* h_q_
   // workspace is left in flight on any path)
   if (cudaStreamWaitEvent(cs, g_ev_q[dev], 0) != cudaSuccess && st == DSA_OK) st = DSA_ERR_CUDA;
   if (cudaStreamWaitEvent(cs, g_ev_out[dev], 0) != cudaSuccess && st == DSA_OK) st = DSA_ERR_CUDA;
+  // the slot is free once everything enqueued so far has run, on the error
+  // paths too (kernels enqueued before a failure may still read it)
+  if (cudaEventRecord(g_ev_free[dev][slot], cs) != cudaSuccess && st == DSA_OK) st = DSA_ERR_CUDA;
   if (st != DSA_OK) return st;
-  if (cudaEventRecord(g_ev_free[dev][slot], cs) != cudaSuccess) return DSA_ERR_CUDA;  // the slot is read
   const cudaStream_t os = async ? g_out_stream[dev] : cs;
   if (async && (cudaEventRecord(g_ev_attn[dev], cs) != cudaSuccess ||
                 cudaStreamWaitEvent(os, g_ev_attn[dev], 0) != cudaSuccess))
