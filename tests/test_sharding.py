@@ -119,3 +119,42 @@ def test_gather_range_must_fit_the_cache():
             sharding.gather_cache_rows(torch.zeros(1, 10, 2), 0, 3, 5)  # 4 chunks of 2 rows from row 3 > 10
     finally:
         dist.get_world_size, dist.get_rank = orig
+
+
+def _worker_dropout(rank, world, port, out):
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    import time
+    import torch.distributed as dist
+    from long_context_indexing_lightning_b200 import sharding as sh
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=10))
+    if rank == 1:
+        # this rank leaves between steps, before the exchange, without a word
+        os._exit(0)
+    cache = torch.zeros(1, 32, 4, dtype=torch.bfloat16)
+    t0 = time.monotonic()
+    try:
+        sh.gather_cache_rows(cache, 0, 0, 32)
+        out[rank] = ("no error", time.monotonic() - t0)
+    except Exception as e:  # the survivor learns of it from the collective
+        out[rank] = (type(e).__name__, time.monotonic() - t0)
+
+
+def test_a_rank_that_leaves_before_the_exchange_fails_the_collective():
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        out = mgr.dict()
+        procs = [ctx.Process(target=_worker_dropout, args=(r, 2, port, out)) for r in range(2)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(timeout=120)
+        for p in procs:
+            if p.is_alive():
+                p.kill()
+        res = dict(out)
+    assert 0 in res, "the surviving rank did not report"
+    kind, secs = res[0]
+    assert kind != "no error" and secs < 60, res
