@@ -280,6 +280,29 @@ def test_topk_matches_lexsort_bruteforce(seed):
         np.testing.assert_array_equal(idx[r], _brute_topk(scores[r], pos[r], k))
 
 
+def test_topk_matches_bruteforce_on_arbitrary_finite_floats():
+    """Property test: any finite fp32 values (subnormals, signed zeros, the
+    extremes, heavy repetition), any row length, k and causal position."""
+    hyp = pytest.importorskip("hypothesis")
+    st = hyp.strategies
+
+    finite = st.floats(width=32, allow_nan=False, allow_infinity=False)
+    pool = st.lists(finite, min_size=1, max_size=6)  # few distinct values -> ties
+
+    @hyp.settings(max_examples=300, deadline=None, derandomize=True)
+    @hyp.given(data=st.data())
+    def check(data):
+        S = data.draw(st.integers(1, 48))
+        vals = data.draw(pool)
+        row = np.array(data.draw(st.lists(st.sampled_from(vals), min_size=S, max_size=S)), np.float32)
+        p = data.draw(st.integers(0, S - 1))
+        k = data.draw(st.integers(1, S + 3))
+        got = oracle.topk(row[None, :], np.array([p], np.int32), k)[0]
+        np.testing.assert_array_equal(got, _brute_topk(row, p, k))
+
+    check()
+
+
 def test_topk_invariants():
     g = np.random.default_rng(11)
     S, k = 50, 16
