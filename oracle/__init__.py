@@ -45,6 +45,7 @@ def _load():
                                         P, i32, f64, i32, P, P, P, P]
         lib.orc_dense_masked_attn.argtypes = [i32, i32, i32, i32, i32, i32, P, i32, P, i32, P, i32,
                                               P, P, i32, f64, i32, P, P, P]
+        lib.orc_linear.argtypes = [i64, i32, i32, P, i32, P, i32, P]
         lib.orc_num_threads.restype = i32
         _lib = lib
     return _lib
@@ -178,6 +179,25 @@ def cache_append(k_cache, kv_cache, k_new, kv_new, pos, k_scale=None, v_cache=No
             if v_cache is not None:
                 v_cache[b, r] = v_new[b, i]
     return k_cache, k_scale, kv_cache, v_cache
+
+
+def linear(x, w):
+    """The indexer's projections (DeepSeek-V3.2 doc: `wq_b` on the query
+    latent, the single-head key projection, `weights_proj`): Y = X W^T in fp64.
+
+    x [..., K] and w [N, K] in a stored type (fp32 or bf16 bits).  Returns
+    fp64 [..., N].
+    """
+    xa, xt = _typed(x)
+    wa, wt = _typed(w)
+    K = xa.shape[-1]
+    N = wa.shape[0]
+    if wa.shape[1] != K:
+        raise ValueError("x and w disagree on K")
+    M = xa.size // K
+    y = np.empty(xa.shape[:-1] + (N,), dtype=np.float64)
+    _load().orc_linear(M, N, K, _ptr(xa), xt, _ptr(wa), wt, _ptr(y))
+    return y
 
 
 def e4m3_encode(x):

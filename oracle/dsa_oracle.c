@@ -28,6 +28,10 @@
  *            qk_rope_head_dim 64.
  *   [USE]    section "Usage example": the indexer's weights_proj stays out of
  *            FP8 quantisation.
+ *   [PROJ]   the note on the query LoRA path (the indexer scores queries from
+ *            the low-rank latent q_a_layernorm(q_a_proj(x)) through `wq_b`,
+ *            sized by q_lora_rank) with [CFG] and [USE]: the indexer's
+ *            projections are plain linear maps kept in bf16.
  * The score's combination rule (per-head ReLU of the query-key dot product,
  * summed over index heads with the weights_proj outputs as weights) is a
  * reading of [DSA-1] + [USE]; the pages do not print the formula.
@@ -485,6 +489,31 @@ void orc_dense_masked_attn(int n_q, int s_max, int H, int KVH, int d_qk, int d_v
         }
         free(logit);
         free(mask);
+    }
+}
+
+/* ------------------------------------------------------ projections -- */
+
+/*
+ * The indexer's linear projections [PROJ]: Y = X W^T, written out,
+ *     Y[m][n] = sum_k X[m][k] * W[n][k],
+ * with X [M][K] and W [N][K] in a stored type (fp32 or bf16 bits), summed in
+ * double.  wq_b maps the query latent (K = q_lora_rank = 1536) to the
+ * H_I * D_I = 64 * 128 index-query columns; the key projection and
+ * weights_proj map the hidden state (K = hidden_size = 7168) to the D_I = 128
+ * key columns and the H_I = 64 head weights.  Parity: pinned against a BLAS
+ * matrix product and exact special cases (tests/test_oracle_pins.py).
+ */
+void orc_linear(int64_t M, int N, int K, const void *x, int x_dtype, const void *w, int w_dtype, double *y)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int k = 0; k < K; ++k)
+                acc += orc_load(x, x_dtype, m * K + k) * orc_load(w, w_dtype, (int64_t)n * K + k);
+            y[m * N + n] = acc;
+        }
     }
 }
 

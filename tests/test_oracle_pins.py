@@ -533,3 +533,46 @@ def test_cache_append_then_score_equals_scoring_the_full_keys():
     cf, sf, _ = oracle.hadamard_quant(k_full)
     np.testing.assert_array_equal(c8, cf)
     np.testing.assert_array_equal(s8, sf)
+
+
+# -------------------------------------------------------------- projections --
+
+def test_linear_matches_blas_on_bf16_inputs():
+    """Y = X W^T: the oracle's loop sum against a BLAS matrix product of the
+    exactly widened bf16 values, on the wq_b inner size (q_lora_rank 1536)
+    and the hidden size (7168)."""
+    g = torch.Generator().manual_seed(3)
+    for K, N in ((1536, 96), (7168, 40)):
+        x = torch.randn(13, K, generator=g) / math.sqrt(K)
+        w = torch.randn(N, K, generator=g)
+        xb, wb = _bf16_bits(x), _bf16_bits(w)
+        xf = x.to(torch.bfloat16).double().numpy()
+        wf = w.to(torch.bfloat16).double().numpy()
+        np.testing.assert_allclose(oracle.linear(xb, wb), xf @ wf.T, rtol=1e-12, atol=1e-12)
+
+
+def test_linear_one_hot_rows_select_columns_and_orientation():
+    """A one-hot row n of W (1 at column c_n) makes output column n equal to
+    input column c_n exactly; a transposed operand or swapped index fails."""
+    g = np.random.default_rng(4)
+    M, K, N = 9, 64, 5
+    x = g.standard_normal((M, K)).astype(np.float32)
+    cols = [3, 0, 63, 17, 17]
+    w = np.zeros((N, K), dtype=np.float32)
+    for n, c in enumerate(cols):
+        w[n, c] = 1.0
+    y = oracle.linear(x, w)
+    for n, c in enumerate(cols):
+        np.testing.assert_array_equal(y[:, n], x[:, c].astype(np.float64))
+    # rows of X stay rows of Y: leading shape kept, rows independent
+    y3 = oracle.linear(x.reshape(3, 3, K), w)
+    np.testing.assert_array_equal(y3.reshape(M, N), y)
+
+
+def test_linear_is_linear_in_both_operands():
+    g = np.random.default_rng(5)
+    x1, x2 = g.standard_normal((2, 6, 32)).astype(np.float32)
+    w = g.standard_normal((7, 32)).astype(np.float32)
+    a = oracle.linear(x1, w) + oracle.linear(x2, w)
+    np.testing.assert_allclose(oracle.linear((x1 + x2).astype(np.float32), w), a, rtol=1e-6, atol=1e-5)
+    np.testing.assert_allclose(oracle.linear(x1, (-w).astype(np.float32)), -oracle.linear(x1, w), rtol=0, atol=0)
