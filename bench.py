@@ -58,12 +58,13 @@ class ClockSampler:
     def __init__(self, index):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        self.path = None
 
     def start(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
+            import tempfile
+            fd, self.path = tempfile.mkstemp(prefix=f"dsa_clocks_rank{self.index}_", suffix=".csv")
+            self.f = os.fdopen(fd, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
                                           "--format=csv,noheader,nounits", "-lms", "200"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
@@ -79,9 +80,12 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.f.close()
+        with open(self.path) as f:
+            lines = f.read().splitlines()
+        os.unlink(self.path)
         sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
+        for line in lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
@@ -186,11 +190,15 @@ def run_ours(args, wl):
     out = torch.empty(wl.batch, wl.n_q, wl.heads, wl.d_v, dtype=t["q"].dtype, device=dev)
     k_idx, k_scale, q_idx, q_scale = t["k_idx"], None, t["q_idx"], None
     q8 = qs = None
+    k_ref = None
     if wl.idx_fp8:
         k_idx, k_scale = dsa.hadamard_quant_fp8(t["k_idx"])   # the cache as stored (quantise-on-write)
         q8 = torch.empty(q_idx.shape, dtype=torch.uint8, device=dev)
         qs = torch.empty(q_idx.shape[:-1], dtype=torch.float32, device=dev)
-        del t["k_idx"]
+        if wl.idx_rescore > 0:
+            k_ref = t["k_idx"]       # the bf16 key cache kept beside the FP8 one for re-scoring
+        else:
+            del t["k_idx"]
 
     # prefill runs in rounds of `chunk` queries (positions shifted by the
     # round's first query); decode is a single round
@@ -204,7 +212,14 @@ def run_ours(args, wl):
         raise SystemExit("prefill rounds are cut per sequence: use batch 1")
     scores = torch.empty(wl.batch, chunk, ld, dtype=torch.float32, device=dev)
     idx = torch.empty(wl.batch, chunk, wl.topk, dtype=torch.int32, device=dev)
+    kc = wl.topk + wl.idx_rescore if (wl.idx_fp8 and wl.idx_rescore > 0) else 0
+    if kc:
+        # e4m3 indexer with re-scoring: the FP8 top-(k + margin) candidates, their bf16 scores
+        cand = torch.empty(wl.batch, chunk, kc, dtype=torch.int32, device=dev)
+        cand_sc = torch.empty(wl.batch, chunk, kc, dtype=torch.float32, device=dev)
     ws_topk = torch.empty(max(1, dsa.workspace_bytes(rounds[0][2], dsa.WS_TOPK)), dtype=torch.uint8, device=dev)
+    # the indexer -> top-k handoff (first-digit histograms from the indexer epilogue at decode)
+    hist = torch.empty(dsa.workspace_bytes(shape, dsa.WS_HIST), dtype=torch.uint8, device=dev)
     ws_attn = torch.empty(max(1, dsa.workspace_bytes(rounds[0][2], dsa.WS_ATTN)), dtype=torch.uint8, device=dev)
 
     def step(evr=None):
@@ -218,10 +233,19 @@ def run_ours(args, wl):
             ev = evr[ri] if evr is not None else None
             sl = slice(t0, t0 + c)
             if ev: ev[0].record(stream)
-            dsa.indexer_scores(sh, qi[:, sl], k_idx, t["w"][:, sl], t["ctx_len"], pos0, scores=scores[:, :c],
-                               q_scale=None if qsc is None else qsc[:, sl], k_scale=k_scale, stream=stream)
+            dsa.indexer_scores_hist(sh, qi[:, sl], k_idx, t["w"][:, sl], t["ctx_len"], pos0, hist,
+                                    scores=scores[:, :c], q_scale=None if qsc is None else qsc[:, sl],
+                                    k_scale=k_scale, stream=stream)
             if ev: ev[1].record(stream)
-            dsa.topk(sh, scores[:, :c], t["ctx_len"], pos0, idx=idx[:, :c], workspace=ws_topk, stream=stream)
+            if kc:
+                dsa.topk_hist(sh.replace(topk=kc), scores[:, :c], t["ctx_len"], pos0, hist, idx=cand[:, :c],
+                              stream=stream)
+                dsa.indexer_rescore(sh, q_idx[:, sl], k_ref, t["w"][:, sl], cand[:, :c], kc, t["ctx_len"], pos0,
+                                    scores=cand_sc[:, :c], stream=stream)
+                dsa.topk_candidates(sh, cand_sc[:, :c], cand[:, :c], kc, t["ctx_len"], pos0, idx=idx[:, :c],
+                                    stream=stream)
+            else:
+                dsa.topk_hist(sh, scores[:, :c], t["ctx_len"], pos0, hist, idx=idx[:, :c], stream=stream)
             if ev: ev[2].record(stream)
             dsa.sparse_mla_attn(sh, t["q"][:, sl], t["kv"], idx[:, :c], t["ctx_len"], out=out[:, sl],
                                 workspace=ws_attn, stream=stream)
@@ -266,7 +290,7 @@ def run_ours(args, wl):
 
     # end to end through the host-buffer entry point
     e2e = _e2e(args, wl, dsa, dsa.shape_from_workload(wl, q_chunk=chunk if len(rounds) > 1 else 0), t, k_idx,
-               k_scale, dev, stream)
+               k_scale, dev, stream, k_ref)
     e2e["ms"] = max_over_ranks(e2e["ms"], dev)
 
     res = None
@@ -307,18 +331,25 @@ def run_ours(args, wl):
                              else "latent cache fits L2 (9.4 MB at 8K); no flush between steps"},
             "stages_ms": stage_ms,
             "roofline": roof,
-            "gpu_launches": args.steps * (len(rounds) * (3 + _attn_extra_launches(wl, dsa, rounds[0][2]))
+            "roofline_bytes": ("indexer launch: index-key rows read + query block + head weights + fp32 score row "
+                               "written" if decode else "indexer launch: 2 * 64 * 128 flop per causal (query, key) pair"),
+            "gpu_launches": args.steps * (len(rounds) * (3 + (2 if kc else 0)
+                                                         + _attn_extra_launches(wl, dsa, rounds[0][2]))
                                           + (1 if wl.idx_fp8 else 0)),
             "clocks": clk,
             "e2e": {"value": q_total / (e2e["ms"] * 1e-3), "unit": "queries/s" if decode else "tokens/s",
-                    "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
+                    "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                    "ms_per_step": e2e["ms"],
+                    # this box's pinned copy rates: the step cannot run faster than its own copies
+                    "copy": e2e["copy"],
+                    "copy_bound_per_s": q_total / (max(e2e["copy"]["both_ms_per_step"], ms_per_step) * 1e-3)},
         }
     if ws > 1:
         torch.distributed.destroy_process_group()
     return res
 
 
-def _e2e(args, wl, dsa, shape, t, k_idx, k_scale, dev, stream):
+def _e2e(args, wl, dsa, shape, t, k_idx, k_scale, dev, stream, k_ref=None):
     """dsa_forward_host_async, one call a step: this step's queries copied in
     from pinned memory and the output copied back every step (the copy-back
     runs under the next step's indexer and top-k), caches resident on the
@@ -330,7 +361,8 @@ def _e2e(args, wl, dsa, shape, t, k_idx, k_scale, dev, stream):
     wsb = torch.empty(dsa.workspace_bytes(shape, dsa.WS_FORWARD_HOST), dtype=torch.uint8, device=dev)
     done = torch.cuda.Event()
     call = lambda: dsa.forward_host_async(shape, h["q_idx"], h["w"], h["q"], h["ctx_len"], h["q_pos0"], k_idx,
-                                          t["kv"], h_out, done=done, k_scale=k_scale, workspace=wsb, stream=stream)
+                                          t["kv"], h_out, done=done, k_scale=k_scale, workspace=wsb, stream=stream,
+                                          k_rescore=k_ref)
     for _ in range(max(1, args.warmup)):
         call()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -343,7 +375,50 @@ def _e2e(args, wl, dsa, shape, t, k_idx, k_scale, dev, stream):
     torch.cuda.synchronize(dev)
     h2d = sum(v.numel() * v.element_size() for v in h.values())
     d2h = h_out.numel() * h_out.element_size()
-    return {"ms": s.elapsed_time(e) / args.steps, "h2d": h2d, "d2h": d2h}
+    ms = s.elapsed_time(e) / args.steps
+    return {"ms": ms, "h2d": h2d, "d2h": d2h, "copy": _copy_rates(h["q"], h_out, dev)}
+
+
+def _copy_rates(h_in, h_out, dev, reps=10):
+    """Pinned host <-> device copy rates of this machine for the step's two largest
+    transfers (the attention queries in, the output back): each direction
+    alone, then both at once on two streams (as the asynchronous step
+    overlaps them)."""
+    d_in = torch.empty_like(h_in, device=dev)
+    d_out = torch.empty_like(h_out, device=dev)
+    s1, s2 = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    nb_in = h_in.numel() * h_in.element_size()
+    nb_out = h_out.numel() * h_out.element_size()
+
+    def timed(fn, stream):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / reps
+
+    with torch.cuda.stream(s1):
+        h2d_ms = timed(lambda: d_in.copy_(h_in, non_blocking=True), s1)
+        d2h_ms = timed(lambda: h_out.copy_(d_out, non_blocking=True), s1)
+    # both directions at once: the wall time of `reps` of each, overlapped
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    a.record(s1)
+    s2.wait_event(a)
+    for _ in range(reps):
+        with torch.cuda.stream(s1):
+            d_in.copy_(h_in, non_blocking=True)
+        with torch.cuda.stream(s2):
+            h_out.copy_(d_out, non_blocking=True)
+    s1.wait_stream(s2)
+    b.record(s1)
+    torch.cuda.synchronize(dev)
+    both_ms = a.elapsed_time(b) / reps
+    return {"h2d_gbs": nb_in / (h2d_ms * 1e-3) / 1e9, "d2h_gbs": nb_out / (d2h_ms * 1e-3) / 1e9,
+            "both_ms_per_step": both_ms}
 
 
 def _oracle_sample(wl, n_rows, seed=0):
@@ -551,6 +626,7 @@ def main():
     ap.add_argument("--workload", default="decode128k", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling runs)")
+    ap.add_argument("--ctx", type=int, default=0, help="override the workload's cache length (profiling runs)")
     ap.add_argument("--q-chunk", type=int, default=4096, help="prefill: queries per indexer/top-k/attention round")
     ap.add_argument("--op", default="step", choices=["step", "append", "topk"],
                     help="step: the layer step (default); append: the cache append of one prefill chunk; "
@@ -559,7 +635,14 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
-    wl = workloads.get(args.workload, **({"batch": args.batch} if args.batch else {}))
+    over = {}
+    if args.batch:
+        over["batch"] = args.batch
+    if args.ctx:
+        over["s_max"] = args.ctx
+        if workloads.get(args.workload).n_q > 1:
+            over["n_q"] = args.ctx
+    wl = workloads.get(args.workload, **over)
     if args.op in ("append", "topk") and args.impl == "ours":
         line = run_append(args) if args.op == "append" else run_topk_structures(args)
         if line is not None:

@@ -79,10 +79,14 @@ typedef struct {
     float sm_scale;     /* softmax scale of the attention logits (1/sqrt(192) for MLA) */
     int32_t q_chunk;    /* dsa_forward only: queries per sequence processed per round of
                            indexer -> top-k -> attention; 0 = all n_q at once */
+    int32_t idx_rescore;/* step with the E4M3 indexer only: > 0 keeps the top
+                           (topk + idx_rescore) keys of the FP8 scores, re-scores them
+                           from the BF16 key cache (dsa_indexer_rescore) and selects the
+                           final topk among them; 0 = select on the FP8 scores */
 } dsa_shape_t;
 
 /* Which workspace dsa_workspace_bytes() sizes. */
-enum { DSA_WS_TOPK = 0, DSA_WS_ATTN = 1, DSA_WS_FORWARD = 2, DSA_WS_FORWARD_HOST = 3 };
+enum { DSA_WS_TOPK = 0, DSA_WS_ATTN = 1, DSA_WS_FORWARD = 2, DSA_WS_FORWARD_HOST = 3, DSA_WS_HIST = 4 };
 
 /*
  * Lightning-indexer scores (section DSA, item 1; key cache paragraph).
@@ -129,6 +133,118 @@ dsa_status_t dsa_topk(const dsa_shape_t *shape,
                       int32_t *idx,
                       void *workspace, size_t workspace_bytes,
                       void *stream);
+
+/*
+ * The indexer's projections, which produce the step's indexer inputs
+ * (DeepSeek-V3.2 model doc: the note on the query LoRA path -- the indexer
+ * scores queries from the low-rank latent q_a_layernorm(q_a_proj(x)) through
+ * its `wq_b` projection, sized by q_lora_rank = 1536; section DeepseekV32Config
+ * -- index_n_heads 64, index_head_dim 128, hidden_size 7168; section "Usage
+ * example" -- weights_proj stays out of FP8).  Each is a plain linear map
+ * Y = X W^T on the tensor cores: bf16 operands, fp32 accumulation.
+ * Normalisations and rotary embeddings around them are the caller's.
+ *
+ * dsa_indexer_proj_q: q_idx[t, h, d] = sum_j q_latent[t, j] * wq_b[h * D_I + d, j]
+ *   q_latent [n_tokens][q_lora_rank] BF16, wq_b [H_I * D_I][q_lora_rank] BF16,
+ *   q_idx    [n_tokens][H_I][D_I] BF16 output (rounded to nearest even).
+ *   q_lora_rank a multiple of 64; H_I * D_I a multiple of 256 (or 64, 128, 192).
+ */
+dsa_status_t dsa_indexer_proj_q(const dsa_shape_t *shape, int32_t n_tokens, int32_t q_lora_rank,
+                                const void *q_latent, const void *wq_b, void *q_idx, void *stream);
+
+/*
+ * dsa_indexer_proj_kw: the single-head index key and the head weights of
+ * each token, from its hidden state, in one pass over x:
+ *   k_new[t, d] = sum_j x[t, j] * w_kw[d, j]          (d < D_I; BF16 out)
+ *   w[t, h]     = sum_j x[t, j] * w_kw[D_I + h, j]    (h < H_I; fp32 out)
+ *   x [n_tokens][hidden] BF16; w_kw [D_I + H_I][hidden] BF16: the key
+ *   projection's rows followed by weights_proj's rows.  hidden a multiple of
+ *   64; D_I + H_I in {64, 128, 192} or a multiple of 256, D_I a multiple of 32.
+ *   k_new feeds dsa_cache_append, w feeds the indexer (any constant factor of
+ *   the score goes into shape->idx_scale or into w_kw).
+ * All pointers 16-byte aligned.
+ */
+dsa_status_t dsa_indexer_proj_kw(const dsa_shape_t *shape, int32_t n_tokens, int32_t hidden,
+                                 const void *x, const void *w_kw, void *k_new, float *w, void *stream);
+
+/*
+ * The indexer -> top-k pair with a handoff (section DSA, items 1-2: the
+ * index score exists to feed the per-query top-index_topk selection).
+ * dsa_indexer_scores_hist computes exactly what dsa_indexer_scores computes
+ * and, where the indexer's schedule allows it (tensor-core indexer, one
+ * query per sequence, i.e. decode, on rows of at least a few thousand keys),
+ * its epilogue also counts the first 11-bit radix digit of every score into
+ * `hist`; dsa_topk_hist then selects exactly what dsa_topk selects, starting
+ * from those counts instead of a first pass over each score row.  Elsewhere
+ * the pair behaves as dsa_indexer_scores + dsa_topk (hist unused).
+ * Arguments as in those two calls, plus
+ *   hist  device buffer of dsa_workspace_bytes(shape, DSA_WS_HIST) bytes,
+ *         16-byte aligned, opaque; written by the indexer call, read by the
+ *         top-k call.  The two calls must be made with the same shape on the
+ *         same device, with the top-k reading the scores the indexer call
+ *         wrote, and nothing else writing `hist` in between.
+ */
+dsa_status_t dsa_indexer_scores_hist(const dsa_shape_t *shape,
+                                     const void *q_idx, const float *q_scale,
+                                     const void *k_idx, const float *k_scale,
+                                     const float *w,
+                                     const int32_t *ctx_len, const int32_t *q_pos0,
+                                     float *scores, int64_t ld_scores,
+                                     void *hist, size_t hist_bytes,
+                                     void *stream);
+dsa_status_t dsa_topk_hist(const dsa_shape_t *shape,
+                           const float *scores, int64_t ld_scores,
+                           const int32_t *ctx_len, const int32_t *q_pos0,
+                           const void *hist, size_t hist_bytes,
+                           int32_t *idx, void *stream);
+
+/*
+ * Selection among listed candidates (section DSA, item 2, applied to a
+ * candidate list): for each query, the min(topk, n) entries of
+ * cand[b,t,0:n] with the largest cand_scores, n = min(n_cand, pos+1,
+ * ctx_len[b]) -- the first n entries are the candidates.  The candidates
+ * are key indices in ascending order (as dsa_topk writes them), so "ties go
+ * to the lower index" is "ties go to the earlier entry".
+ * Arguments
+ *   cand_scores [B][n_q][cand_ld] fp32, finite for the n listed entries;
+ *   cand        [B][n_q][cand_ld] int32 ascending key indices;
+ *   cand_ld >= n_cand, a multiple of 4.
+ *   idx         [B][n_q][topk] int32 output: the kept key indices (values of
+ *               cand), ascending, then -1 padding.
+ * The E4M3 step uses it after dsa_indexer_rescore.  No workspace.
+ */
+dsa_status_t dsa_topk_candidates(const dsa_shape_t *shape,
+                                 const float *cand_scores, const int32_t *cand,
+                                 int64_t cand_ld, int32_t n_cand,
+                                 const int32_t *ctx_len, const int32_t *q_pos0,
+                                 int32_t *idx, void *stream);
+
+/*
+ * Index scores of listed keys from BF16 rows (section DSA, item 1: the
+ * reference indexer runs in FP8 after the Hadamard rotation, and FP8 is only
+ * a precision optimisation of this same score).  For each query and each of
+ * its first n = min(n_cand, pos+1, ctx_len[b]) listed keys s = cand[b,t,j]:
+ *   scores[b,t,j] = sum_h w[b,t,h] * max(0, idx_scale * <q_idx[b,t,h,:], k_idx[b,s,:]>)
+ * computed as dsa_indexer_scores computes it for BF16 inputs (tensor cores,
+ * fp32 accumulation).  Used by the E4M3 step (shape->idx_rescore > 0) to
+ * re-score the FP8 indexer's top (topk + idx_rescore) keys before the final
+ * selection, so that the selection matches the BF16 indexer's.
+ * Arguments
+ *   q_idx [B][n_q][H_I][D_I] BF16 and k_idx [B][s_max][D_I] BF16, whatever
+ *         shape->idx_dtype says; 16-byte aligned.  D_I = 128,
+ *         H_I in {16, 32, 64, 128}.
+ *   w     [B][n_q][H_I] fp32;  ctx_len, q_pos0 [B] int32.
+ *   cand  [B][n_q][cand_ld] int32: listed key indices, each in [0, ctx_len[b])
+ *         (an entry outside is scored as an all-zero key and sets
+ *         DSA_ERR_BAD_INDEX in the device error word).
+ *   scores [B][n_q][ld_scores] fp32 output, entries j < n written;
+ *         cand_ld, ld_scores >= n_cand.
+ */
+dsa_status_t dsa_indexer_rescore(const dsa_shape_t *shape,
+                                 const void *q_idx, const void *k_idx, const float *w,
+                                 const int32_t *cand, int64_t cand_ld, int32_t n_cand,
+                                 const int32_t *ctx_len, const int32_t *q_pos0,
+                                 float *scores, int64_t ld_scores, void *stream);
 
 /*
  * Attention over the selected keys only (section DSA, item 2).  For head h
@@ -206,13 +322,19 @@ dsa_status_t dsa_cache_append(const dsa_shape_t *shape, int32_t n_new,
  * the workspace).  Inputs as in the calls above, except with
  * idx_dtype == E4M3: q_idx is BF16 [B][n_q][H_I][D_I] and is rotated and
  * quantised inside the step (q_scale must be NULL), while k_idx/k_scale are
- * the FP8 key cache as written by dsa_hadamard_quant_fp8.
+ * the FP8 key cache as written by dsa_hadamard_quant_fp8 (or dsa_cache_append).
+ *   k_rescore  E4M3 with shape->idx_rescore > 0: the BF16 key cache
+ *              [B][s_max][D_I] (the same keys before rotation and
+ *              quantisation), from which the FP8 indexer's top
+ *              (topk + idx_rescore) candidates are re-scored before the final
+ *              top-k; otherwise NULL.
  *   idx_out [B][n_q][topk] int32 or NULL: the selected indices.
  *   workspace: dsa_workspace_bytes(shape, DSA_WS_FORWARD) bytes.
  */
 dsa_status_t dsa_forward(const dsa_shape_t *shape,
                          const void *q_idx, const float *q_scale,
                          const void *k_idx, const float *k_scale,
+                         const void *k_rescore,
                          const float *w,
                          const void *q, const void *kv, const void *v,
                          const int32_t *ctx_len, const int32_t *q_pos0,
@@ -224,7 +346,7 @@ dsa_status_t dsa_forward(const dsa_shape_t *shape,
  * dsa_forward with the per-step tensors in HOST memory: q_idx, w, q,
  * ctx_len, q_pos0 (inputs) and out, lse (outputs; lse may be NULL) are HOST
  * pointers (page-locked memory gives asynchronous copies), while the caches
- * k_idx, k_scale, kv, v stay on the device as the layer's resident state.
+ * k_idx, k_scale, k_rescore, kv, v stay on the device as the layer's resident state.
  * The call copies the inputs in (one cudaMemcpyAsync each), runs the step,
  * copies the outputs back and synchronises `stream` before returning.
  * workspace: dsa_workspace_bytes(shape, DSA_WS_FORWARD_HOST) bytes: the
@@ -239,7 +361,7 @@ dsa_status_t dsa_forward(const dsa_shape_t *shape,
 dsa_status_t dsa_forward_host(const dsa_shape_t *shape,
                               const void *h_q_idx, const float *h_w, const void *h_q,
                               const int32_t *h_ctx_len, const int32_t *h_q_pos0,
-                              const void *k_idx, const float *k_scale,
+                              const void *k_idx, const float *k_scale, const void *k_rescore,
                               const void *kv, const void *v,
                               void *h_out, float *h_lse,
                               void *workspace, size_t workspace_bytes,
@@ -267,14 +389,16 @@ dsa_status_t dsa_forward_host(const dsa_shape_t *shape,
  *     not be read, until done_event has completed (or the device has been
  *     synchronised).
  *   - Errors: argument errors return before anything is enqueued; device
- *     errors are read with dsa_get_error.  Calls on one device are
- *     serialised by the caller (the library's streams and events are per
- *     device).
+ *     errors are read with dsa_get_error.
+ *   - Threads: host-buffer calls (either form) may come from several host
+ *     threads; the library's staging slots, streams and events are per
+ *     device, and a per-device lock makes each call's enqueue atomic, so
+ *     concurrent calls run one after the other in the order they take it.
  */
 dsa_status_t dsa_forward_host_async(const dsa_shape_t *shape,
                                     const void *h_q_idx, const float *h_w, const void *h_q,
                                     const int32_t *h_ctx_len, const int32_t *h_q_pos0,
-                                    const void *k_idx, const float *k_scale,
+                                    const void *k_idx, const float *k_scale, const void *k_rescore,
                                     const void *kv, const void *v,
                                     void *h_out, float *h_lse,
                                     void *workspace, size_t workspace_bytes,
@@ -315,6 +439,14 @@ size_t dsa_workspace_bytes(const dsa_shape_t *shape, int32_t which);
  * device.  Synchronises the device.  Returns DSA_OK, DSA_ERR_TIMEOUT or
  * DSA_ERR_BAD_INDEX (the first recorded kind), or DSA_ERR_CUDA if the read
  * itself failed.  `detail`, if not NULL, receives the raw word.
+ * Sharing: the word lives in the library's own device memory, one per
+ * device, not in a caller's workspace -- several entry points that can
+ * record an error (dsa_indexer_scores, dsa_cache_append,
+ * dsa_sparse_mla_attn_static) take no workspace.  So every caller and every
+ * stream on a device records into the same word (bits are OR-ed, nothing is
+ * lost), and a clear by one caller also clears what another caller's kernels
+ * recorded: a program with several independent users of one device should
+ * read with clear = 0 and clear at an agreed point.
  */
 dsa_status_t dsa_get_error(int32_t clear, uint32_t *detail);
 

@@ -33,9 +33,15 @@ bool ensure_device(int dev) {
   std::lock_guard<std::mutex> lock(g_mutex);
   if (g_sm_count[dev] > 0 && g_err_ptr[dev] != nullptr) return true;
   int sms = 0;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) return false;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+    (void)cudaGetLastError();  // consumed here, so it is not reported against a later call
+    return false;
+  }
   void* p = nullptr;
-  if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess || p == nullptr) return false;
+  if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess || p == nullptr) {
+    (void)cudaGetLastError();
+    return false;
+  }
   g_sm_count[dev] = sms;
   g_err_ptr[dev] = static_cast<uint32_t*>(p);
   return true;
@@ -60,7 +66,8 @@ dsa_status_t check_shape(const dsa_shape_t* s) {
     return DSA_ERR_INVALID_ARG;
   if (!(s->idx_scale > 0.f) || !std::isfinite(s->idx_scale)) return DSA_ERR_INVALID_ARG;
   if (!std::isfinite(s->sm_scale)) return DSA_ERR_INVALID_ARG;
-  if (s->q_chunk < 0) return DSA_ERR_INVALID_ARG;
+  if (s->q_chunk < 0 || s->idx_rescore < 0) return DSA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(s->topk) + s->idx_rescore > INT32_MAX / 4) return DSA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(s->batch) * s->s_max > INT32_MAX) return DSA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(s->batch) * s->n_q * s->idx_heads > INT32_MAX) return DSA_ERR_UNSUPPORTED;
   return DSA_OK;
@@ -70,8 +77,9 @@ dsa_status_t check_shape(const dsa_shape_t* s) {
 dsa_status_t run_indexer(const dsa_shape_t* s, int dev, cudaStream_t st, int B, int n_q, int t_off,
                          const void* q_idx, const float* q_scale, const void* k_idx, const float* k_scale,
                          const float* w, const int32_t* ctx_len, const int32_t* q_pos0, float* scores,
-                         int64_t ld) {
+                         int64_t ld, uint32_t* hist_parts = nullptr) {
   IndexerArgs a;
+  a.hist_parts = hist_parts;
   a.device = dev;
   a.stream = st;
   a.B = B;
@@ -97,16 +105,24 @@ dsa_status_t run_indexer(const dsa_shape_t* s, int dev, cudaStream_t st, int B, 
   return indexer_tc(a);
 }
 
-dsa_status_t run_topk(const dsa_shape_t* s, int dev, cudaStream_t st, int B, int n_q, int t_off, const float* scores,
+// Top-k of rows of `row_len` scores (the cache length, or the candidate list
+// length when `remap` maps list slots to key indices).
+dsa_status_t run_topk(int dev, cudaStream_t st, int B, int n_q, int t_off, int row_len, int k, const float* scores,
                       int64_t ld, const int32_t* ctx_len, const int32_t* q_pos0, int32_t* idx, void* ws,
-                      size_t ws_bytes) {
+                      size_t ws_bytes, const int32_t* remap = nullptr, int64_t remap_ld = 0,
+                      const uint32_t* hist_parts = nullptr, int hist_per_cta = 0, int hist_tpr = 0) {
   TopkArgs a;
+  a.hist_parts = hist_parts;
+  a.hist_per_cta = hist_per_cta;
+  a.hist_tpr = hist_tpr;
   a.device = dev;
   a.stream = st;
   a.B = B;
   a.n_q = n_q;
-  a.s_max = s->s_max;
-  a.k = s->topk;
+  a.s_max = row_len;
+  a.k = k;
+  a.remap = remap;
+  a.remap_ld = remap_ld;
   a.scores = scores;
   a.ld = ld;
   a.ctx_len = ctx_len;
@@ -118,6 +134,48 @@ dsa_status_t run_topk(const dsa_shape_t* s, int dev, cudaStream_t st, int B, int
   a.err = g_err_ptr[dev];
   if (B == 0 || n_q == 0) return DSA_OK;
   return topk_radix(a);
+}
+
+dsa_status_t run_rescore(const dsa_shape_t* s, int dev, cudaStream_t st, int B, int n_q, int t_off,
+                         const void* q_idx, const void* k_idx, const float* w, const int32_t* cand, int64_t cand_ld,
+                         int n_cand, const int32_t* ctx_len, const int32_t* q_pos0, float* out, int64_t out_ld) {
+  RescoreArgs a;
+  a.device = dev;
+  a.stream = st;
+  a.B = B;
+  a.n_q = n_q;
+  a.s_max = s->s_max;
+  a.H = s->idx_heads;
+  a.D = s->idx_dim;
+  a.n_cand = n_cand;
+  a.t_off = t_off;
+  a.q_idx = q_idx;
+  a.k_idx = k_idx;
+  a.w = w;
+  a.cand = cand;
+  a.cand_ld = cand_ld;
+  a.ctx_len = ctx_len;
+  a.q_pos0 = q_pos0;
+  a.out = out;
+  a.out_ld = out_ld;
+  a.idx_scale = s->idx_scale;
+  a.err = g_err_ptr[dev];
+  if (B == 0 || n_q == 0 || n_cand == 0) return DSA_OK;
+  return indexer_rescore(a);
+}
+
+// The indexer -> top-k histogram handoff for a call over B x n_q queries:
+// whether the indexer's schedule emits it (tensor-core indexer, one query per
+// sequence, runs spanning at most two rows), and its run length and tiles per row.
+struct HistPlan {
+  bool on = false;
+  int per_cta = 0, tpr = 0;
+};
+HistPlan hist_plan(const dsa_shape_t* s, int dev, int B, int n_q) {
+  HistPlan h;
+  if (s->idx_dtype == DSA_F32 || !indexer_tc_supported(s->idx_heads, s->idx_dim)) return h;
+  h.on = indexer_hist_plan(B, n_q, s->s_max, device_sm_count(dev), &h.per_cta, &h.tpr);
+  return h;
 }
 
 dsa_status_t run_attn(const dsa_shape_t* s, int dev, cudaStream_t st, int B, int n_q, const void* q, const void* kv,
@@ -155,7 +213,8 @@ dsa_status_t run_attn(const dsa_shape_t* s, int dev, cudaStream_t st, int B, int
 struct FwdLayout {
   int chunk;          // queries per sequence per round
   int64_t ld;         // score row stride
-  size_t off_scores, off_idx, off_q8, off_qs, off_topk, off_attn;
+  int kc;             // E4M3 with re-scoring: candidates per query (topk + idx_rescore), else 0
+  size_t off_scores, off_idx, off_q8, off_qs, off_topk, off_attn, off_cand, off_rs, off_hist;
   size_t topk_bytes, attn_bytes;
   size_t total;
   // host-variant staging: two input slots (consecutive calls alternate, so a
@@ -184,6 +243,13 @@ FwdLayout forward_layout(const dsa_shape_t* s) {
     L.off_qs = off;
     off = align_up(off + static_cast<size_t>(B) * s->n_q * s->idx_heads * 4, 256);
   }
+  L.kc = (s->idx_dtype == DSA_E4M3 && s->idx_rescore > 0) ? s->topk + s->idx_rescore : 0;
+  L.off_cand = off;
+  off = align_up(off + static_cast<size_t>(B) * L.chunk * L.kc * 4, 256);
+  L.off_rs = off;
+  off = align_up(off + static_cast<size_t>(B) * L.chunk * L.kc * 4, 256);
+  L.off_hist = off;
+  if (L.chunk == 1) off = align_up(off + kHistPartsBytes, 256);
   L.off_topk = off;
   L.topk_bytes = topk_workspace_bytes(B, L.chunk, s->s_max, s->topk);
   off = align_up(off + L.topk_bytes, 256);
@@ -271,6 +337,10 @@ cudaEvent_t g_ev_free[kMaxDevices][2] = {}, g_ev_in[kMaxDevices] = {}, g_ev_q[kM
 cudaEvent_t g_ev_attn[kMaxDevices] = {}, g_ev_out[kMaxDevices] = {}, g_ev_join[kMaxDevices] = {};
 int g_slot[kMaxDevices] = {};
 const void* g_last_ws[kMaxDevices] = {};
+// Held by a host-buffer call from its slot choice to its last event record,
+// so that calls from several host threads on one device cannot take the same
+// staging slot or interleave their event records.
+std::mutex g_host_mutex[kMaxDevices];
 bool ensure_copy_stream(int dev) {
   std::lock_guard<std::mutex> lock(g_mutex);
   if (g_copy_stream[dev] != nullptr) return true;
@@ -353,8 +423,120 @@ dsa_status_t dsa_topk(const dsa_shape_t* shape, const float* scores, int64_t ld_
   const size_t need = topk_workspace_bytes(shape->batch, shape->n_q, shape->s_max, shape->topk);
   if (workspace_bytes < need || (need > 0 && workspace == nullptr)) return DSA_ERR_WORKSPACE;
   DSA_SETUP(dev);
-  return run_topk(shape, dev, static_cast<cudaStream_t>(stream), shape->batch, shape->n_q, 0, scores, ld_scores,
-                  ctx_len, q_pos0, idx, workspace, workspace_bytes);
+  return run_topk(dev, static_cast<cudaStream_t>(stream), shape->batch, shape->n_q, 0, shape->s_max, shape->topk,
+                  scores, ld_scores, ctx_len, q_pos0, idx, workspace, workspace_bytes);
+}
+
+dsa_status_t dsa_indexer_proj_q(const dsa_shape_t* shape, int32_t n_tokens, int32_t q_lora_rank,
+                                const void* q_latent, const void* wq_b, void* q_idx, void* stream) {
+  dsa_status_t st = check_shape(shape);
+  if (st != DSA_OK) return st;
+  if (n_tokens < 0 || q_lora_rank <= 0) return DSA_ERR_INVALID_ARG;
+  if (n_tokens > 0 && (!q_latent || !wq_b || !q_idx)) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_latent) || !aligned16(wq_b) || !aligned16(q_idx)) return DSA_ERR_INVALID_ARG;
+  const int N = shape->idx_heads * shape->idx_dim;
+  if (!proj_gemm_supported(N, q_lora_rank, N)) return DSA_ERR_UNSUPPORTED;
+  DSA_SETUP(dev);
+  GemmArgs a;
+  a.device = dev;
+  a.stream = static_cast<cudaStream_t>(stream);
+  a.M = n_tokens;
+  a.N = N;
+  a.K = q_lora_rank;
+  a.n_split = N;
+  a.x = q_latent;
+  a.w = wq_b;
+  a.out0 = q_idx;
+  a.ld0 = N;
+  a.out1 = nullptr;
+  a.ld1 = 0;
+  a.err = g_err_ptr[dev];
+  return proj_gemm(a);
+}
+
+dsa_status_t dsa_indexer_proj_kw(const dsa_shape_t* shape, int32_t n_tokens, int32_t hidden, const void* x,
+                                 const void* w_kw, void* k_new, float* w, void* stream) {
+  dsa_status_t st = check_shape(shape);
+  if (st != DSA_OK) return st;
+  if (n_tokens < 0 || hidden <= 0) return DSA_ERR_INVALID_ARG;
+  if (n_tokens > 0 && (!x || !w_kw || !k_new || !w)) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_kw) || !aligned16(k_new) || !aligned16(w)) return DSA_ERR_INVALID_ARG;
+  const int D = shape->idx_dim, HI = shape->idx_heads;
+  if ((HI & 3) != 0 || (D & 7) != 0) return DSA_ERR_UNSUPPORTED;
+  if (!proj_gemm_supported(D + HI, hidden, D)) return DSA_ERR_UNSUPPORTED;
+  DSA_SETUP(dev);
+  GemmArgs a;
+  a.device = dev;
+  a.stream = static_cast<cudaStream_t>(stream);
+  a.M = n_tokens;
+  a.N = D + HI;
+  a.K = hidden;
+  a.n_split = D;
+  a.x = x;
+  a.w = w_kw;
+  a.out0 = k_new;
+  a.ld0 = D;
+  a.out1 = w;
+  a.ld1 = HI;
+  a.err = g_err_ptr[dev];
+  return proj_gemm(a);
+}
+
+dsa_status_t dsa_indexer_scores_hist(const dsa_shape_t* shape, const void* q_idx, const float* q_scale,
+                                     const void* k_idx, const float* k_scale, const float* w,
+                                     const int32_t* ctx_len, const int32_t* q_pos0, float* scores,
+                                     int64_t ld_scores, void* hist, size_t hist_bytes, void* stream) {
+  dsa_status_t st = check_shape(shape);
+  if (st != DSA_OK) return st;
+  st = check_indexer_inputs(shape, q_idx, q_scale, k_idx, k_scale, w, ctx_len, q_pos0);
+  if (st != DSA_OK) return st;
+  if (!scores || ld_scores < shape->s_max || (ld_scores & 3) != 0 || !aligned16(scores)) return DSA_ERR_INVALID_ARG;
+  if (hist == nullptr || hist_bytes < kHistPartsBytes || !aligned16(hist)) return DSA_ERR_WORKSPACE;
+  DSA_SETUP(dev);
+  const HistPlan hp = hist_plan(shape, dev, shape->batch, shape->n_q);
+  return run_indexer(shape, dev, static_cast<cudaStream_t>(stream), shape->batch, shape->n_q, 0, q_idx, q_scale,
+                     k_idx, k_scale, w, ctx_len, q_pos0, scores, ld_scores,
+                     hp.on ? static_cast<uint32_t*>(hist) : nullptr);
+}
+
+dsa_status_t dsa_topk_hist(const dsa_shape_t* shape, const float* scores, int64_t ld_scores, const int32_t* ctx_len,
+                           const int32_t* q_pos0, const void* hist, size_t hist_bytes, int32_t* idx, void* stream) {
+  dsa_status_t st = check_shape(shape);
+  if (st != DSA_OK) return st;
+  if (!scores || !ctx_len || !q_pos0 || !idx) return DSA_ERR_INVALID_ARG;
+  if (ld_scores < shape->s_max || (ld_scores & 3) != 0 || !aligned16(scores)) return DSA_ERR_INVALID_ARG;
+  if (hist == nullptr || hist_bytes < kHistPartsBytes) return DSA_ERR_WORKSPACE;
+  DSA_SETUP(dev);
+  const HistPlan hp = hist_plan(shape, dev, shape->batch, shape->n_q);
+  return run_topk(dev, static_cast<cudaStream_t>(stream), shape->batch, shape->n_q, 0, shape->s_max, shape->topk,
+                  scores, ld_scores, ctx_len, q_pos0, idx, nullptr, 0, nullptr, 0,
+                  hp.on ? static_cast<const uint32_t*>(hist) : nullptr, hp.per_cta, hp.tpr);
+}
+
+dsa_status_t dsa_topk_candidates(const dsa_shape_t* shape, const float* cand_scores, const int32_t* cand,
+                                 int64_t cand_ld, int32_t n_cand, const int32_t* ctx_len, const int32_t* q_pos0,
+                                 int32_t* idx, void* stream) {
+  dsa_status_t st = check_shape(shape);
+  if (st != DSA_OK) return st;
+  if (!cand_scores || !cand || !ctx_len || !q_pos0 || !idx) return DSA_ERR_INVALID_ARG;
+  if (n_cand < 0 || cand_ld < n_cand || (cand_ld & 3) != 0 || !aligned16(cand_scores)) return DSA_ERR_INVALID_ARG;
+  DSA_SETUP(dev);
+  return run_topk(dev, static_cast<cudaStream_t>(stream), shape->batch, shape->n_q, 0, n_cand, shape->topk,
+                  cand_scores, cand_ld, ctx_len, q_pos0, idx, nullptr, 0, cand, cand_ld);
+}
+
+dsa_status_t dsa_indexer_rescore(const dsa_shape_t* shape, const void* q_idx, const void* k_idx, const float* w,
+                                 const int32_t* cand, int64_t cand_ld, int32_t n_cand, const int32_t* ctx_len,
+                                 const int32_t* q_pos0, float* scores, int64_t ld_scores, void* stream) {
+  dsa_status_t st = check_shape(shape);
+  if (st != DSA_OK) return st;
+  if (!q_idx || !k_idx || !w || !cand || !ctx_len || !q_pos0 || !scores) return DSA_ERR_INVALID_ARG;
+  if (n_cand < 0 || cand_ld < n_cand || ld_scores < n_cand) return DSA_ERR_INVALID_ARG;
+  if (!aligned16(q_idx) || !aligned16(k_idx)) return DSA_ERR_INVALID_ARG;
+  if (!indexer_rescore_supported(shape->idx_heads, shape->idx_dim)) return DSA_ERR_UNSUPPORTED;
+  DSA_SETUP(dev);
+  return run_rescore(shape, dev, static_cast<cudaStream_t>(stream), shape->batch, shape->n_q, 0, q_idx, k_idx, w,
+                     cand, cand_ld, n_cand, ctx_len, q_pos0, scores, ld_scores);
 }
 
 dsa_status_t dsa_sparse_mla_attn(const dsa_shape_t* shape, const void* q, const void* kv, const void* v,
@@ -437,16 +619,73 @@ size_t dsa_workspace_bytes(const dsa_shape_t* shape, int32_t which) {
       return forward_layout(shape).total;
     case DSA_WS_FORWARD_HOST:
       return forward_layout(shape).total_host;
+    case DSA_WS_HIST:
+      return kHistPartsBytes;
     default:
       return 0;
   }
 }
 
+// One round of the step over B_ sequences x c queries (pointers already at
+// the round's first query; t_off shifts the query positions): indexer
+// scores, top-k (the e4m3 indexer with re-scoring: FP8 top-(k + margin)
+// candidates, their bf16 scores, then the top-k among them), attention.
+struct RoundIn {
+  const void* qi;      // indexer queries as the indexer reads them (e4m3 codes or bf16/fp32)
+  const float* qsc;    // e4m3 query scales (or null)
+  const void* q_ref;   // bf16 queries for re-scoring (or null)
+  const void* k_idx;
+  const float* k_scale;
+  const void* k_ref;   // bf16 key cache for re-scoring (or null)
+  const float* w;
+  const void* q;
+  const void* kv;
+  const void* v;
+  const int32_t* ctx_len;
+  const int32_t* q_pos0;
+  void* out;
+  float* lse;
+  int32_t* idx;
+};
+
+static dsa_status_t forward_round(const dsa_shape_t* s, int dev, cudaStream_t st, int B_, int c, int t_off,
+                                  const RoundIn& in, uint8_t* ws, const FwdLayout& L, cudaEvent_t q_ready,
+                                  cudaEvent_t out_free) {
+  float* scores = reinterpret_cast<float*>(ws + L.off_scores);
+  // decode: the indexer's epilogue also counts the first radix digit of each
+  // score row, so the top-k starts from the threshold bin
+  const HistPlan hp = (L.chunk == 1) ? hist_plan(s, dev, B_, c) : HistPlan{};
+  uint32_t* hist = hp.on ? reinterpret_cast<uint32_t*>(ws + L.off_hist) : nullptr;
+  dsa_status_t rc = run_indexer(s, dev, st, B_, c, t_off, in.qi, in.qsc, in.k_idx, in.k_scale, in.w, in.ctx_len,
+                                in.q_pos0, scores, L.ld, hist);
+  if (rc != DSA_OK) return rc;
+  if (L.kc > 0) {
+    int32_t* cand = reinterpret_cast<int32_t*>(ws + L.off_cand);
+    float* rs = reinterpret_cast<float*>(ws + L.off_rs);
+    rc = run_topk(dev, st, B_, c, t_off, s->s_max, L.kc, scores, L.ld, in.ctx_len, in.q_pos0, cand,
+                  ws + L.off_topk, L.topk_bytes, nullptr, 0, hist, hp.per_cta, hp.tpr);
+    if (rc != DSA_OK) return rc;
+    rc = run_rescore(s, dev, st, B_, c, t_off, in.q_ref, in.k_ref, in.w, cand, L.kc, L.kc, in.ctx_len, in.q_pos0,
+                     rs, L.kc);
+    if (rc != DSA_OK) return rc;
+    rc = run_topk(dev, st, B_, c, t_off, L.kc, s->topk, rs, L.kc, in.ctx_len, in.q_pos0, in.idx, ws + L.off_topk,
+                  L.topk_bytes, cand, L.kc);
+  } else {
+    rc = run_topk(dev, st, B_, c, t_off, s->s_max, s->topk, scores, L.ld, in.ctx_len, in.q_pos0, in.idx,
+                  ws + L.off_topk, L.topk_bytes, nullptr, 0, hist, hp.per_cta, hp.tpr);
+  }
+  if (rc != DSA_OK) return rc;
+  if (q_ready != nullptr && cudaStreamWaitEvent(st, q_ready, 0) != cudaSuccess) return DSA_ERR_CUDA;
+  if (out_free != nullptr && cudaStreamWaitEvent(st, out_free, 0) != cudaSuccess) return DSA_ERR_CUDA;
+  return run_attn(s, dev, st, B_, c, in.q, in.kv, in.v, in.idx, in.ctx_len, in.out, in.lse, ws + L.off_attn,
+                  L.attn_bytes);
+}
+
 static dsa_status_t forward_impl(const dsa_shape_t* s, int dev, cudaStream_t st, const void* q_idx,
-                                 const float* q_scale, const void* k_idx, const float* k_scale, const float* w,
-                                 const void* q, const void* kv, const void* v, const int32_t* ctx_len,
-                                 const int32_t* q_pos0, void* out, float* lse, int32_t* idx_out, uint8_t* ws,
-                                 const FwdLayout& L, cudaEvent_t q_ready = nullptr,
+                                 const float* q_scale, const void* k_idx, const float* k_scale, const void* k_ref,
+                                 const float* w, const void* q, const void* kv, const void* v,
+                                 const int32_t* ctx_len, const int32_t* q_pos0, void* out, float* lse,
+                                 int32_t* idx_out, uint8_t* ws, const FwdLayout& L, cudaEvent_t q_ready = nullptr,
                                  cudaEvent_t out_free = nullptr) {
   const int B = s->batch, n_q = s->n_q;
   if (B == 0 || n_q == 0) return DSA_OK;
@@ -454,7 +693,6 @@ static dsa_status_t forward_impl(const dsa_shape_t* s, int dev, cudaStream_t st,
   // FP8 indexer: rotate + quantise this step's queries
   const void* qi = q_idx;
   const float* qsc = q_scale;
-  dsa_shape_t si = *s;
   if (s->idx_dtype == DSA_E4M3) {
     rc = hadamard_quant(q_idx, DSA_BF16, static_cast<int64_t>(B) * n_q * s->idx_heads, s->idx_dim, ws + L.off_q8,
                         reinterpret_cast<float*>(ws + L.off_qs), st);
@@ -462,48 +700,39 @@ static dsa_status_t forward_impl(const dsa_shape_t* s, int dev, cudaStream_t st,
     qi = ws + L.off_q8;
     qsc = reinterpret_cast<float*>(ws + L.off_qs);
   }
-  float* scores = reinterpret_cast<float*>(ws + L.off_scores);
   const size_t ei = elem_size(s->idx_dtype);
   const size_t ea = elem_size(s->attn_dtype);
+  RoundIn in;
   if (L.chunk == n_q) {
-    int32_t* idx = idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + L.off_idx);
-    rc = run_indexer(&si, dev, st, B, n_q, 0, qi, qsc, k_idx, k_scale, w, ctx_len, q_pos0, scores, L.ld);
-    if (rc != DSA_OK) return rc;
-    rc = run_topk(&si, dev, st, B, n_q, 0, scores, L.ld, ctx_len, q_pos0, idx, ws + L.off_topk, L.topk_bytes);
-    if (rc != DSA_OK) return rc;
-    if (q_ready != nullptr && cudaStreamWaitEvent(st, q_ready, 0) != cudaSuccess) return DSA_ERR_CUDA;
-    if (out_free != nullptr && cudaStreamWaitEvent(st, out_free, 0) != cudaSuccess) return DSA_ERR_CUDA;
-    return run_attn(&si, dev, st, B, n_q, q, kv, v, idx, ctx_len, out, lse, ws + L.off_attn, L.attn_bytes);
+    in = {qi, qsc, q_idx, k_idx, k_scale, k_ref, w, q, kv, v, ctx_len, q_pos0, out, lse,
+          idx_out ? idx_out : reinterpret_cast<int32_t*>(ws + L.off_idx)};
+    return forward_round(s, dev, st, B, n_q, 0, in, ws, L, q_ready, out_free);
   }
   // Rounds of `chunk` queries, one sequence at a time (positions shift by t0).
+  const int64_t qrow = static_cast<int64_t>(s->idx_heads) * s->idx_dim;
   for (int b = 0; b < B; ++b) {
     for (int t0 = 0; t0 < n_q; t0 += L.chunk) {
       const int c = std::min(L.chunk, n_q - t0);
       const int64_t row0 = static_cast<int64_t>(b) * n_q + t0;
-      const uint8_t* qi_b = static_cast<const uint8_t*>(qi) + row0 * s->idx_heads * s->idx_dim * ei;
-      const float* qs_b = qsc ? qsc + row0 * s->idx_heads : nullptr;
-      const uint8_t* k_b = static_cast<const uint8_t*>(k_idx) + static_cast<int64_t>(b) * s->s_max * s->idx_dim * ei;
-      const float* ks_b = k_scale ? k_scale + static_cast<int64_t>(b) * s->s_max : nullptr;
-      const float* w_b = w + row0 * s->idx_heads;
-      int32_t* idx_b = idx_out ? idx_out + row0 * s->topk : reinterpret_cast<int32_t*>(ws + L.off_idx);
-      const uint8_t* q_b = static_cast<const uint8_t*>(q) + row0 * s->heads * s->d_qk * ea;
-      const uint8_t* kv_b =
-          static_cast<const uint8_t*>(kv) + static_cast<int64_t>(b) * s->s_max * s->kv_heads * s->d_qk * ea;
-      const uint8_t* v_b =
-          v ? static_cast<const uint8_t*>(v) + static_cast<int64_t>(b) * s->s_max * s->kv_heads * s->d_v * ea : nullptr;
-      uint8_t* out_b = static_cast<uint8_t*>(out) + row0 * s->heads * s->d_v * ea;
-      float* lse_b = lse ? lse + row0 * s->heads : nullptr;
-      rc = run_indexer(&si, dev, st, 1, c, t0, qi_b, qs_b, k_b, ks_b, w_b, ctx_len + b, q_pos0 + b, scores, L.ld);
-      if (rc != DSA_OK) return rc;
-      rc = run_topk(&si, dev, st, 1, c, t0, scores, L.ld, ctx_len + b, q_pos0 + b, idx_b, ws + L.off_topk,
-                    L.topk_bytes);
-      if (rc != DSA_OK) return rc;
-      if (b == 0 && t0 == 0) {
-        if (q_ready != nullptr && cudaStreamWaitEvent(st, q_ready, 0) != cudaSuccess) return DSA_ERR_CUDA;
-        if (out_free != nullptr && cudaStreamWaitEvent(st, out_free, 0) != cudaSuccess) return DSA_ERR_CUDA;
-      }
-      rc = run_attn(&si, dev, st, 1, c, q_b, kv_b, v_b, idx_b, ctx_len + b, out_b, lse_b, ws + L.off_attn,
-                    L.attn_bytes);
+      in.qi = static_cast<const uint8_t*>(qi) + row0 * qrow * ei;
+      in.qsc = qsc ? qsc + row0 * s->idx_heads : nullptr;
+      in.q_ref = static_cast<const uint8_t*>(q_idx) + row0 * qrow * 2;
+      in.k_idx = static_cast<const uint8_t*>(k_idx) + static_cast<int64_t>(b) * s->s_max * s->idx_dim * ei;
+      in.k_scale = k_scale ? k_scale + static_cast<int64_t>(b) * s->s_max : nullptr;
+      in.k_ref = k_ref ? static_cast<const uint8_t*>(k_ref) + static_cast<int64_t>(b) * s->s_max * s->idx_dim * 2
+                       : nullptr;
+      in.w = w + row0 * s->idx_heads;
+      in.q = static_cast<const uint8_t*>(q) + row0 * s->heads * s->d_qk * ea;
+      in.kv = static_cast<const uint8_t*>(kv) + static_cast<int64_t>(b) * s->s_max * s->kv_heads * s->d_qk * ea;
+      in.v = v ? static_cast<const uint8_t*>(v) + static_cast<int64_t>(b) * s->s_max * s->kv_heads * s->d_v * ea
+               : nullptr;
+      in.ctx_len = ctx_len + b;
+      in.q_pos0 = q_pos0 + b;
+      in.out = static_cast<uint8_t*>(out) + row0 * s->heads * s->d_v * ea;
+      in.lse = lse ? lse + row0 * s->heads : nullptr;
+      in.idx = idx_out ? idx_out + row0 * s->topk : reinterpret_cast<int32_t*>(ws + L.off_idx);
+      const bool first = (b == 0 && t0 == 0);
+      rc = forward_round(s, dev, st, 1, c, t0, in, ws, L, first ? q_ready : nullptr, first ? out_free : nullptr);
       if (rc != DSA_OK) return rc;
     }
   }
@@ -511,20 +740,29 @@ static dsa_status_t forward_impl(const dsa_shape_t* s, int dev, cudaStream_t st,
 }
 
 static dsa_status_t check_forward(const dsa_shape_t* shape, const void* q_idx, const float* q_scale,
-                                  const void* k_idx, const float* k_scale, const float* w, const void* q,
-                                  const void* kv, const void* v, const int32_t* ctx_len, const int32_t* q_pos0,
-                                  const void* out, bool on_host) {
+                                  const void* k_idx, const float* k_scale, const void* k_ref, const float* w,
+                                  const void* q, const void* kv, const void* v, const int32_t* ctx_len,
+                                  const int32_t* q_pos0, const void* out, bool on_host) {
   dsa_status_t st = check_shape(shape);
   if (st != DSA_OK) return st;
   if (shape->idx_dtype == DSA_E4M3) {
     if (q_scale != nullptr || !k_scale || !q_idx || !k_idx || !w || !ctx_len || !q_pos0) return DSA_ERR_INVALID_ARG;
     if (!aligned16(k_idx) || (!on_host && !aligned16(q_idx))) return DSA_ERR_INVALID_ARG;
     if (!indexer_tc_supported(shape->idx_heads, shape->idx_dim)) return DSA_ERR_UNSUPPORTED;
-  } else if (!on_host) {
-    st = check_indexer_inputs(shape, q_idx, q_scale, k_idx, k_scale, w, ctx_len, q_pos0);
-    if (st != DSA_OK) return st;
+    if (shape->idx_rescore > 0) {
+      if (!k_ref || !aligned16(k_ref)) return DSA_ERR_INVALID_ARG;
+      if (!indexer_rescore_supported(shape->idx_heads, shape->idx_dim)) return DSA_ERR_UNSUPPORTED;
+    } else if (k_ref != nullptr) {
+      return DSA_ERR_INVALID_ARG;
+    }
   } else {
-    if (!q_idx || !k_idx || !w || !ctx_len || !q_pos0) return DSA_ERR_INVALID_ARG;
+    if (k_ref != nullptr) return DSA_ERR_INVALID_ARG;
+    if (!on_host) {
+      st = check_indexer_inputs(shape, q_idx, q_scale, k_idx, k_scale, w, ctx_len, q_pos0);
+      if (st != DSA_OK) return st;
+    } else if (!q_idx || !k_idx || !w || !ctx_len || !q_pos0) {
+      return DSA_ERR_INVALID_ARG;
+    }
   }
   if (!q || !kv || !out) return DSA_ERR_INVALID_ARG;
   if (!on_host) {
@@ -535,16 +773,17 @@ static dsa_status_t check_forward(const dsa_shape_t* shape, const void* q_idx, c
 }
 
 dsa_status_t dsa_forward(const dsa_shape_t* shape, const void* q_idx, const float* q_scale, const void* k_idx,
-                         const float* k_scale, const float* w, const void* q, const void* kv, const void* v,
-                         const int32_t* ctx_len, const int32_t* q_pos0, void* out, float* lse, int32_t* idx_out,
-                         void* workspace, size_t workspace_bytes, void* stream) {
-  dsa_status_t st = check_forward(shape, q_idx, q_scale, k_idx, k_scale, w, q, kv, v, ctx_len, q_pos0, out, false);
+                         const float* k_scale, const void* k_rescore, const float* w, const void* q, const void* kv,
+                         const void* v, const int32_t* ctx_len, const int32_t* q_pos0, void* out, float* lse,
+                         int32_t* idx_out, void* workspace, size_t workspace_bytes, void* stream) {
+  dsa_status_t st = check_forward(shape, q_idx, q_scale, k_idx, k_scale, k_rescore, w, q, kv, v, ctx_len, q_pos0,
+                                  out, false);
   if (st != DSA_OK) return st;
   const FwdLayout L = forward_layout(shape);
   if (workspace == nullptr || workspace_bytes < L.total || !aligned16(workspace)) return DSA_ERR_WORKSPACE;
   DSA_SETUP(dev);
-  return forward_impl(shape, dev, static_cast<cudaStream_t>(stream), q_idx, q_scale, k_idx, k_scale, w, q, kv, v,
-                      ctx_len, q_pos0, out, lse, idx_out, static_cast<uint8_t*>(workspace), L);
+  return forward_impl(shape, dev, static_cast<cudaStream_t>(stream), q_idx, q_scale, k_idx, k_scale, k_rescore, w, q,
+                      kv, v, ctx_len, q_pos0, out, lse, idx_out, static_cast<uint8_t*>(workspace), L);
 }
 
 // The step with host-memory inputs and outputs.  Synchronous: the output is
@@ -555,11 +794,12 @@ dsa_status_t dsa_forward(const dsa_shape_t* shape, const void* q_idx, const floa
 // for the copy before it rewrites the device output.
 static dsa_status_t forward_host_impl(const dsa_shape_t* shape, const void* h_q_idx, const float* h_w,
                                       const void* h_q, const int32_t* h_ctx_len, const int32_t* h_q_pos0,
-                                      const void* k_idx, const float* k_scale, const void* kv, const void* v,
+                                      const void* k_idx, const float* k_scale, const void* k_rescore,
+                                      const void* kv, const void* v,
                                       void* h_out, float* h_lse, void* workspace, size_t workspace_bytes,
                                       void* stream, bool async, cudaEvent_t done) {
-  dsa_status_t st = check_forward(shape, h_q_idx, nullptr, k_idx, k_scale, h_w, h_q, kv, v, h_ctx_len, h_q_pos0,
-                                  h_out, true);
+  dsa_status_t st = check_forward(shape, h_q_idx, nullptr, k_idx, k_scale, k_rescore, h_w, h_q, kv, v, h_ctx_len,
+                                  h_q_pos0, h_out, true);
   if (st != DSA_OK) return st;
   const FwdLayout L = forward_layout(shape);
   if (workspace == nullptr || workspace_bytes < L.total_host || !aligned16(workspace)) return DSA_ERR_WORKSPACE;
@@ -580,6 +820,7 @@ static dsa_status_t forward_host_impl(const dsa_shape_t* shape, const void* h_q_
   // (the bulk of the input: waited for just before attention, so that they
   // land under the indexer and top-k)
   if (!ensure_copy_stream(dev)) return DSA_ERR_CUDA;
+  std::lock_guard<std::mutex> host_lock(g_host_mutex[dev]);
   const cudaStream_t xs = g_copy_stream[dev];
   const int slot = g_slot[dev];
   g_slot[dev] ^= 1;
@@ -601,7 +842,8 @@ static dsa_status_t forward_host_impl(const dsa_shape_t* shape, const void* h_q_
       cudaEventRecord(g_ev_q[dev], xs) != cudaSuccess || cudaStreamWaitEvent(cs, g_ev_in[dev], 0) != cudaSuccess)
     return DSA_ERR_CUDA;
   dsa_shape_t s2 = *shape;
-  st = forward_impl(&s2, dev, cs, in + L.off_h_qidx, nullptr, k_idx, k_scale, reinterpret_cast<float*>(in + L.off_h_w),
+  st = forward_impl(&s2, dev, cs, in + L.off_h_qidx, nullptr, k_idx, k_scale, k_rescore,
+                    reinterpret_cast<float*>(in + L.off_h_w),
                     in + L.off_h_q, kv, v, reinterpret_cast<int32_t*>(in + L.off_h_ctx),
                     reinterpret_cast<int32_t*>(in + L.off_h_pos), ws + L.off_h_out,
                     h_lse ? reinterpret_cast<float*>(ws + L.off_h_lse) : nullptr, nullptr, ws, L, g_ev_q[dev],
@@ -629,18 +871,20 @@ static dsa_status_t forward_host_impl(const dsa_shape_t* shape, const void* h_q_
 
 dsa_status_t dsa_forward_host(const dsa_shape_t* shape, const void* h_q_idx, const float* h_w, const void* h_q,
                               const int32_t* h_ctx_len, const int32_t* h_q_pos0, const void* k_idx,
-                              const float* k_scale, const void* kv, const void* v, void* h_out, float* h_lse,
-                              void* workspace, size_t workspace_bytes, void* stream) {
-  return forward_host_impl(shape, h_q_idx, h_w, h_q, h_ctx_len, h_q_pos0, k_idx, k_scale, kv, v, h_out, h_lse,
+                              const float* k_scale, const void* k_rescore, const void* kv, const void* v,
+                              void* h_out, float* h_lse, void* workspace, size_t workspace_bytes, void* stream) {
+  return forward_host_impl(shape, h_q_idx, h_w, h_q, h_ctx_len, h_q_pos0, k_idx, k_scale, k_rescore, kv, v, h_out,
+                           h_lse,
                            workspace, workspace_bytes, stream, false, nullptr);
 }
 
 dsa_status_t dsa_forward_host_async(const dsa_shape_t* shape, const void* h_q_idx, const float* h_w,
                                     const void* h_q, const int32_t* h_ctx_len, const int32_t* h_q_pos0,
-                                    const void* k_idx, const float* k_scale, const void* kv, const void* v,
-                                    void* h_out, float* h_lse, void* workspace, size_t workspace_bytes,
-                                    void* done_event, void* stream) {
-  return forward_host_impl(shape, h_q_idx, h_w, h_q, h_ctx_len, h_q_pos0, k_idx, k_scale, kv, v, h_out, h_lse,
+                                    const void* k_idx, const float* k_scale, const void* k_rescore, const void* kv,
+                                    const void* v, void* h_out, float* h_lse, void* workspace,
+                                    size_t workspace_bytes, void* done_event, void* stream) {
+  return forward_host_impl(shape, h_q_idx, h_w, h_q, h_ctx_len, h_q_pos0, k_idx, k_scale, k_rescore, kv, v, h_out,
+                           h_lse,
                            workspace, workspace_bytes, stream, true, static_cast<cudaEvent_t>(done_event));
 }
 
@@ -711,7 +955,10 @@ void* static_attn_scratch(int dev) {
   std::lock_guard<std::mutex> lock(g_static_mutex);
   if (g_static_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_attn_scratch) != cudaSuccess) return nullptr;
+    if (cudaGetSymbolAddress(&p, g_attn_scratch) != cudaSuccess) {
+      (void)cudaGetLastError();  // consumed here, so it is not reported against a later call
+      return nullptr;
+    }
     g_static_scratch_ptr[dev] = p;
   }
   return g_static_scratch_ptr[dev];

@@ -38,7 +38,20 @@ struct IndexerArgs {
   int64_t ld;
   float idx_scale;
   uint32_t* err;
+  // Optional (one-query schedule only, see indexer_hist_plan): each CTA also
+  // writes the first 11-bit digit histograms of the (at most two) score rows
+  // its run of key tiles covers, [cta][2][2048] (second row's zero if none).
+  uint32_t* hist_parts = nullptr;
 };
+
+// Largest grid for which the indexer writes score histograms.
+constexpr int kMaxHistCtas = 256;
+// Bytes of the histogram handoff between the indexer and the top-k.
+constexpr size_t kHistPartsBytes = static_cast<size_t>(kMaxHistCtas) * 2 * 2048 * 4;
+// Whether the indexer's one-query schedule for (B, n_q, s_max) on num_sms SMs
+// can emit score histograms (every CTA's run spans at most two rows); if so,
+// the run length (tiles per CTA) and the key tiles per row.
+bool indexer_hist_plan(int B, int n_q, int s_max, int num_sms, int* per_cta, int* tpr);
 
 struct TopkArgs {
   int device;
@@ -53,6 +66,15 @@ struct TopkArgs {
   void* ws;
   size_t ws_bytes;
   uint32_t* err;
+  // Optional: output index = remap[row * remap_ld + s] instead of s (a
+  // selection among a candidate list whose entries are ascending indices).
+  const int32_t* remap = nullptr;
+  int64_t remap_ld = 0;
+  // Optional: the indexer's partial first-digit histograms (IndexerArgs::
+  // hist_parts, written with runs of hist_per_cta tiles, hist_tpr tiles a
+  // row), summed per row instead of reading the row for them.
+  const uint32_t* hist_parts = nullptr;
+  int hist_per_cta = 0, hist_tpr = 0;
 };
 
 // Cache append (csrc/cache_append.cu): token (b, i) -> cache row pos[b] + i.
@@ -96,6 +118,46 @@ struct AttnArgs {
   size_t ws_bytes;
   uint32_t* err;
 };
+
+// Exact bf16 scores of listed candidate keys (csrc/indexer_rescore.cu).
+struct RescoreArgs {
+  int device;
+  cudaStream_t stream;
+  int B, n_q, s_max, H, D;
+  int n_cand;               // entries listed per row (the first min(n_cand, pos + 1) are read)
+  int t_off;
+  const void* q_idx;        // [B][n_q][H][D] bf16
+  const void* k_idx;        // [B][s_max][D] bf16
+  const float* w;           // [B][n_q][H]
+  const int32_t* cand;      // [B][n_q][cand_ld]
+  int64_t cand_ld;
+  const int32_t* ctx_len;
+  const int32_t* q_pos0;
+  float* out;               // [B][n_q][out_ld]
+  int64_t out_ld;
+  float idx_scale;
+  uint32_t* err;
+};
+dsa_status_t indexer_rescore(const RescoreArgs& a);
+bool indexer_rescore_supported(int H, int D);
+
+// Y = X W^T on the tensor cores (csrc/proj_gemm.cu): X [M][K], W [N][K]
+// bf16 row-major; columns [0, n_split) of Y go to out0 (bf16, row stride
+// ld0), columns [n_split, N) to out1 (fp32, row stride ld1).
+struct GemmArgs {
+  int device;
+  cudaStream_t stream;
+  int M, N, K, n_split;
+  const void* x;
+  const void* w;
+  void* out0;
+  int64_t ld0;
+  float* out1;
+  int64_t ld1;
+  uint32_t* err;
+};
+dsa_status_t proj_gemm(const GemmArgs& a);
+bool proj_gemm_supported(int N, int K, int n_split);
 
 dsa_status_t indexer_tc(const IndexerArgs& a);    // BF16 / E4M3, tensor cores
 dsa_status_t indexer_simt(const IndexerArgs& a);  // F32, CUDA cores

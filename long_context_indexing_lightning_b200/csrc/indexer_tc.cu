@@ -33,8 +33,9 @@ namespace {
 
 constexpr int kTileKeys = 128;  // MMA M
 constexpr int kIdxDim = 128;    // D_I
+constexpr int kHistBins = 2048; // first 11-bit digit of the order-preserving score key
 
-template <bool kFP8, int kQG, int kHI, int kEpiWarps, int kStages, int kQBufs>
+template <bool kFP8, int kQG, int kHI, int kEpiWarps, int kStages, int kQBufs, bool kHist>
 struct IdxCfg {
   static constexpr int N = kQG * kHI;
   static constexpr int kElem = kFP8 ? 1 : 2;
@@ -54,7 +55,11 @@ struct IdxCfg {
   static constexpr int kOffBar = kOffW + 2 * kQG * kHI * 4;  // two weight buffers
   static constexpr int kNumBars = 2 * kStages + 2 * kQBufs + 2 * kNumAcc + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+  // first-digit histograms of the (at most two) score rows the CTA writes
+  static constexpr int kOffHist = kOffMisc + 16;
+  static constexpr int kHistWords = kHist ? 2 * kHistBins : 0;
+  static constexpr int kSmemBytes = kOffHist + kHistWords * 4 + 1024;  // + alignment slack
+  static_assert(!kHist || kQG == 1, "score histograms are built in the one-query (decode) schedule");
   static_assert(N % 16 == 0 && N >= 16 && N <= 256, "MMA N");
   static_assert(kHI % 16 == 0, "heads per query");
   // 8 epilogue warps: two groups of four split the query block (kQG even),
@@ -135,14 +140,14 @@ __device__ __forceinline__ bool iter_next(const Sched& S, UnitIter& it, int cta,
   return true;
 }
 
-template <bool kFP8, int kQG, int kHI, int kEpiWarps, int kStages, int kQBufs>
-__global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQBufs>::kThreads, 1)
+template <bool kFP8, int kQG, int kHI, int kEpiWarps, int kStages, int kQBufs, bool kHist>
+__global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQBufs, kHist>::kThreads, 1)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_q,
                       const float* __restrict__ w, const float* __restrict__ q_scale,
                       const float* __restrict__ k_scale, const int32_t* __restrict__ ctx_len,
                       const int32_t* __restrict__ q_pos0, float* __restrict__ scores, int64_t ld,
-                      float idx_scale, Sched S, uint32_t* err) {
-  using C = IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQBufs>;
+                      float idx_scale, Sched S, uint32_t* err, uint32_t* __restrict__ hist_out) {
+  using C = IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQBufs, kHist>;
   pdl_wait();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -169,6 +174,10 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
+  }
+  uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + C::kOffHist);
+  if constexpr (kHist) {
+    for (int i = threadIdx.x; i < C::kHistWords; i += C::kThreads) hist_s[i] = 0u;
   }
   if (warp == 1) {
     tmem_alloc(smem_addr(tmem_slot), C::kTmemCols);
@@ -300,9 +309,12 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
     int last_bg = -1;
     float wreg[kQG == 1 ? kHI : 1];
     UnitIter it = iter_begin(S, cta);
+    // histogram slot of a score row: 0 for the first row of this CTA's run, 1 for the next
+    const int first_bg = S.tpr > 0 ? it.i / S.tpr : 0;
     Unit U;
     while (iter_next<kQG>(S, it, cta, U, ctx_len, q_pos0)) {
       if (U.kt_end <= U.kt0) continue;
+      uint32_t* hslot = hist_s + ((U.b * S.G + U.t0 / kQG) == first_bg ? 0 : kHistBins);
       if (kQG == 1 && U.kt_comp > U.kt0) {
         // one query: its head weights live in registers
         const int bg = U.b * S.G + U.t0;
@@ -382,8 +394,11 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
           }
           if (s < U.L) {
             const int p = U.p0 + U.t0;
-            scores[(static_cast<int64_t>(U.b) * S.n_q + U.t0) * ld + s] =
-                (s <= p) ? ((acc0 + acc1) + (acc2 + acc3)) * ks : -INFINITY;
+            const float v = ((acc0 + acc1) + (acc2 + acc3)) * ks;
+            scores[(static_cast<int64_t>(U.b) * S.n_q + U.t0) * ld + s] = (s <= p) ? v : -INFINITY;
+            if constexpr (kHist) {
+              if (s <= p) atomicAdd(&hslot[float_order_key(v) >> 21], 1u);
+            }
           }
         } else
 #pragma unroll 1
@@ -403,7 +418,11 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
           }
           if (j < U.nq && s < U.L) {
             const int p = U.p0 + U.t0 + j;
-            scores[(static_cast<int64_t>(U.b) * S.n_q + U.t0 + j) * ld + s] = (s <= p) ? (acc0 + acc1) * ks : -INFINITY;
+            const float v = (acc0 + acc1) * ks;
+            scores[(static_cast<int64_t>(U.b) * S.n_q + U.t0 + j) * ld + s] = (s <= p) ? v : -INFINITY;
+            if constexpr (kHist) {
+              if (s <= p) atomicAdd(&hslot[float_order_key(v) >> 21], 1u);
+            }
           }
         }
         tc_fence_before_sync();
@@ -420,6 +439,13 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
             scores[(static_cast<int64_t>(U.b) * S.n_q + U.t0 + j) * ld + s] = -INFINITY;
       }
     }
+    if constexpr (kHist) {
+      // this CTA's partial first-digit histograms of its first and second
+      // score rows (zeros where it wrote none): the top-k sums them
+      named_bar_sync(2, C::kEpiThreads);
+      uint32_t* dst = hist_out + static_cast<int64_t>(cta) * C::kHistWords;
+      for (int i = tid_e; i < C::kHistWords; i += C::kEpiThreads) dst[i] = hist_s[i];
+    }
   }
 
   pdl_trigger();
@@ -431,10 +457,10 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
   }
 }
 
-template <bool kFP8, int kQG, int kHI, int kEpiWarps, int kStages, int kQBufs>
+template <bool kFP8, int kQG, int kHI, int kEpiWarps, int kStages, int kQBufs, bool kHist>
 dsa_status_t launch_indexer_tc(const IndexerArgs& a) {
-  using C = IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQBufs>;
-  auto kern = indexer_tc_kernel<kFP8, kQG, kHI, kEpiWarps, kStages, kQBufs>;
+  using C = IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQBufs, kHist>;
+  auto kern = indexer_tc_kernel<kFP8, kQG, kHI, kEpiWarps, kStages, kQBufs, kHist>;
   const int dev = a.device;
   const int num_sms = device_sm_count(dev);
 
@@ -485,23 +511,44 @@ dsa_status_t launch_indexer_tc(const IndexerArgs& a) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tmk, tmq, a.w, a.q_scale, a.k_scale, a.ctx_len, a.q_pos0,
-                                           a.scores, a.ld, a.idx_scale, S, a.err);
+                                           a.scores, a.ld, a.idx_scale, S, a.err, a.hist_parts);
   return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 }  // namespace
+
+bool indexer_hist_plan(int B, int n_q, int s_max, int num_sms, int* per_cta, int* tpr) {
+  // the decode schedule: one query per tile, each CTA a contiguous run of
+  // key tiles; histograms only when a run spans at most two score rows
+  if (n_q != 1 || B <= 0 || s_max <= 0 || num_sms <= 0 || num_sms > kMaxHistCtas) return false;
+  const int64_t t = (s_max + kTileKeys - 1) / kTileKeys;
+  const int64_t total = static_cast<int64_t>(B) * t;
+  const int64_t grid = std::min<int64_t>(total, num_sms);
+  const int64_t pc = (total + grid - 1) / grid;
+  if (pc > t || total > INT32_MAX / 2) return false;
+  *per_cta = static_cast<int>(pc);
+  *tpr = static_cast<int>(t);
+  return true;
+}
 
 dsa_status_t indexer_tc(const IndexerArgs& a) {
   // decode (n_q == 1): one query per tile; prefill: a block of queries filling N.
   const bool fp8 = (a.dtype == DSA_E4M3);
   if (a.D != kIdxDim) return DSA_ERR_UNSUPPORTED;
   const bool one = (a.n_q == 1);
-#define DSA_IDX_CASE(HI, QGP)                                                              \
-  if (a.H == HI) {                                                                         \
-    if (one) return fp8 ? launch_indexer_tc<true, 1, HI, 8, 12, 2>(a)                       \
-                        : launch_indexer_tc<false, 1, HI, 4, 5, 2>(a);                     \
-    return fp8 ? launch_indexer_tc<true, QGP, HI, ((QGP) % 2 == 0 ? 8 : 4), 6, 1>(a)       \
-               : launch_indexer_tc<false, QGP, HI, ((QGP) % 2 == 0 ? 8 : 4), 4, 1>(a);     \
+  const bool hist = a.hist_parts != nullptr;
+  if (hist) {
+    int pc = 0, tp = 0;
+    if (!indexer_hist_plan(a.B, a.n_q, a.s_max, device_sm_count(a.device), &pc, &tp)) return DSA_ERR_UNSUPPORTED;
+  }
+#define DSA_IDX_CASE(HI, QGP)                                                                  \
+  if (a.H == HI) {                                                                             \
+    if (one && hist) return fp8 ? launch_indexer_tc<true, 1, HI, 8, 12, 2, true>(a)             \
+                                : launch_indexer_tc<false, 1, HI, 4, 5, 2, true>(a);           \
+    if (one) return fp8 ? launch_indexer_tc<true, 1, HI, 8, 12, 2, false>(a)                    \
+                        : launch_indexer_tc<false, 1, HI, 4, 5, 2, false>(a);                  \
+    return fp8 ? launch_indexer_tc<true, QGP, HI, ((QGP) % 2 == 0 ? 8 : 4), 6, 1, false>(a)    \
+               : launch_indexer_tc<false, QGP, HI, ((QGP) % 2 == 0 ? 8 : 4), 4, 1, false>(a);  \
   }
   DSA_IDX_CASE(64, 4)
   DSA_IDX_CASE(32, 8)

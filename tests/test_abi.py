@@ -75,10 +75,25 @@ def test_argument_errors_need_no_gpu(L):
     assert L.dsa_cache_append(ctypes.byref(s.replace(d_qk=575)), 1, 16, 16, None, 16, 16, None, 16, None, None) == 2
     assert L.dsa_cache_append(ctypes.byref(s), 1, 18, 16, None, 16, 16, None, 16, None, None) == 1
     # host-buffer step, asynchronous form: null inputs, a workspace too small
-    assert L.dsa_forward_host_async(ctypes.byref(s), None, None, None, None, None, 16, None, 16, None, 16, None,
-                                    16, 1 << 30, None, None) == 1
-    assert L.dsa_forward_host_async(ctypes.byref(s), 16, 16, 16, 16, 16, 16, None, 16, None, 16, None,
+    assert L.dsa_forward_host_async(ctypes.byref(s), None, None, None, None, None, 16, None, None, 16, None, 16,
+                                    None, 16, 1 << 30, None, None) == 1
+    assert L.dsa_forward_host_async(ctypes.byref(s), 16, 16, 16, 16, 16, 16, None, None, 16, None, 16, None,
                                     16, 16, None, None) == 3
+    # e4m3 step with re-scoring: the bf16 key cache is required, and only then
+    e4r = e4.replace(idx_rescore=1024)
+    assert L.dsa_forward(ctypes.byref(e4r), 16, None, 16, 16, None, 16, 16, 16, None, 16, 16, 16, None, None,
+                         16, 1 << 30, None) == 1
+    assert L.dsa_forward(ctypes.byref(s), 16, None, 16, None, 16, 16, 16, 16, None, 16, 16, 16, None, None,
+                         16, 1 << 30, None) == 1
+    assert L.dsa_forward(ctypes.byref(s.replace(idx_rescore=-1)), 16, None, 16, None, None, 16, 16, 16, None, 16,
+                         16, 16, None, None, 16, 1 << 30, None) == 1
+    # re-scoring and candidate selection: null lists, lists shorter than n_cand
+    assert L.dsa_indexer_rescore(ctypes.byref(s), 16, 16, 16, None, 1024, 1024, 16, 16, 16, 1024, None) == 1
+    assert L.dsa_indexer_rescore(ctypes.byref(s), 16, 16, 16, 16, 1000, 1024, 16, 16, 16, 1024, None) == 1
+    assert L.dsa_indexer_rescore(ctypes.byref(s.replace(idx_heads=48)), 16, 16, 16, 16, 1024, 1024, 16, 16, 16,
+                                 1024, None) == 2
+    assert L.dsa_topk_candidates(ctypes.byref(s), 16, None, 1024, 1024, 16, 16, 16, None) == 1
+    assert L.dsa_topk_candidates(ctypes.byref(s), 16, 16, 1022, 1022, 16, 16, 16, None) == 1
 
 
 def test_workspace_arithmetic(L):
@@ -93,3 +108,7 @@ def test_workspace_arithmetic(L):
     assert dsa.workspace_bytes(p, dsa.WS_FORWARD) < 4096 * 65536 * 4 * 1.2
     full = p.replace(q_chunk=0)
     assert dsa.workspace_bytes(full, dsa.WS_FORWARD) >= 65536 * 65536 * 4
+    # e4m3 with re-scoring adds the candidate lists and their bf16 scores
+    e4 = s.replace(idx_dtype=dsa.DSA_E4M3)
+    e4r = e4.replace(idx_rescore=1024)
+    assert dsa.workspace_bytes(e4r, dsa.WS_FORWARD) >= dsa.workspace_bytes(e4, dsa.WS_FORWARD) + 2 * 32 * 3072 * 4

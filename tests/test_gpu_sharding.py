@@ -9,12 +9,16 @@ the attention tolerance (the split-K layout of the attention may differ with
 the number of rows), and one rank's append-then-score must equal scoring its
 rows on the filled caches.
 """
+import numpy as np
 import pytest
 import torch
 
 import long_context_indexing_lightning_b200 as dsa
+import oracle
 import workloads
 from long_context_indexing_lightning_b200 import build, sharding
+
+from _parity import check_idx_valid, check_topk_near_ties
 
 pytestmark = pytest.mark.gpu
 
@@ -54,6 +58,21 @@ def test_balanced_row_ranges_reproduce_the_unsplit_prefill():
     torch.testing.assert_close(torch.cat(idxs, 1), idx_full, rtol=0, atol=0)
     assert (torch.cat(outs, 1).float() - full.float()).abs().max().item() <= ATTN_ATOL_BF16
     assert dsa.get_error()[0] == 0
+    # and the split run against the oracle, on rows of every rank's range
+    # (each range's first and last row, and one inside)
+    H = workloads.to_numpy
+    h = {k: H(v) for k, v in t.items()}
+    picks = sorted({r for r0, r1 in ranges for r in (r0, (r0 + r1) // 2, r1 - 1)})
+    rows = [(0, r) for r in picks]
+    o_sc = oracle.indexer_scores(h["q_idx"], h["k_idx"], h["w"], h["ctx_len"], h["q_pos0"], rows=rows)
+    pos = np.array(picks, dtype=np.int32)
+    o_idx = oracle.topk(np.where(np.isfinite(o_sc), o_sc, -np.inf).astype(np.float32), pos, wl.topk)
+    g_idx = torch.cat(idxs, 1)[0, picks].cpu().numpy()
+    check_idx_valid(g_idx, pos, wl.topk)
+    check_topk_near_ties(g_idx, o_idx, o_sc, wl.topk)
+    o = oracle.sparse_attn(h["q"], h["kv"], o_idx, wl.sm_scale, v=wl.d_v, rows=rows)
+    got = torch.cat(outs, 1)[0, picks].float().cpu().numpy().astype(np.float64)
+    assert np.abs(got - o).max() <= ATTN_ATOL_BF16
 
 
 def test_prefill_rank_appends_then_scores_its_rows():

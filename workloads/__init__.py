@@ -41,6 +41,7 @@ class Workload:
     idx_scale: float = 1.0
     decode: bool = False  # query sits at ctx_len-1 (its own key is already cached)
     idx_fp8: bool = False
+    idx_rescore: int = 0  # e4m3 indexer: extra FP8 candidates re-scored from the bf16 keys
     ctx_len: tuple = field(default=None)  # per-sequence lengths; None = all s_max
 
     def lengths(self):
@@ -67,7 +68,7 @@ WORKLOADS = {
     "prefill64k": Workload("prefill64k", batch=1, n_q=65536, s_max=65536, **_MLA),
     "decode128k": Workload("decode128k", batch=32, n_q=1, s_max=131072, decode=True, **_MLA),
     "decode128k_fp8": Workload("decode128k_fp8", batch=32, n_q=1, s_max=131072, decode=True,
-                               idx_fp8=True, **_MLA),
+                               idx_fp8=True, idx_rescore=1024, **_MLA),
 }
 
 
