@@ -92,7 +92,6 @@ struct AttnParams {
   float* part_o;            // [R][S][2][128][256] (splits > 1)
   float* part_ml;           // [R][S][2][128]: m then l (splits > 1)
   int n_q, s_max, k, splits, rows_per_split;
-  int pair;                 // 1: two splits per 4-CTA cluster, merged in the kernel (splits == 2)
   float scale_log2;         // sm_scale * log2(e)
   uint32_t* err;
 };
@@ -329,9 +328,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
 
   const int warp = threadIdx.x >> 5;
   const int lane = lane_id();
-  const uint32_t crank_c = cluster_rank();
-  const uint32_t crank = crank_c & 1u;    // latent columns [256c, 256c + 256), rope [512 + 32c, 544 + 32c)
-  const uint32_t peer = crank_c ^ 1u;     // the other column half of the same split
+  const uint32_t crank = cluster_rank();  // latent columns [256c, 256c + 256), rope [512 + 32c, 544 + 32c)
+  const uint32_t peer = crank ^ 1u;
   const int a0 = crank * kLatAtoms;                       // first 64-column latent atom of this CTA
   const int rope0 = kLatCols * 2 + crank * kRopeCols;     // first rope column of this CTA
   // work item of the cluster
@@ -381,9 +379,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
   tc_fence_after_sync();
   cluster_sync_all();  // both CTAs' barriers exist (and are armed) before any remote arrival
   const uint32_t tmem = *tmem_slot;
-  // the even split of a pair keeps its result in TMEM until the odd split's is in memory
-  float out_m = -INFINITY, out_l = 0.f;
-  bool out_ok = false;
 
   if (warp == kCommWarp) {
     // --------------------------------------- copies and cross-CTA signals --
@@ -700,11 +695,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
     pdl_trigger();
     // (PV of tile T - 2 was awaited at tile T - 1: this parity is unambiguous)
     if (ok && T >= 1) ok = mbar_wait_warp(pv_done, (T - 1) & 1, abort_flag, P.err);
-    if (ok && P.pair && (sp & 1) == 0) {
-      out_ok = true;
-      out_m = m_fin;
-      out_l = l_fin;
-    } else if (ok) {
+    if (ok) {
       tc_fence_after_sync();
       const int64_t rh = static_cast<int64_t>(r) * kH + h;
       const int c_lo = kh * 128, c_hi = c_lo + 128;
@@ -751,64 +742,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
     }
   }
 
-  if (P.pair) {
-    // two splits of one query in this cluster: once the odd split's partial
-    // output and (m, l) are in memory, the even split's softmax threads merge
-    // them with its own accumulator (base-2 log-sum-exp weights) and write
-    // the output -- the combine kernel's work, without its launch
-    tc_fence_before_sync();
-    cluster_sync_all();
-    tc_fence_after_sync();
-    if (out_ok) {
-      const int quarter = warp & 3;
-      const int kh = (warp - (kGatherWarps + 1)) >> 2;
-      const int h = quarter * 32 + lane;
-      const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-      const int64_t ms1 = static_cast<int64_t>(r) * P.splits + sp + 1;
-      const float m1 = P.part_ml[(ms1 * 2 + 0) * kH + h];
-      const float l1 = P.part_ml[(ms1 * 2 + 1) * kH + h];
-      float M = -INFINITY;
-      if (out_l > 0.f) M = out_m;
-      if (l1 > 0.f) M = fmaxf(M, m1);
-      const float c0 = out_l > 0.f ? exp2f(out_m - M) : 0.f;
-      const float c1 = l1 > 0.f ? exp2f(m1 - M) : 0.f;
-      const float Ls = c0 * out_l + c1 * l1;
-      const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-      const float w0 = c0 * inv, w1 = c1 * inv;
-      const int64_t rh = static_cast<int64_t>(r) * kH + h;
-      const float* src = P.part_o + ((ms1 * 2 + crank) * kH + h) * kDvHalf;
-      __nv_bfloat16* dst = P.out + rh * kDv + crank * kDvHalf;
-      const int c_lo = kh * 128, c_hi = c_lo + 128;
-#pragma unroll 1
-      for (int c = c_lo; c < c_hi; c += 32) {
-        float o[32];
-        if (T >= 1) tmem_ld32(tl + c, o);
-        else
-          for (int i = 0; i < 32; ++i) o[i] = 0.f;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4 a = *reinterpret_cast<const float4*>(src + c + q * 8);
-          const float4 b2 = *reinterpret_cast<const float4*>(src + c + q * 8 + 4);
-          uint4 v;
-          v.x = pack_bf16(fmaf(w0, o[q * 8 + 0], w1 * a.x), fmaf(w0, o[q * 8 + 1], w1 * a.y));
-          v.y = pack_bf16(fmaf(w0, o[q * 8 + 2], w1 * a.z), fmaf(w0, o[q * 8 + 3], w1 * a.w));
-          v.z = pack_bf16(fmaf(w0, o[q * 8 + 4], w1 * b2.x), fmaf(w0, o[q * 8 + 5], w1 * b2.y));
-          v.w = pack_bf16(fmaf(w0, o[q * 8 + 6], w1 * b2.z), fmaf(w0, o[q * 8 + 7], w1 * b2.w));
-          *reinterpret_cast<uint4*>(dst + c + q * 8) = v;
-        }
-      }
-      if (P.lse != nullptr && crank == 0 && kh == 0)
-        P.lse[rh] = Ls > 0.f ? (M + log2f(Ls)) * 0.6931471805599453f : -INFINITY;
-    }
-  }
-
   tc_fence_before_sync();
   __syncthreads();
   if (warp == kMmaWarp) {
     tc_fence_after_sync();
     tmem_dealloc(tmem, kTmemCols);
   }
-  cluster_sync_all();  // no CTA leaves while another may still touch its shared memory
+  cluster_sync_all();  // no CTA leaves while the other may still touch its shared memory
 }
 }  // namespace
 }  // namespace dsa
@@ -897,34 +837,6 @@ SplitPlan plan_splits(int64_t R, int k, int num_sms) {
   return p;
 }
 
-// Whether R 4-CTA clusters of the attention kernel are co-resident on the
-// device (queried once per device: the answer depends only on the kernel's
-// resources and the GPU's layout of SMs into clusters).
-bool pair_clusters_fit(int dev, int64_t R) {
-  static int max_clusters[64] = {};
-  if (dev < 0 || dev >= 64) return false;
-  if (max_clusters[dev] == 0) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(4, 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = kSmemBytes;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 4;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, attn_mla_tc_kernel, &cfg) != cudaSuccess || n <= 0) {
-      (void)cudaGetLastError();
-      n = -1;
-    }
-    max_clusters[dev] = n;
-  }
-  return max_clusters[dev] > 0 && R <= max_clusters[dev];
-}
-
 size_t scratch_bytes(int64_t R, const SplitPlan& p) {
   if (p.splits <= 1) return 0;
   const size_t items = static_cast<size_t>(R) * p.splits * 2;
@@ -973,7 +885,6 @@ dsa_status_t attn_tc(const AttnArgs& a) {
   P.err = a.err;
   P.part_o = nullptr;
   P.part_ml = nullptr;
-  P.pair = 0;
   if (p.splits > 1) {
     const size_t need = scratch_bytes(R, p);
     if (a.ws == nullptr || a.ws_bytes < need) return DSA_ERR_WORKSPACE;
@@ -1001,14 +912,8 @@ dsa_status_t attn_tc(const AttnArgs& a) {
   attr[1] = pdl_attribute();
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  // two splits: one 4-CTA cluster per query merges them in the kernel, when
-  // all the clusters fit on the GPU at once (else 2-CTA clusters + combine)
-  if (p.splits == 2 && pair_clusters_fit(a.device, R)) {
-    attr[0].val.clusterDim.x = 4;
-    P.pair = 1;
-  }
   if (cudaLaunchKernelEx(&cfg, attn_mla_tc_kernel, P) != cudaSuccess) return DSA_ERR_CUDA;
-  if (p.splits > 1 && !P.pair) {
+  if (p.splits > 1) {
     cudaLaunchConfig_t cc = {};
     cc.gridDim = dim3(static_cast<unsigned>(R), kH / kCombineHeads, 1);
     cc.blockDim = dim3(256, 1, 1);

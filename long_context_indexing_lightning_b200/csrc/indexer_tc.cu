@@ -361,23 +361,10 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
       };
       const int kt_first = C::kAltTiles ? U.kt0 + ((grp - ncomp) & 1) : U.kt0;
       if (C::kAltTiles && U.kt_comp > U.kt0) ncomp += U.kt_comp - U.kt0;
-      float ks0 = 1.f, ks1 = 1.f, ks2 = 1.f, ks3 = 1.f;
-      if (kFP8) {
-        ks0 = load_ks(kt_first);
-        ks1 = load_ks(kt_first + kStep);
-        ks2 = load_ks(kt_first + 2 * kStep);
-        ks3 = load_ks(kt_first + 3 * kStep);
-      }
-      bool ok = true;
-      for (int kt = kt_first; kt < U.kt_comp; kt += kStep) {
-        const float ks = ks0;
-        if (kFP8) {
-          ks0 = ks1;
-          ks1 = ks2;
-          ks2 = ks3;
-          ks3 = load_ks(kt + 4 * kStep);
-        }
-        if (!mbar_wait_warp(acc_full(ab), aph, abort_flag, err)) { ok = false; break; }
+      // One key tile of the epilogue (FP8: its keys' scale ks); false if a
+      // wait expired.
+      auto tile = [&](int kt, float ks) -> bool {
+        if (!mbar_wait_warp(acc_full(ab), aph, abort_flag, err)) return false;
         tc_fence_after_sync();
         const int s = kt * kTileKeys + row;
         const uint32_t tl = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(ab * C::N);
@@ -429,6 +416,30 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
         mbar_arrive(acc_empty(ab));
         ab += kStep;
         if (ab >= C::kNumAcc) { ab -= C::kNumAcc; aph ^= 1; }
+        return true;
+      };
+      bool ok = true;
+      if constexpr (kFP8) {
+        // unrolled four ways so that each scale register is read four tiles
+        // after its load, with no register moves in between (a move of a
+        // load still in flight would wait for it)
+        float ks0 = load_ks(kt_first), ks1 = load_ks(kt_first + kStep), ks2 = load_ks(kt_first + 2 * kStep),
+              ks3 = load_ks(kt_first + 3 * kStep);
+        for (int kt = kt_first; ok && kt < U.kt_comp; kt += 4 * kStep) {
+          ok = tile(kt, ks0);
+          ks0 = load_ks(kt + 4 * kStep);
+          if (!ok || kt + kStep >= U.kt_comp) break;
+          ok = tile(kt + kStep, ks1);
+          ks1 = load_ks(kt + 5 * kStep);
+          if (!ok || kt + 2 * kStep >= U.kt_comp) break;
+          ok = tile(kt + 2 * kStep, ks2);
+          ks2 = load_ks(kt + 6 * kStep);
+          if (!ok || kt + 3 * kStep >= U.kt_comp) break;
+          ok = tile(kt + 3 * kStep, ks3);
+          ks3 = load_ks(kt + 7 * kStep);
+        }
+      } else {
+        for (int kt = kt_first; ok && kt < U.kt_comp; kt += kStep) ok = tile(kt, 1.f);
       }
       if (!ok) break;
       // key tiles entirely after every query of the block: -inf only

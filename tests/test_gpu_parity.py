@@ -217,6 +217,22 @@ def test_topk_prefill_rows_all_positions():
     _topk_case(1, n_q, S, k, [S], [0], sc)
 
 
+def test_topk_many_long_rows_walked_in_chunks():
+    """A launch with more rows than twice the SM count (a prefill round) runs
+    one CTA per row, walking it in 8K-key chunks: 400 query rows at
+    positions 39600..39999 of a 40,000-key row (five chunks), gaussian rows
+    with exact ties, rows of equal scores and rows inside one exponent bucket
+    (the overflow path), exact against the oracle."""
+    g = np.random.default_rng(21)
+    n_q, S, k = 400, 40000, 2048
+    sc = g.standard_normal((1, n_q, S)).astype(np.float32)
+    sc[0, :, ::5] = np.round(sc[0, :, ::5] * 4) / 4          # exact ties
+    sc[0, 7] = np.float32(-0.5)                              # all equal
+    sc[0, 8] = (1.0 + g.random(S)).astype(np.float32)        # one exponent bucket
+    sc[0, 9, ::2] = -0.0                                     # signed zeros
+    _topk_case(1, n_q, S, k, [S], [S - n_q], sc)
+
+
 def test_topk_gaussian_decode128k_shape():
     g = np.random.default_rng(9)
     B, S, k = 32, 131072, 2048
@@ -331,11 +347,11 @@ def test_attention_bf16_ragged_selection_and_padding():
     assert err <= ATTN_ATOL_BF16, err
 
 
-def test_attention_bf16_two_splits_merged_in_cluster():
-    """32 decode queries: the split plan gives each query two splits, which
-    one 4-CTA cluster merges in the kernel.  Rows with an empty second split
-    (at most 1024 selected keys) and a partial one, -1 padding, unsorted
-    indices; output and lse against the oracle."""
+def test_attention_bf16_two_splits_per_query():
+    """32 decode queries (the benchmark's batch): the split plan gives each
+    query two splits, merged by the combine kernel.  Rows with an empty
+    second split (at most 1024 selected keys) and a partial one, -1 padding,
+    unsorted indices; output and lse against the oracle."""
     lengths = tuple([4096] * 28 + [100, 1024, 1500, 2049])
     wl = _custom("decode32k", batch=32, s_max=4096, ctx_len=lengths)
     t = workloads.make_inputs(wl, DEV, seed=18)
