@@ -547,20 +547,39 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
     {
       // this CTA's columns of q[r, h, :] as packed bf16 pairs (element 2i in
       // the low half of column i); the quarter's two warps take half each
+      // (a thread's loads are all issued ahead of its tensor-memory stores:
+      // a store is a compiler barrier, and loads issued one chunk at a time
+      // would put five memory round trips before the first MMA)
       const uint16_t* qrow = P.q + (static_cast<int64_t>(r) * kH + h) * kDqk;
-      constexpr int kChunks = kQk / 32;  // 32-column chunks: latent 0..7, rope 8
-      for (int c = kh == 0 ? 0 : (kChunks + 1) / 2; c < (kh == 0 ? (kChunks + 1) / 2 : kChunks); ++c) {
-        const uint4* qs = reinterpret_cast<const uint4*>(qrow + (c < kLatCols / 32 ? a0 * 64 + c * 32 : rope0));
-        uint32_t u[16];
+      constexpr int kChunks = kQk / 32;           // 32-column chunks: latent 0..7, rope 8
+      constexpr int kMine = (kChunks + 1) / 2;    // chunks of the first warp of a quarter (the second: one fewer)
+      const int c0 = kh == 0 ? 0 : kMine;
+      const int nmine = kh == 0 ? kMine : kChunks - kMine;
+      constexpr int kBatch = kMine;  // chunks whose loads are in flight together
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const uint4 x = __ldg(qs + v);
-          u[4 * v + 0] = x.x;
-          u[4 * v + 1] = x.y;
-          u[4 * v + 2] = x.z;
-          u[4 * v + 3] = x.w;
+      for (int i0 = 0; i0 < kMine; i0 += kBatch) {
+        uint4 x[kBatch][4];
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+          const int i = i0 + j, c = c0 + i;
+          const uint4* qs = reinterpret_cast<const uint4*>(qrow + (c < kLatCols / 32 ? a0 * 64 + c * 32 : rope0));
+#pragma unroll
+          for (int v = 0; v < 4; ++v) x[j][v] = i < nmine ? __ldg(qs + v) : make_uint4(0u, 0u, 0u, 0u);
         }
-        tmem_st16(tl + kQCol + c * 16, u);
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+          const int i = i0 + j;
+          if (i >= nmine) break;
+          uint32_t u[16];
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            u[4 * v + 0] = x[j][v].x;
+            u[4 * v + 1] = x[j][v].y;
+            u[4 * v + 2] = x[j][v].z;
+            u[4 * v + 3] = x[j][v].w;
+          }
+          tmem_st16(tl + kQCol + (c0 + i) * 16, u);
+        }
       }
       tmem_st_wait();
       tc_fence_before_sync();
@@ -762,9 +781,13 @@ constexpr int kCombineHeads = 8;  // heads per combine block
 // Merge the per-split partial outputs of each query: O = sum_i 2^(m_i - M) O_i
 // / sum_i 2^(m_i - M) l_i with M = max_i m_i (base-2 log-sum-exp combine).
 // Block = (query, group of 8 heads); 256 threads, 4 output columns a step.
+// kS = the split count, a template argument so that every load of a thread
+// (four output positions x kS splits) is issued before the first is used.
+template <int kS>
 __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restrict__ part_o,
-                                                           const float* __restrict__ part_ml, int splits,
+                                                           const float* __restrict__ part_ml,
                                                            __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+  constexpr int splits = kS;
   pdl_wait();
   __shared__ float coef[kMaxSplits][kCombineHeads];
   const int r = blockIdx.x;
@@ -794,23 +817,36 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
       lse[static_cast<int64_t>(r) * kH + h] = Ls > 0.f ? (M + log2f(Ls)) * 0.6931471805599453f : -INFINITY;
   }
   __syncthreads();
+  constexpr int kItr = kCombineHeads * (kDv / 4) / 256;  // output positions a thread
+  float4 o[kItr][kS];
 #pragma unroll
-  for (int itr = 0; itr < kCombineHeads * (kDv / 4) / 256; ++itr) {
+  for (int itr = 0; itr < kItr; ++itr) {
     const int x = itr * 256 + tid;
     const int hl = x / (kDv / 4);
     const int c4 = x % (kDv / 4);
     const int h = h0 + hl;
     const int hv = c4 / (kDvHalf / 4);
     const int cc = (c4 % (kDvHalf / 4)) * 4;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int i = 0; i < splits; ++i) {
+#pragma unroll
+    for (int i = 0; i < kS; ++i) {
       const int64_t it = (static_cast<int64_t>(r) * splits + i) * 2 + hv;
-      const float4 o = __ldg(reinterpret_cast<const float4*>(part_o + (it * kH + h) * kDvHalf + cc));
+      o[itr][i] = __ldg(reinterpret_cast<const float4*>(part_o + (it * kH + h) * kDvHalf + cc));
+    }
+  }
+#pragma unroll
+  for (int itr = 0; itr < kItr; ++itr) {
+    const int x = itr * 256 + tid;
+    const int hl = x / (kDv / 4);
+    const int c4 = x % (kDv / 4);
+    const int h = h0 + hl;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < kS; ++i) {
       const float c = coef[i][hl];
-      acc.x = fmaf(c, o.x, acc.x);
-      acc.y = fmaf(c, o.y, acc.y);
-      acc.z = fmaf(c, o.z, acc.z);
-      acc.w = fmaf(c, o.w, acc.w);
+      acc.x = fmaf(c, o[itr][i].x, acc.x);
+      acc.y = fmaf(c, o[itr][i].y, acc.y);
+      acc.z = fmaf(c, o[itr][i].z, acc.z);
+      acc.w = fmaf(c, o[itr][i].w, acc.w);
     }
     uint2 v;
     v.x = pack_bf16(acc.x, acc.y);
@@ -921,9 +957,19 @@ dsa_status_t attn_tc(const AttnArgs& a) {
     cudaLaunchAttribute cattr[1] = {pdl_attribute()};
     cc.attrs = cattr;
     cc.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cc, attn_combine_kernel, static_cast<const float*>(P.part_o),
-                           static_cast<const float*>(P.part_ml), p.splits, P.out, a.lse) != cudaSuccess)
-      return DSA_ERR_CUDA;
+    cudaError_t e = cudaErrorInvalidValue;
+    const float* po = P.part_o;
+    const float* pm = P.part_ml;
+    switch (p.splits) {
+#define DSA_COMBINE_CASE(S) \
+  case S: e = cudaLaunchKernelEx(&cc, attn_combine_kernel<S>, po, pm, P.out, a.lse); break;
+      DSA_COMBINE_CASE(2) DSA_COMBINE_CASE(3) DSA_COMBINE_CASE(4) DSA_COMBINE_CASE(5) DSA_COMBINE_CASE(6)
+      DSA_COMBINE_CASE(7) DSA_COMBINE_CASE(8) DSA_COMBINE_CASE(9) DSA_COMBINE_CASE(10) DSA_COMBINE_CASE(11)
+      DSA_COMBINE_CASE(12) DSA_COMBINE_CASE(13) DSA_COMBINE_CASE(14) DSA_COMBINE_CASE(15) DSA_COMBINE_CASE(16)
+#undef DSA_COMBINE_CASE
+      default: return DSA_ERR_UNSUPPORTED;
+    }
+    if (e != cudaSuccess) return DSA_ERR_CUDA;
   }
   return DSA_OK;
 }

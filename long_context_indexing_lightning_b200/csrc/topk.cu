@@ -489,6 +489,9 @@ __global__ void __launch_bounds__(kThreads, 2) topk_cluster_kernel(RowSel P) {
   // ---- overflow: the remaining digits from histograms of every CTA's keys,
   // merged in the leader (h2sum, h3sum; with C == 1 the CTA's own)
   const uint32_t lead2 = map_rank(sm.h2sum, 0), lead3 = map_rank(sm.h3sum, 0);
+  // every thread has taken ncand from sm.hist before it is cleared: a warp
+  // that read a cleared bin would take the fits branch on its own
+  __syncthreads();
   for (int i = tid; i < kBins1; i += kThreads) sm.hist[i] = 0;
   __syncthreads();
   for (int ch = 0; ch < nch; ++ch) {

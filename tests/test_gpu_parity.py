@@ -233,6 +233,26 @@ def test_topk_many_long_rows_walked_in_chunks():
     _topk_case(1, n_q, S, k, [S], [S - n_q], sc)
 
 
+@pytest.mark.parametrize("B,n_q,S", [
+    (1, 600, 65536),   # a prefill round: one CTA a row, eight 8K-key chunks
+    (24, 1, 131072),   # decode rows: a cluster of eight CTAs a row
+])
+def test_topk_every_row_on_the_overflow_path(B, n_q, S):
+    """Every row's candidate bin (the first 11 key bits) holds far more than
+    the 4096 keys the leader's lists take: scores inside [1, 2) on a grid of
+    2^-12 (a quarter of the keys a first-digit bin, thousands of exact
+    ties), a few rows of one value.  Exact against the oracle."""
+    g = np.random.default_rng(31)
+    sc = (1.0 + g.integers(0, 4096, size=(B, n_q, S)) / 4096.0).astype(np.float32)
+    sc[0, 0] = np.float32(1.25)
+    sc[-1, -1] = np.float32(1.5)
+    k = 2048
+    if n_q > 1:
+        _topk_case(B, n_q, S, k, [S] * B, [S - n_q] * B, sc)
+    else:
+        _topk_case(B, n_q, S, k, [S] * B, [S - 1] * B, sc)
+
+
 def test_topk_gaussian_decode128k_shape():
     g = np.random.default_rng(9)
     B, S, k = 32, 131072, 2048
