@@ -51,7 +51,10 @@ typedef enum {
     DSA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than dsa_workspace_bytes() */
     DSA_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
     DSA_ERR_TIMEOUT = 5,      /* (device) a bounded wait inside a kernel expired */
-    DSA_ERR_BAD_INDEX = 6     /* (device) an attention index was >= ctx_len and was skipped */
+    DSA_ERR_BAD_INDEX = 6,    /* (device) an attention index was >= ctx_len and was skipped */
+    DSA_ERR_HIST_MISMATCH = 7 /* (device) dsa_topk_hist was given partial histograms that do not
+                                 describe its scores (not from the dsa_indexer_scores_hist call
+                                 that wrote them); the affected rows' indices are undefined */
 } dsa_status_t;
 
 typedef enum {
@@ -182,7 +185,10 @@ dsa_status_t dsa_indexer_proj_kw(const dsa_shape_t *shape, int32_t n_tokens, int
  *         16-byte aligned, opaque; written by the indexer call, read by the
  *         top-k call.  The two calls must be made with the same shape on the
  *         same device, with the top-k reading the scores the indexer call
- *         wrote, and nothing else writing `hist` in between.
+ *         wrote, and nothing else writing `hist` in between.  The top-k
+ *         checks the counts against the scores it reads: where they differ
+ *         it records DSA_ERR_HIST_MISMATCH in the device error word and the
+ *         row's indices are undefined (no access outside the buffers).
  */
 dsa_status_t dsa_indexer_scores_hist(const dsa_shape_t *shape,
                                      const void *q_idx, const float *q_scale,
@@ -436,8 +442,9 @@ size_t dsa_workspace_bytes(const dsa_shape_t *shape, int32_t which);
 
 /*
  * Reads (and, if clear != 0, resets) the device error word of the current
- * device.  Synchronises the device.  Returns DSA_OK, DSA_ERR_TIMEOUT or
- * DSA_ERR_BAD_INDEX (the first recorded kind), or DSA_ERR_CUDA if the read
+ * device.  Synchronises the device.  Returns DSA_OK, DSA_ERR_TIMEOUT,
+ * DSA_ERR_BAD_INDEX or DSA_ERR_HIST_MISMATCH (the first recorded kind in that
+ * order), or DSA_ERR_CUDA if the read
  * itself failed.  `detail`, if not NULL, receives the raw word.
  * Sharing: the word lives in the library's own device memory, one per
  * device, not in a caller's workspace -- several entry points that can

@@ -21,7 +21,7 @@ WS_TOPK, WS_ATTN, WS_FORWARD, WS_FORWARD_HOST, WS_HIST = 0, 1, 2, 3, 4
 
 STATUS = {
     0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "DSA_ERR_WORKSPACE",
-    4: "DSA_ERR_CUDA", 5: "DSA_ERR_TIMEOUT", 6: "DSA_ERR_BAD_INDEX",
+    4: "DSA_ERR_CUDA", 5: "DSA_ERR_TIMEOUT", 6: "DSA_ERR_BAD_INDEX", 7: "DSA_ERR_HIST_MISMATCH",
 }
 
 EXPORTS = (

@@ -412,11 +412,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
     // Row reads from HBM take microseconds while a ring stage is held; pull
     // each tile's rows into L2 up to kPrefetchAhead tiles before its gather,
     // so the gather into the ring reads L2.  Lane l covers rows l and l + 32.
+    // The ring's first kStages tiles are gathered at once; prefetching starts
+    // behind those gathers (issued ahead of them, the prefetches of a whole
+    // GPU delay the first tiles by microseconds).
     const uint64_t t0 = global_timer_ns();
-    for (int t = 1; t < T; ++t) {
+    const int first = min(T, kStages);
+    for (int t = kStages; t < T; ++t) {
       // stay at most kPrefetchAhead tiles ahead of the issued gathers (bounded)
       bool go = true;
-      for (uint32_t i = 0; *gather_progress + kPrefetchAhead < t; ++i) {
+      for (uint32_t i = 0; *gather_progress < first || *gather_progress + kPrefetchAhead < t; ++i) {
         if ((i & 63u) == 63u && (*abort_flag || global_timer_ns() - t0 > kWaitLimitNs)) {
           go = false;
           break;
@@ -630,6 +634,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
         }
       }
       const uint32_t valid = __ballot_sync(0xffffffffu, ((vbits >> (j - vbase)) & 1u) != 0);
+      // tile j + 1's partial goes out first, from every warp at the same
+      // point, so its copy runs while this CTA waits for the other CTA's
+      // partial of tile j and under this tile's softmax (tile j depends on
+      // the other CTA's tiles j - 1 and j - 2 only)
+      if (j + 1 < T) {
+        if (!mbar_wait_warp(s_full, (j + 1) & 1, abort_flag, P.err)) { ok = false; break; }
+        read_s(snext);
+        // the copy of tile j has read xout
+        if (!mbar_wait_warp(xout_free, j & 1, abort_flag, P.err)) { ok = false; break; }
+        write_x(snext);
+      }
       // S = S_0 + S_1
       if (!mbar_wait_warp_cluster(x_full(bb), (j >> 1) & 1, abort_flag, P.err)) { ok = false; break; }
       // arm for tile j + 2 (the other CTA sends it only after x_empty of tile j)
@@ -643,15 +658,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
         sreg[4 * c + 3] += v.w;
       }
       mbar_arrive(xin_read(bb));
-      // tile j + 1's partial goes out before this tile's softmax, from every
-      // warp at the same point, so the copy runs under the softmax
-      if (j + 1 < T) {
-        if (!mbar_wait_warp(s_full, (j + 1) & 1, abort_flag, P.err)) { ok = false; break; }
-        read_s(snext);
-        // the copy of tile j has read xout
-        if (!mbar_wait_warp(xout_free, j & 1, abort_flag, P.err)) { ok = false; break; }
-        write_x(snext);
-      }
       float mt = -INFINITY;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {

@@ -900,6 +900,7 @@ dsa_status_t dsa_get_error(int32_t clear, uint32_t* detail) {
   if (detail) *detail = word[0];
   if (word[0] & kErrTimeout) return DSA_ERR_TIMEOUT;
   if (word[0] & kErrBadIndex) return DSA_ERR_BAD_INDEX;
+  if (word[0] & kErrHistMismatch) return DSA_ERR_HIST_MISMATCH;
   return DSA_OK;
 }
 
@@ -912,6 +913,7 @@ const char* dsa_status_string(dsa_status_t status) {
     case DSA_ERR_CUDA: return "CUDA error";
     case DSA_ERR_TIMEOUT: return "a bounded wait inside a kernel expired";
     case DSA_ERR_BAD_INDEX: return "attention index out of range (skipped)";
+    case DSA_ERR_HIST_MISMATCH: return "handed-over histograms do not match the scores";
   }
   return "unknown status";
 }

@@ -13,7 +13,7 @@ namespace dsa {
 
 // ---------------------------------------------------------------- errors --
 // Bits of the per-device error word (see dsa_get_error).
-enum : uint32_t { kErrTimeout = 1u, kErrBadIndex = 2u };
+enum : uint32_t { kErrTimeout = 1u, kErrBadIndex = 2u, kErrHistMismatch = 4u };
 
 // Every wait on an mbarrier gives up after this long (ns of %globaltimer) or
 // this many polls, records kErrTimeout and lets the kernel unwind.
@@ -159,6 +159,23 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
       : "memory");
+}
+
+// The same load with an L2 eviction-priority hint (a policy from
+// l2_evict_first()): for data read once, so that it does not push out what a
+// later kernel reads (this GPU's own memory; no multicast).
+__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
+                                                 uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
 }
 
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* map) {

@@ -200,6 +200,7 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
       int st = 0, qb = 0;
       uint32_t kph = 0, qph = 0;
       int last_bg = -1;
+      const uint64_t key_policy = l2_evict_first();
       uint32_t issued_k[kStages];
       uint32_t issued_q[kQBufs];
       for (int i = 0; i < kStages; ++i) issued_k[i] = 0;
@@ -227,9 +228,17 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
           mbar_arrive_expect_tx(k_full(st), C::kKTile);
           const int krow = U.b * S.s_max + kt * kTileKeys;
           const uint32_t kdst = sbase + C::kOffK + st * C::kKTile;
+          // decode reads each key tile once: marked first to leave L2, so the
+          // score rows (read next by the top-k) stay there; prefill re-reads
+          // key tiles across query blocks and keeps the default
 #pragma unroll
-          for (int kb = 0; kb < C::kKBlocks; ++kb)
-            tma_load_2d(kdst + kb * kTileKeys * 128, &tmap_k, k_full(st), kb * (128 / C::kElem), krow);
+          for (int kb = 0; kb < C::kKBlocks; ++kb) {
+            if constexpr (kQG == 1)
+              tma_load_2d_hint(kdst + kb * kTileKeys * 128, &tmap_k, k_full(st), kb * (128 / C::kElem), krow,
+                               key_policy);
+            else
+              tma_load_2d(kdst + kb * kTileKeys * 128, &tmap_k, k_full(st), kb * (128 / C::kElem), krow);
+          }
           issued_k[st]++;
           if (++st == kStages) { st = 0; kph ^= 1; }
         }

@@ -5,27 +5,40 @@
 // Radix select on order-preserving 32-bit keys, no sort.  One query row is
 // split over a thread-block cluster of C CTAs (C = 1..16, 16K keys a CTA in
 // two chunks of 8K, read with coalesced loads); when a launch has many rows
-// (prefill), C = 1 and each CTA walks its row chunk by chunk.  The key splits into
-// digits of 11, 11 and 10 bits; T, the key of the k-th largest score, is
+// (prefill), C = 1 and each CTA walks its row chunk by chunk.  The key splits
+// into digits of 11, 11 and 10 bits; T, the key of the k-th largest score, is
 // found digit by digit:
 //   1. the first digit's histogram: summed from the partial histograms the
-//      indexer's epilogue built (TopkArgs::hist_parts), or counted by each CTA
-//      and merged in the cluster's first CTA (the leader); the bin D1 holding
-//      the k-th largest key follows;
-//   2. each CTA keeps, in index order, its "sure" keys (first digit > D1;
-//      fewer than k in the row) and its candidates (first digit == D1; on index
-//      scores a few thousand in a 128K row) in shared memory -- warp scans
-//      give each flagged key its slot (no atomics, no sort);
-//   3. one cluster barrier; the leader appends the other CTAs' lists to its
-//      own (distributed shared memory, rank order = index order), takes the
-//      second and third digits from the candidates, selects them (key > T,
-//      then the lowest-indexed keys == T: ties go to the lower index) and
-//      merges them with the sure keys into the ascending output.
-// Rows whose candidates or sure keys overflow the leader's lists (all-equal
-// rows, rows inside one exponent bucket) take the second and third digits
-// from cluster-wide histograms of every CTA's slice (merged in the leader),
-// then every CTA writes its own kept keys at offsets from the lower-ranked
-// CTAs' counts.  Rows with at most k candidates are written directly.
+//      indexer's epilogue built (TopkArgs::hist_parts) straight into
+//      registers, or counted by each CTA and merged in the cluster's first
+//      CTA (the leader); every CTA finds the bin D1 holding the k-th largest
+//      key, the keys above it and the keys in it;
+//   2. each CTA lists its keys with first digit >= D1 (the sure keys above D1
+//      and the candidates in it) in index order in its shared memory: a
+//      chunk's keys are ordered by warp scans (no sort, no atomics), and the
+//      candidates' second digits are counted on the way;
+//   3. the second and third digits: each CTA adds its counts into the
+//      leader's histograms (remote atomics, one cluster barrier each) and
+//      every CTA selects the digit from them; only the few listed keys in the
+//      second digit's bin are read again for their third digit;
+//   4. each CTA counts its kept keys (key > T, then the lowest-indexed keys ==
+//      T: ties go to the lower index), learns the lower-ranked CTAs' counts
+//      through the leader, and writes its kept keys into its own range of the
+//      ascending output, warps ranking the list with ballots.
+// A list entry is one word: bit 31 = sure key (first digit > D1), bits 19..29
+// = the second digit (after the third-digit pass, for the entries in the
+// second digit's bin D2: the third digit, flagged by bit 30), bits 13..18 =
+// the chunk of the CTA's walk, bits 0..12 = the key's offset in that chunk.
+// A CTA of a cluster lists at most its own 16K keys, so every clustered row
+// fits.  A single CTA whose row lists more keys than its list holds
+// (all-equal rows, rows inside one exponent bucket) takes the second and
+// third digits from histograms of the whole row and writes its kept keys
+// chunk by chunk.  Rows with at most k candidates are written directly.
+//
+// The handed-over partial histograms are checked against the scores: a
+// mismatch (a histogram from another call) records DSA_ERR_HIST_MISMATCH in
+// the device error word and leaves the row's output undefined, never an
+// access out of bounds.
 #include "dsa_common.cuh"
 #include "dsa_internal.h"
 
@@ -36,13 +49,22 @@ constexpr int kThreads = 512;
 constexpr int kPer = 16;                   // keys a thread in a chunk
 constexpr int kSteps = kPer / 4;           // float4 steps a lane
 constexpr int kChunk = kThreads * kPer;    // keys a chunk: 8192
-constexpr int kCtaChunks = 2;              // chunks a CTA of a cluster takes
-constexpr int kSlice = kCtaChunks * kChunk;  // keys a CTA of a cluster: 16384
+// Two instances: clustered rows (decode) with CTAs of 4 chunks (32K keys, one
+// CTA an SM, the slice brought into shared memory by one bulk copy), and one
+// CTA walking a row (many rows: two CTAs an SM, keys read chunk by chunk).
+constexpr int kClusterChunks = 4;          // chunks a CTA of a cluster takes
+constexpr int kClusterSlice = kClusterChunks * kChunk;  // keys a CTA of a cluster: 32768
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxCluster = 16;
 constexpr int kBins1 = 2048;               // first and second digits: 11 bits
 constexpr int kBins3 = 1024;               // third digit: 10 bits
-constexpr int kListCap = 4096;             // leader's sure / candidate list capacity
+constexpr int kListCapCluster = kClusterSlice;  // a clustered CTA lists at most its slice
+constexpr int kListCapRow = 16384;         // a CTA walking a row: longer lists take the overflow path
+constexpr uint32_t kNoBin = 0xFFFFFFFFu;   // select found no bin: the counts do not add up
+constexpr uint32_t kSure = 1u << 31;       // list entry: first digit > D1
+constexpr uint32_t kHasD3 = 1u << 30;      // list entry: bits 19..29 hold the third digit
+constexpr uint32_t kOffMask = kChunk - 1;  // list entry: offset in the chunk
+static_assert(kChunk == 8192, "13-bit chunk offsets");
 
 // ------------------------------------------------- distributed shared memory --
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -56,10 +78,21 @@ __device__ __forceinline__ uint32_t map_rank(const void* p, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
   return r;
 }
+__device__ __forceinline__ uint4 ld_cluster_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
 __device__ __forceinline__ uint32_t ld_cluster(uint32_t addr) {
   uint32_t v;
   asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
   return v;
+}
+__device__ __forceinline__ void st_cluster(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 __device__ __forceinline__ void red_add_cluster(uint32_t addr, uint32_t v) {
   asm volatile("red.relaxed.cluster.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
@@ -73,6 +106,11 @@ __device__ __forceinline__ void cluster_wait() {
 __device__ __forceinline__ void cluster_sync() {
   cluster_arrive();
   cluster_wait();
+}
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
 }
 
 // ------------------------------------------------------------------ scans --
@@ -106,68 +144,95 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* wsum, 
   return res;
 }
 
-// The bin of `hist` (nbins, counted from the top) that holds the
-// `remaining`-th largest key: *digit, and *above = keys in higher bins.
-__device__ __forceinline__ void select_bin(const uint32_t* hist, int nbins, uint32_t remaining, uint32_t* wsum,
-                                           uint32_t* s_digit, uint32_t* s_above) {
-  const int bpt = nbins / kThreads;  // bins a thread, taken from the top
-  const int top = nbins - 1 - static_cast<int>(threadIdx.x) * bpt;
+// The bin holding the `remaining`-th largest key of a histogram of
+// kBpt * kThreads bins, thread t holding the counts of bins top - j (j <
+// kBpt, top = bins - 1 - t kBpt) in h[j].  Writes res[0] = the bin (kNoBin if
+// the counts add up to fewer than `remaining`), res[1] = keys in higher bins,
+// res[2] = keys in the bin.  Ends with a barrier.
+template <int kBpt>
+__device__ __forceinline__ void select_bin(const uint32_t (&h)[kBpt], uint32_t remaining, uint32_t* wsum,
+                                           uint32_t* res) {
+  if (threadIdx.x == 0) {
+    res[0] = kNoBin;
+    res[1] = 0;
+    res[2] = 0;
+  }
   uint32_t cnt = 0;
-  for (int i = 0; i < bpt; ++i) cnt += hist[top - i];
+#pragma unroll
+  for (int j = 0; j < kBpt; ++j) cnt += h[j];
   uint32_t total;
-  const uint32_t excl = block_excl_scan(cnt, wsum, &total);
+  const uint32_t excl = block_excl_scan(cnt, wsum, &total);  // (its barriers order the defaults first)
   if (excl < remaining && remaining <= excl + cnt) {
     uint32_t cum = excl;
-    for (int i = 0; i < bpt; ++i) {
-      const uint32_t h = hist[top - i];
-      if (remaining <= cum + h) {
-        *s_digit = static_cast<uint32_t>(top - i);
-        *s_above = cum;
-        break;
+    bool done = false;
+#pragma unroll
+    for (int j = 0; j < kBpt; ++j) {
+      if (!done && remaining <= cum + h[j]) {
+        res[0] = static_cast<uint32_t>(kBpt * kThreads - 1 - static_cast<int>(threadIdx.x) * kBpt - j);
+        res[1] = cum;
+        res[2] = h[j];
+        done = true;
       }
-      cum += h;
+      cum += h[j];
     }
   }
   __syncthreads();
 }
 
-// Slots, in index order, of this thread's keys flagged in two sets (bit q =
-// key q of the thread: step q / 4, element q % 4 of the layout at key_pos).
-// Packed warp scans (four 8-bit step counts a word) order a warp's keys by
-// step, lane, element; one block scan orders the warps.
+// This thread's counts of a shared histogram in select_bin's order.
+__device__ __forceinline__ void my_bins4(const uint32_t* hist, uint32_t (&h)[4]) {
+  const uint4 v = *reinterpret_cast<const uint4*>(hist + kBins1 - 4 - 4 * threadIdx.x);
+  h[0] = v.w;
+  h[1] = v.z;
+  h[2] = v.y;
+  h[3] = v.x;
+}
+__device__ __forceinline__ void my_bins2(const uint32_t* hist, uint32_t (&h)[2]) {
+  const uint2 v = *reinterpret_cast<const uint2*>(hist + kBins3 - 2 - 2 * threadIdx.x);
+  h[0] = v.y;
+  h[1] = v.x;
+}
+
+// Packed step counts (a byte a step of kSteps keys-of-4): bit q of `f` is key
+// q of the thread (step q / 4, element q % 4 of the layout at key_pos).
+__device__ __forceinline__ uint32_t step_counts(uint32_t f) {
+  uint32_t c = 0;
+#pragma unroll
+  for (int i = 0; i < kSteps; ++i) c |= static_cast<uint32_t>(__popc((f >> (4 * i)) & 0xFu)) << (8 * i);
+  return c;
+}
+// The bytes of steps 0..i-1 of a packed word summed (i <= 4; a byte never
+// carries: a step has at most 128 keys a warp).
+__device__ __forceinline__ uint32_t bytes_before(uint32_t t, int i) {
+  const uint32_t low = i == 0 ? 0u : (t & (0xFFFFFFFFu >> (32 - 8 * i)));
+  return (low & 0xFFu) + ((low >> 8) & 0xFFu) + ((low >> 16) & 0xFFu) + (low >> 24);
+}
+__device__ __forceinline__ uint32_t byte_of(uint32_t w, int i) { return (w >> (8 * i)) & 0xFFu; }
+
+// Slots, in index order, of this thread's keys flagged in two sets (overflow
+// rows): packed warp scans order a warp's keys by step, lane, element; one
+// block scan orders the warps.
 struct Slots {
   uint32_t sa, sb;  // exclusive scans over lanes of the step counts (a byte a step)
   uint32_t ta, tb;  // the warp's step totals (a byte a step)
   uint32_t base;    // keys of earlier warps (a << 16 | b)
-  __device__ __forceinline__ static uint32_t field(uint32_t w, int i) { return (w >> (8 * i)) & 0xFFu; }
-  // the bytes of steps 0..i-1 summed (i <= 4; a byte never carries: a step
-  // has at most 128 keys a warp)
-  __device__ __forceinline__ static uint32_t before(uint32_t t, int i) {
-    const uint32_t low = i == 0 ? 0u : (t & (0xFFFFFFFFu >> (32 - 8 * i)));
-    return (low & 0xFFu) + ((low >> 8) & 0xFFu) + ((low >> 16) & 0xFFu) + (low >> 24);
-  }
   // slot (from the chunk's first key) of this thread's first set-a / set-b key of step i
-  __device__ __forceinline__ uint32_t a(int i) const { return (base >> 16) + before(ta, i) + field(sa, i); }
-  __device__ __forceinline__ uint32_t b(int i) const { return (base & 0xFFFFu) + before(tb, i) + field(sb, i); }
+  __device__ __forceinline__ uint32_t a(int i) const { return (base >> 16) + bytes_before(ta, i) + byte_of(sa, i); }
+  __device__ __forceinline__ uint32_t b(int i) const { return (base & 0xFFFFu) + bytes_before(tb, i) + byte_of(sb, i); }
 };
 
 // Fills *S for the flag sets fa, fb; returns the CTA's totals (a << 16 | b).
 __device__ __forceinline__ uint32_t order_slots(uint32_t fa, uint32_t fb, Slots* S, uint32_t* wsum) {
   static_assert(kSteps == 4, "one packed word of step counts");
   const int lane = lane_id(), warp = threadIdx.x >> 5;
-  uint32_t ca = 0, cb = 0;
-#pragma unroll
-  for (int i = 0; i < kSteps; ++i) {
-    ca |= static_cast<uint32_t>(__popc((fa >> (4 * i)) & 0xFu)) << (8 * i);
-    cb |= static_cast<uint32_t>(__popc((fb >> (4 * i)) & 0xFu)) << (8 * i);
-  }
+  const uint32_t ca = step_counts(fa), cb = step_counts(fb);
   const uint32_t ia = warp_incl_scan(ca), ib = warp_incl_scan(cb);
   S->sa = ia - ca;
   S->sb = ib - cb;
   S->ta = __shfl_sync(0xffffffffu, ia, 31);
   S->tb = __shfl_sync(0xffffffffu, ib, 31);
-  const uint32_t wa = Slots::before(S->ta, 4);  // the warp's totals
-  const uint32_t wb = Slots::before(S->tb, 4);
+  const uint32_t wa = bytes_before(S->ta, 4);  // the warp's totals
+  const uint32_t wb = bytes_before(S->tb, 4);
   if (lane == 0) wsum[warp] = (wa << 16) | wb;
   __syncthreads();
   if (warp == 0) {
@@ -194,41 +259,98 @@ struct RowSel {
   int64_t remap_ld;
   const uint32_t* hist_parts;  // the indexer's partial first-digit histograms, or null
   int hist_per_cta, hist_tpr;
+  uint32_t* err;
 };
 
 // Shared memory of one CTA (the same layout in every CTA of a cluster).
+template <int kListCap>
 struct TopkSmem {
-  uint32_t hist[kBins1];     // the row's first-digit histogram; later scratch for local counts
-  uint32_t hsum[kBins1];     // leader: the cluster's first-digit counts (when counted here)
-  uint32_t h2sum[kBins1];    // leader: the cluster's second-digit counts (overflow rows)
-  uint32_t h3sum[kBins3];    // leader: the cluster's third-digit counts
-  uint32_t wsum[kWarps + 1];
-  uint32_t res[8];
-  uint32_t meta[4];          // this CTA's list sizes and kept-key counts, read by the others
-  int32_t sure[kListCap];
-  int32_t selc[kListCap];
-  uint32_t ckey[kListCap];
-  int32_t cidx[kListCap];
+  uint32_t ent[kListCap];    // this CTA's keys with first digit >= D1, in index order (one word each)
+  uint32_t hist[kBins1];     // first-digit counts when counted here; overflow rows: second/third-digit counts
+  uint32_t hsum[kBins1];     // leader: the cluster's first-digit counts (counted here, C > 1)
+  uint32_t h2[kBins1];       // leader: the row's second-digit counts
+  uint32_t h3[kBins3];       // leader: the row's third-digit counts
+  uint32_t lh2[kBins1];      // this CTA's second-digit counts (C > 1)
+  uint32_t lh3[kBins3];      // this CTA's third-digit counts (C > 1)
+  uint32_t wsum[kWarps + 2];
+  uint32_t res[12];          // selected digits: [0..2] first, [3..5] second, [6..8] third
+  uint32_t kept[kMaxCluster];  // leader: each CTA's kept keys (keys > T << 16 | keys == T)
+  uint32_t wcnt[kWarps];     // a warp's keys > T and == T (gt << 16 | eq)
+  uint64_t kbar;             // clustered CTAs: the slice's bulk copy landed
+  int abort_flag;
 };
 
-__global__ void __launch_bounds__(kThreads, 2) topk_cluster_kernel(RowSel P) {
+// kCtaChunks: chunks a CTA of a cluster takes; kListCap: list entries;
+// kMinBlocks: CTAs an SM.  kStaged (the clustered instance): the CTA's slice
+// of the score row is copied into its list array first (one bulk copy, all
+// of it in flight at once) and the chunks are read from there; the list then
+// overwrites the slice from the front, never past the chunk being read.
+template <int kCtaChunks, int kListCap, int kMinBlocks>
+__global__ void __launch_bounds__(kThreads, kMinBlocks) topk_cluster_kernel(RowSel P) {
+  constexpr bool kStaged = kMinBlocks == 1;
+  static_assert(!kStaged || kCtaChunks * kChunk <= kListCap, "the slice fits the list array");
   pdl_wait();
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  TopkSmem& sm = *reinterpret_cast<TopkSmem*>(smem_raw);
+  TopkSmem<kListCap>& sm = *reinterpret_cast<TopkSmem<kListCap>*>(smem_raw);
   const int C = P.C;
   const uint32_t c = cluster_rank();
+  const bool lead = (c == 0);
   const int r = blockIdx.x / C;
   const int b = r / P.n_q, t = r % P.n_q;
-  const int L = min(max(__ldg(P.ctx_len + b), 0), P.s_max);
-  const int n = max(0, min(__ldg(P.q_pos0 + b) + P.t_off + t + 1, L));  // candidates s in [0, n)
-  int32_t* out = P.idx + static_cast<int64_t>(r) * P.k;
-  const int32_t* remap = P.remap ? P.remap + static_cast<int64_t>(r) * P.remap_ld : nullptr;
-  const float* row = P.scores + static_cast<int64_t>(r) * P.ld;
+  const int k = P.k;
   const int tid = threadIdx.x, lane = lane_id(), warp = tid >> 5;
-  auto emit = [&](int pos, int s) { out[pos] = remap ? __ldg(remap + s) : s; };
+  const float* row = P.scores + static_cast<int64_t>(r) * P.ld;
+  const int ctx = __ldg(P.ctx_len + b), pos0 = __ldg(P.q_pos0 + b);
 
-  if (n <= P.k) {  // the same in every CTA of the cluster: nobody syncs
-    for (int j = static_cast<int>(c) * kThreads + tid; j < P.k; j += C * kThreads) {
+  // ---- issued before the row length is known: the first digit's partial
+  // histograms
+  uint32_t h1[4] = {0u, 0u, 0u, 0u};
+  if (P.hist_parts != nullptr) {
+    // row r's key tiles [r tpr, (r + 1) tpr) were scored by the indexer CTAs
+    // i_lo..i_hi (runs of per_cta tiles); CTA i kept this row in slot 0 if
+    // its run starts in it, else in slot 1.  This thread sums its four bins.
+    const int64_t tile0 = static_cast<int64_t>(r) * P.hist_tpr;
+    const int i_lo = static_cast<int>(tile0 / P.hist_per_cta);
+    const int i_hi = static_cast<int>((tile0 + P.hist_tpr - 1) / P.hist_per_cta);
+    constexpr int kParts = 8;  // partials whose loads are in flight together
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    for (int i0 = i_lo; i0 <= i_hi; i0 += kParts) {
+      uint4 x[kParts];
+#pragma unroll
+      for (int u = 0; u < kParts; ++u) {
+        const int i = i0 + u;
+        const int slot = (static_cast<int64_t>(i) * P.hist_per_cta) / P.hist_tpr == r ? 0 : 1;
+        const uint4* src = reinterpret_cast<const uint4*>(P.hist_parts + (static_cast<int64_t>(i) * 2 + slot) * kBins1 +
+                                                          (kBins1 - 4 - 4 * tid));
+        x[u] = i <= i_hi ? __ldg(src) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kParts; ++u) {
+        v.x += x[u].x;
+        v.y += x[u].y;
+        v.z += x[u].z;
+        v.w += x[u].w;
+      }
+    }
+    h1[0] = v.w;
+    h1[1] = v.z;
+    h1[2] = v.y;
+    h1[3] = v.x;
+  }
+
+  const int L = min(max(ctx, 0), P.s_max);
+  const int n = max(0, min(pos0 + P.t_off + t + 1, L));  // candidates s in [0, n)
+  int32_t* out = P.idx + static_cast<int64_t>(r) * k;
+  const int32_t* remap = P.remap ? P.remap + static_cast<int64_t>(r) * P.remap_ld : nullptr;
+  // (a position at or past k only comes from a histogram that does not
+  // describe these scores)
+  auto emit = [&](uint32_t pos, int s) {
+    if (pos < static_cast<uint32_t>(k)) out[pos] = remap ? __ldg(remap + s) : s;
+    else raise_error(P.err, kErrHistMismatch);
+  };
+
+  if (n <= k) {  // the same in every CTA of the cluster: nobody syncs
+    for (int j = static_cast<int>(c) * kThreads + tid; j < k; j += C * kThreads) {
       if (j < n) emit(j, j);
       else out[j] = -1;
     }
@@ -236,22 +358,25 @@ __global__ void __launch_bounds__(kThreads, 2) topk_cluster_kernel(RowSel P) {
     return;
   }
 
-  // ---- the keys: with C > 1, CTA c takes the slice [c kSlice, (c + 1) kSlice)
-  // as two chunks; with C == 1 the CTA walks the row in chunks of kChunk keys.
+  // ---- the keys: with C > 1, CTA c takes kCtaChunks chunks from chunk
+  // c kCtaChunks; with C == 1 the CTA walks the row in chunks of kChunk keys.
   // In a chunk, warp w covers [w 32 kPer, (w + 1) 32 kPer) and step i of lane
   // l holds the four keys 4 (32 i + l) + e of that range.
   const int nch = C > 1 ? kCtaChunks : (n + kChunk - 1) / kChunk;
-  int cbase = C > 1 ? static_cast<int>(c) * kSlice : 0;
+  const int chunk0 = C > 1 ? static_cast<int>(c) * kCtaChunks : 0;  // the CTA's first chunk of the row
+  int cbase = chunk0 * kChunk;
   auto key_pos = [&](int i, int e) { return cbase + warp * (32 * kPer) + 4 * (32 * i + lane) + e; };
-  // (keys are loaded again where a later phase needs them, rather than kept
-  // live across the scans: the reloads hit L1/L2)
-  auto load_slice = [&](uint32_t* key) -> uint32_t {
+  // the keys of the chunk at `base` (this thread's kPer of them) and their
+  // validity; staged: from the slice in shared memory
+  const float* staged = reinterpret_cast<const float*>(sm.ent) - chunk0 * kChunk;  // (index by row position)
+  auto load_at = [&](int base, uint32_t* key) -> uint32_t {
     uint32_t m = 0;
 #pragma unroll
     for (int i = 0; i < kSteps; ++i) {
-      const int p0 = key_pos(i, 0);
+      const int p0 = base + warp * (32 * kPer) + 4 * (32 * i + lane);
       if (p0 + 4 <= n) {
-        const float4 f = __ldg(reinterpret_cast<const float4*>(row + p0));
+        const float4 f = kStaged ? *reinterpret_cast<const float4*>(staged + p0)
+                                 : __ldg(reinterpret_cast<const float4*>(row + p0));
         key[4 * i] = float_order_key(f.x);
         key[4 * i + 1] = float_order_key(f.y);
         key[4 * i + 2] = float_order_key(f.z);
@@ -261,57 +386,91 @@ __global__ void __launch_bounds__(kThreads, 2) topk_cluster_kernel(RowSel P) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const bool v = p0 + e < n;
-          key[4 * i + e] = v ? float_order_key(__ldg(row + p0 + e)) : 0u;
+          key[4 * i + e] = v ? float_order_key(kStaged ? staged[p0 + e] : __ldg(row + p0 + e)) : 0u;
           m |= (v ? 1u : 0u) << (4 * i + e);
         }
       }
     }
     return m;
   };
-  auto chunk = [&](int ch) { cbase = (C > 1 ? static_cast<int>(c) * kCtaChunks + ch : ch) * kChunk; };
+  auto load_slice = [&](uint32_t* key) -> uint32_t { return load_at(cbase, key); };
+  if constexpr (kStaged) {
+    // the slice [chunk0 kChunk, + kCtaChunks kChunk) clipped to the row (to a
+    // multiple of 4 keys: the row's storage is), in one bulk copy
+    if (tid == 0) {
+      sm.abort_flag = 0;
+      const uint32_t bar = smem_addr(&sm.kbar);
+      mbar_init(bar, 1);
+      fence_mbar_init();
+      const int lo = chunk0 * kChunk, hi = min(lo + kCtaChunks * kChunk, (n + 3) & ~3);
+      if (hi > lo) {
+        const uint32_t bytes = static_cast<uint32_t>(hi - lo) * 4u;
+        mbar_arrive_expect_tx(bar, bytes);
+        asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                         smem_addr(sm.ent)),
+                     "l"(row + lo), "r"(bytes), "r"(bar)
+                     : "memory");
+      } else {
+        mbar_arrive(bar);
+      }
+    }
+  }
+  // (staged) every thread waits for the slice before its first key read
+  bool have_slice = !kStaged;
+  auto wait_slice = [&]() {
+    if (kStaged && !have_slice) {
+      mbar_wait(smem_addr(&sm.kbar), 0, &sm.abort_flag, P.err);
+      have_slice = true;
+    }
+  };
+  auto chunk = [&](int ch) { cbase = (chunk0 + ch) * kChunk; };
   uint32_t key[kPer];
   uint32_t vm = 0;
-  for (int i = tid; i < kBins1; i += kThreads) {
-    sm.hist[i] = 0;
-    sm.hsum[i] = 0;
-    sm.h2sum[i] = 0;
-  }
-  for (int i = tid; i < kBins3; i += kThreads) sm.h3sum[i] = 0;
-  __syncthreads();
-  if (C > 1) cluster_sync();  // every CTA's sums are zero before any remote add
 
-  // ---- 1. first digit: the row's histogram in sm.hist of every CTA
-  if (P.hist_parts != nullptr) {
-    // row r's key tiles [r tpr, (r + 1) tpr) were scored by the indexer CTAs
-    // i_lo..i_hi (runs of per_cta tiles); CTA i kept this row in slot 0 if
-    // its run starts in it, else in slot 1
-    const int64_t tile0 = static_cast<int64_t>(r) * P.hist_tpr;
-    const int i_lo = static_cast<int>(tile0 / P.hist_per_cta);
-    const int i_hi = static_cast<int>((tile0 + P.hist_tpr - 1) / P.hist_per_cta);
-    constexpr int kBpt = kBins1 / kThreads;  // bins a thread
-    constexpr int kParts = 8;                // partials whose loads are in flight together
-    uint32_t v[kBpt];
-#pragma unroll
-    for (int j = 0; j < kBpt; ++j) v[j] = 0;
-    for (int i0 = i_lo; i0 <= i_hi; i0 += kParts) {
-      uint32_t x[kParts][kBpt];
-#pragma unroll
-      for (int u = 0; u < kParts; ++u) {
-        const int i = i0 + u;
-        const int slot = (static_cast<int64_t>(i) * P.hist_per_cta) / P.hist_tpr == r ? 0 : 1;
-        const uint32_t* src = P.hist_parts + (static_cast<int64_t>(i) * 2 + slot) * kBins1 + tid;
-#pragma unroll
-        for (int j = 0; j < kBpt; ++j) x[u][j] = i <= i_hi ? __ldg(src + j * kThreads) : 0u;
-      }
-#pragma unroll
-      for (int u = 0; u < kParts; ++u)
-#pragma unroll
-        for (int j = 0; j < kBpt; ++j) v[j] += x[u][j];
+  // Sums start at zero: the leader's (touched by the others only after the
+  // cluster barrier it arrives at once they are) and this CTA's own.
+  if (lead) {
+    for (int i = tid; i < kBins1; i += kThreads) {
+      sm.hsum[i] = 0;
+      sm.h2[i] = 0;
     }
-#pragma unroll
-    for (int j = 0; j < kBpt; ++j) sm.hist[tid + j * kThreads] = v[j];
-    __syncthreads();
-  } else {
+    for (int i = tid; i < kBins3; i += kThreads) sm.h3[i] = 0;
+  }
+  for (int i = tid; i < kBins1; i += kThreads) {
+    sm.lh2[i] = 0;
+    if (P.hist_parts == nullptr) sm.hist[i] = 0;
+  }
+  for (int i = tid; i < kBins3; i += kThreads) sm.lh3[i] = 0;
+  __syncthreads();
+  if (C > 1) cluster_arrive();
+  bool waited = (C == 1);
+  auto wait_zeroed = [&]() {  // before the first access to the leader's sums
+    if (!waited) {
+      cluster_wait();
+      waited = true;
+    }
+  };
+  // leave once nobody can still read the leader's shared memory: every CTA
+  // arrives, the leader waits (every CTA of a cluster calls this at the same
+  // point)
+  auto leave = [&]() {
+    pdl_trigger();
+    if (C > 1) {
+      cluster_arrive();
+      if (lead) cluster_wait();
+    }
+  };
+  // the counts do not add up (only with a mismatched histogram): flag, clear
+  // the row, leave
+  auto give_up = [&]() {
+    if (tid == 0) raise_error(P.err, kErrHistMismatch);
+    if (lead)
+      for (int j = tid; j < k; j += kThreads) out[j] = -1;
+  };
+
+  // ---- 1. first digit
+  if (P.hist_parts == nullptr) {
+    wait_slice();
     for (int ch = 0; ch < nch; ++ch) {
       chunk(ch);
       vm = load_slice(key);
@@ -321,177 +480,230 @@ __global__ void __launch_bounds__(kThreads, 2) topk_cluster_kernel(RowSel P) {
     }
     __syncthreads();
     if (C > 1) {
-      // merge into the leader, then every CTA copies the row's histogram
-      const uint32_t lead = map_rank(sm.hsum, 0);
+      // merge into the leader; every CTA reads the row's counts back
+      wait_zeroed();
+      const uint32_t lsum = map_rank(sm.hsum, 0);
       for (int i = tid; i < kBins1; i += kThreads)
-        if (sm.hist[i]) red_add_cluster(lead + 4u * i, sm.hist[i]);
+        if (sm.hist[i]) red_add_cluster(lsum + 4u * i, sm.hist[i]);
       cluster_sync();
-      for (int i = tid; i < kBins1; i += kThreads) sm.hist[i] = ld_cluster(lead + 4u * i);
-      __syncthreads();
+      const uint4 v = ld_cluster_v4(lsum + 4u * (kBins1 - 4 - 4 * tid));
+      h1[0] = v.w;
+      h1[1] = v.z;
+      h1[2] = v.y;
+      h1[3] = v.x;
+    } else {
+      my_bins4(sm.hist, h1);
     }
   }
-  select_bin(sm.hist, kBins1, static_cast<uint32_t>(P.k), sm.wsum, &sm.res[0], &sm.res[1]);
+  select_bin<4>(h1, static_cast<uint32_t>(k), sm.wsum, &sm.res[0]);
   const uint32_t D1 = sm.res[0];
   const uint32_t above1 = sm.res[1];  // sure keys of the row (first digit > D1)
-  const uint32_t ncand = sm.hist[D1];
-  const bool fits = ncand <= static_cast<uint32_t>(kListCap) && above1 <= static_cast<uint32_t>(kListCap) &&
-                    static_cast<uint32_t>(P.k) - above1 <= static_cast<uint32_t>(kListCap);
+  const uint32_t ncand = sm.res[2];   // keys in bin D1
+  if (D1 == kNoBin) {  // (every CTA read the same counts; none has touched the leader yet)
+    give_up();
+    wait_slice();  // (no CTA leaves with its bulk copy still landing)
+    pdl_trigger();
+    return;
+  }
+  // a CTA of a cluster lists at most its 16K keys; one CTA walking a whole
+  // row must fit the row's listed keys
+  const bool fits = C > 1 || above1 + ncand <= static_cast<uint32_t>(kListCap);
 
   if (fits) {
-    // ---- 2. sure keys and candidates of this CTA's keys, in index order
-    uint32_t own_s = 0, own_c = 0;
+    // ---- 2. this CTA's keys with first digit >= D1, in index order, into
+    // its list; the candidates' second digits counted on the way
+    uint32_t* my_h2 = C > 1 ? sm.lh2 : sm.h2;
+    uint32_t own = 0;
+    wait_slice();
     for (int ch = 0; ch < nch; ++ch) {
       chunk(ch);
       vm = load_slice(key);
-      uint32_t fs = 0, fc = 0;  // sure / candidate flags
+      uint32_t f = 0;
 #pragma unroll
-      for (int q = 0; q < kPer; ++q) {
-        const uint32_t d = key[q] >> 21;
-        fs |= (((vm >> q) & 1u) && d > D1) ? (1u << q) : 0u;
-        fc |= (((vm >> q) & 1u) && d == D1) ? (1u << q) : 0u;
+      for (int q = 0; q < kPer; ++q) f |= (((vm >> q) & 1u) && (key[q] >> 21) >= D1) ? (1u << q) : 0u;
+      const uint32_t cnt = step_counts(f);
+      const uint32_t inc = warp_incl_scan(cnt);
+      const uint32_t sl = inc - cnt;                                  // earlier lanes, a byte a step
+      const uint32_t tw = __shfl_sync(0xffffffffu, inc, 31);          // the warp's step totals
+      if (lane == 0) sm.wsum[warp] = bytes_before(tw, kSteps);
+      __syncthreads();
+      if (warp == 0) {
+        const uint32_t x = lane < kWarps ? sm.wsum[lane] : 0u;
+        const uint32_t xi = warp_incl_scan(x);
+        if (lane < kWarps) sm.wsum[lane] = xi - x;
+        if (lane == 31) sm.wsum[kWarps] = xi;  // the chunk's listed keys
       }
-      Slots S;
-      const uint32_t tot = order_slots(fs, fc, &S, sm.wsum);
+      __syncthreads();
+      const uint32_t wbase = own + sm.wsum[warp];
+      own += sm.wsum[kWarps];
 #pragma unroll
       for (int i = 0; i < kSteps; ++i) {
-        uint32_t ps = own_s + S.a(i), pc = own_c + S.b(i);
+        uint32_t p = wbase + bytes_before(tw, i) + byte_of(sl, i);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int q = 4 * i + e;
-          if ((fs >> q) & 1u) {
-            sm.sure[ps++] = key_pos(i, e);
-          } else if ((fc >> q) & 1u) {
-            const int sp = key_pos(i, e);
-            sm.ckey[pc] = float_order_key(__ldg(row + sp));
-            sm.cidx[pc] = sp;
-            ++pc;
+          if ((f >> q) & 1u) {
+            const bool sure = (key[q] >> 21) > D1;
+            const uint32_t d2 = (key[q] >> 10) & 0x7FFu;
+            if (!sure) atomicAdd(&my_h2[d2], 1u);
+            if (p < static_cast<uint32_t>(kListCap))
+              sm.ent[p] = (sure ? kSure : d2 << 19) | (static_cast<uint32_t>(ch) << 13) |
+                          static_cast<uint32_t>(key_pos(i, e) - cbase);
+            ++p;
           }
         }
       }
-      own_s += tot >> 16;
-      own_c += tot & 0xFFFFu;
+      // (the next chunk writes wsum only after its first barrier, which every
+      // warp reaches after these reads; staged: this chunk's entries land at
+      // or before its own keys, which every warp read before those barriers)
     }
-    if (tid == 0) {
-      sm.meta[0] = own_s;
-      sm.meta[1] = own_c;
+    own = min(own, static_cast<uint32_t>(kListCap));
+    __syncthreads();
+    auto entry_index = [&](uint32_t en) -> int {
+      return (chunk0 + static_cast<int>((en >> 13) & 0x3Fu)) * kChunk + static_cast<int>(en & kOffMask);
+    };
+
+    // ---- 3. second digit: the row's counts in the leader
+    if (C > 1) {
+      wait_zeroed();
+      const uint32_t l2 = map_rank(sm.h2, 0);
+      for (int i = tid; i < kBins1; i += kThreads)
+        if (sm.lh2[i]) red_add_cluster(l2 + 4u * i, sm.lh2[i]);
+      cluster_sync();
+    }
+    const uint32_t rem1 = static_cast<uint32_t>(k) - above1;
+    {
+      const uint4 v = ld_cluster_v4(map_rank(sm.h2, 0) + 4u * (kBins1 - 4 - 4 * tid));
+      uint32_t h[4] = {v.w, v.z, v.y, v.x};
+      select_bin<4>(h, rem1, sm.wsum, &sm.res[3]);
+    }
+    const uint32_t D2 = sm.res[3];
+    if (D2 == kNoBin) {
+      give_up();
+      leave();
+      return;
+    }
+    const uint32_t rem2 = rem1 - sm.res[4];
+    // third digit of this CTA's entries in bin D2 (few: their keys are read
+    // again), kept in place of their second digit; the row's counts in the leader
+    uint32_t* my_h3 = C > 1 ? sm.lh3 : sm.h3;
+    for (uint32_t i = tid; i < own; i += kThreads) {
+      const uint32_t en = sm.ent[i];
+      if (!(en & kSure) && ((en >> 19) & 0x7FFu) == D2) {
+        const int s_idx = entry_index(en);
+        const uint32_t d3 = s_idx < n ? float_order_key(__ldg(row + s_idx)) & 0x3FFu : 0u;
+        atomicAdd(&my_h3[d3], 1u);
+        sm.ent[i] = kHasD3 | (d3 << 19) | (en & ((0x3Fu << 13) | kOffMask));
+      }
     }
     __syncthreads();
     if (C > 1) {
-      cluster_sync();  // lists and counts published
-      if (c != 0) {
-        pdl_trigger();
-        cluster_sync();  // the leader reads our lists; we leave once it is done
-        return;
-      }
-      // ---- 3. (leader) append the other CTAs' lists, in rank order: every
-      // CTA's list sizes in one round of remote loads, their offsets by a
-      // warp scan, then all entries pulled at once (one thread an entry)
-      if (tid < 32) {
-        uint32_t ps_n = 0, pc_n = 0;
-        if (tid < C) {
-          const uint32_t mp = map_rank(sm.meta, tid);
-          ps_n = ld_cluster(mp);
-          pc_n = ld_cluster(mp + 4);
-        }
-        const uint32_t is = warp_incl_scan(ps_n), ic = warp_incl_scan(pc_n);
-        if (tid < C) {
-          sm.wsum[tid] = is - ps_n;                               // sure offsets of each CTA
-          reinterpret_cast<uint32_t*>(sm.selc)[tid] = ic - pc_n;  // candidate offsets (selc is free until the end)
-        }
-      }
-      __syncthreads();
-      const uint32_t* s_off = sm.wsum;
-      const uint32_t* c_off = reinterpret_cast<const uint32_t*>(sm.selc);
-      // entries [off(p), off(p + 1)) of the merged lists come from CTA p
-      for (uint32_t j = own_s + tid; j < above1; j += kThreads) {
-        int p = 1;
-        while (p + 1 < C && s_off[p + 1] <= j) ++p;
-        sm.sure[j] = static_cast<int32_t>(ld_cluster(map_rank(sm.sure, p) + 4u * (j - s_off[p])));
-      }
-      for (uint32_t j = own_c + tid; j < ncand; j += kThreads) {
-        int p = 1;
-        while (p + 1 < C && c_off[p + 1] <= j) ++p;
-        sm.ckey[j] = ld_cluster(map_rank(sm.ckey, p) + 4u * (j - c_off[p]));
-        sm.cidx[j] = static_cast<int32_t>(ld_cluster(map_rank(sm.cidx, p) + 4u * (j - c_off[p])));
-      }
-      __syncthreads();
-      cluster_arrive();  // done with the other CTAs' shared memory
+      const uint32_t l3 = map_rank(sm.h3, 0);
+      for (int i = tid; i < kBins3; i += kThreads)
+        if (sm.lh3[i]) red_add_cluster(l3 + 4u * i, sm.lh3[i]);
+      cluster_sync();
     }
-    // second and third digits from the candidates (all in this CTA now)
-    for (int i = tid; i < kBins1; i += kThreads) sm.hist[i] = 0;
-    __syncthreads();
-    for (uint32_t i = tid; i < ncand; i += kThreads) atomicAdd(&sm.hist[(sm.ckey[i] >> 10) & 0x7FFu], 1u);
-    __syncthreads();
-    const uint32_t rem1 = static_cast<uint32_t>(P.k) - above1;
-    select_bin(sm.hist, kBins1, rem1, sm.wsum, &sm.res[2], &sm.res[3]);
-    const uint32_t pref22 = (D1 << 11) | sm.res[2];
-    const uint32_t rem2 = rem1 - sm.res[3];
-    for (uint32_t i = tid; i < ncand; i += kThreads) {
-      const uint32_t kk = sm.ckey[i];
-      if ((kk >> 10) == pref22) atomicAdd(&sm.h3sum[kk & 0x3FFu], 1u);
+    {
+      const uint32_t l3 = map_rank(sm.h3, 0);
+      const uint2 v = make_uint2(ld_cluster(l3 + 4u * (kBins3 - 2 - 2 * tid)), ld_cluster(l3 + 4u * (kBins3 - 1 - 2 * tid)));
+      uint32_t h[2] = {v.y, v.x};
+      select_bin<2>(h, rem2, sm.wsum, &sm.res[6]);
+    }
+    const uint32_t D3 = sm.res[6];
+    if (D3 == kNoBin) {
+      give_up();
+      leave();
+      return;
+    }
+    const uint32_t take_eq = rem2 - sm.res[7];  // keys == T to keep, lowest index first
+
+    // ---- 4. kept keys: key > T, or key == T among the row's first take_eq of
+    // them.  This CTA's list, in index order, by warps taking G entries each;
+    // a kept key's output slot is the row's keys > T before it plus min(keys
+    // == T before it, take_eq).
+    auto classify = [&](uint32_t en) -> uint32_t {  // 2: key > T, 1: key == T, 0: below
+      if (en & kSure) return 2u;
+      const uint32_t d = (en >> 19) & 0x7FFu;
+      if (en & kHasD3) return d > D3 ? 2u : (d == D3 ? 1u : 0u);
+      return d > D2 ? 2u : 0u;  // (entries in bin D2 all carry their third digit)
+    };
+    const uint32_t G = (own + 32 * kWarps - 1) / (32 * kWarps) * 32;
+    const uint32_t g_lo = static_cast<uint32_t>(warp) * G, g_hi = min(g_lo + G, own);
+    {
+      uint32_t g = 0, e = 0;
+      for (uint32_t g0 = g_lo; g0 < g_hi; g0 += 32) {
+        const uint32_t gg = g0 + lane;
+        const uint32_t cl = gg < g_hi ? classify(sm.ent[gg]) : 0u;
+        g += __popc(__ballot_sync(0xffffffffu, cl == 2u));
+        e += __popc(__ballot_sync(0xffffffffu, cl == 1u));
+      }
+      if (lane == 0) sm.wcnt[warp] = (g << 16) | e;
     }
     __syncthreads();
-    select_bin(sm.h3sum, kBins3, rem2, sm.wsum, &sm.res[4], &sm.res[5]);
-    const uint32_t T = (pref22 << 10) | sm.res[4];
-    const uint32_t take_eq = rem2 - sm.res[5];  // keys == T to keep, lowest index first
-    pdl_trigger();
-    // selected candidates, in index order: key > T, or key == T among the
-    // first take_eq of them
-    constexpr int kCPT = kListCap / kThreads;  // candidates a thread, consecutive
-    const int c0 = tid * kCPT;
-    uint32_t gt = 0, eq = 0;
+    const uint32_t wc = lane < kWarps ? sm.wcnt[lane] : 0u;
+    const uint32_t wi = warp_incl_scan(wc);
+    const uint32_t mine = __shfl_sync(0xffffffffu, wi, 31);  // this CTA's keys > T, == T
+    uint32_t gt_off = 0, eq_off = 0, row_gt = mine >> 16, row_eq = mine & 0xFFFFu;
+    if (C > 1) {
+      // every CTA's counts through the leader: offsets from the lower ranks
+      const uint32_t lk = map_rank(sm.kept, 0);
+      if (tid == 0) st_cluster(lk + 4u * c, mine);
+      cluster_sync();
+      const uint32_t x = lane < C ? ld_cluster(lk + 4u * lane) : 0u;
+      const uint32_t xlo = lane < static_cast<int>(c) ? x : 0u;
+      uint32_t gs = x >> 16, es = x & 0xFFFFu, gl = xlo >> 16, el = xlo & 0xFFFFu;
 #pragma unroll
-    for (int e = 0; e < kCPT; ++e) {
-      const int i = c0 + e;
-      if (i < static_cast<int>(ncand)) {
-        gt += sm.ckey[i] > T ? 1u : 0u;
-        eq += sm.ckey[i] == T ? 1u : 0u;
+      for (int off = 1; off < 32; off <<= 1) {
+        gs += __shfl_xor_sync(0xffffffffu, gs, off);
+        es += __shfl_xor_sync(0xffffffffu, es, off);
+        gl += __shfl_xor_sync(0xffffffffu, gl, off);
+        el += __shfl_xor_sync(0xffffffffu, el, off);
+      }
+      row_gt = gs;
+      row_eq = es;
+      gt_off = gl;
+      eq_off = el;
+    }
+    if (row_gt + min(row_eq, take_eq) != static_cast<uint32_t>(k)) {
+      give_up();
+      leave();
+      return;
+    }
+    {
+      const uint32_t before = __shfl_sync(0xffffffffu, wi - wc, warp);  // earlier warps of this CTA
+      uint32_t gb = gt_off + (before >> 16), eb = eq_off + (before & 0xFFFFu);
+      const uint32_t lt = lanemask_lt();
+      for (uint32_t g0 = g_lo; g0 < g_hi; g0 += 32) {
+        const uint32_t gg = g0 + lane;
+        uint32_t cl = 0, s_idx = 0;
+        if (gg < g_hi) {
+          const uint32_t en = sm.ent[gg];
+          cl = classify(en);
+          s_idx = static_cast<uint32_t>(entry_index(en));
+        }
+        const uint32_t bg = __ballot_sync(0xffffffffu, cl == 2u), be = __ballot_sync(0xffffffffu, cl == 1u);
+        const uint32_t g_before = gb + __popc(bg & lt), e_before = eb + __popc(be & lt);
+        // (with a remap the key's list slot is written here and mapped below)
+        if (cl == 2u) out[g_before + min(e_before, take_eq)] = static_cast<int32_t>(s_idx);
+        else if (cl == 1u && e_before < take_eq) out[g_before + e_before] = static_cast<int32_t>(s_idx);
+        gb += __popc(bg);
+        eb += __popc(be);
       }
     }
-    uint32_t tt;
-    const uint32_t pre = block_excl_scan((gt << 16) | eq, sm.wsum, &tt);
-    uint32_t eq_rank = pre & 0xFFFFu;
-    uint32_t pos = (pre >> 16) + min(eq_rank, take_eq);
-#pragma unroll
-    for (int e = 0; e < kCPT; ++e) {
-      const int i = c0 + e;
-      if (i >= static_cast<int>(ncand)) break;
-      const uint32_t kk = sm.ckey[i];
-      if (kk > T) {
-        sm.selc[pos++] = sm.cidx[i];
-      } else if (kk == T) {
-        if (eq_rank < take_eq) sm.selc[pos++] = sm.cidx[i];
-        ++eq_rank;
-      }
+    if (remap != nullptr) {
+      // this CTA's kept keys fill the output slots [lo, hi)
+      __syncthreads();  // (this CTA's writes of out are visible to all its threads)
+      const uint32_t lo = gt_off + min(eq_off, take_eq);
+      const uint32_t hi = gt_off + (mine >> 16) + min(eq_off + (mine & 0xFFFFu), take_eq);
+      for (uint32_t j = lo + tid; j < hi; j += kThreads) out[j] = __ldg(remap + out[j]);
     }
-    __syncthreads();
-    // merge the two ascending lists: each entry's output slot is its own rank
-    // plus the number of entries of the other list below it
-    const int n_sure = static_cast<int>(above1);
-    const int n_sel = P.k - n_sure;
-    for (int i = tid; i < n_sure + n_sel; i += kThreads) {
-      const bool from_sure = i < n_sure;
-      const int j = from_sure ? i : i - n_sure;
-      const int sv = from_sure ? sm.sure[j] : sm.selc[j];
-      const int32_t* other = from_sure ? sm.selc : sm.sure;
-      int lo = 0, hi = from_sure ? n_sel : n_sure;  // count of `other` entries < sv
-      while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        if (other[mid] < sv) lo = mid + 1;
-        else hi = mid;
-      }
-      emit(j + lo, sv);
-    }
-    if (C > 1) cluster_wait();
+    leave();
     return;
   }
 
-  // ---- overflow: the remaining digits from histograms of every CTA's keys,
-  // merged in the leader (h2sum, h3sum; with C == 1 the CTA's own)
-  const uint32_t lead2 = map_rank(sm.h2sum, 0), lead3 = map_rank(sm.h3sum, 0);
-  // every thread has taken ncand from sm.hist before it is cleared: a warp
-  // that read a cleared bin would take the fits branch on its own
-  __syncthreads();
+  // ---- overflow (C == 1: one CTA walking a row whose listed keys exceed its
+  // list): the second and third digits from histograms of the row's keys,
+  // then the kept keys written chunk by chunk at running offsets
   for (int i = tid; i < kBins1; i += kThreads) sm.hist[i] = 0;
   __syncthreads();
   for (int ch = 0; ch < nch; ++ch) {
@@ -502,16 +714,19 @@ __global__ void __launch_bounds__(kThreads, 2) topk_cluster_kernel(RowSel P) {
       if (((vm >> q) & 1u) && (key[q] >> 21) == D1) atomicAdd(&sm.hist[(key[q] >> 10) & 0x7FFu], 1u);
   }
   __syncthreads();
-  for (int i = tid; i < kBins1; i += kThreads)
-    if (sm.hist[i]) red_add_cluster(lead2 + 4u * i, sm.hist[i]);
-  if (C > 1) cluster_sync();
-  else __syncthreads();
-  for (int i = tid; i < kBins1; i += kThreads) sm.hist[i] = ld_cluster(lead2 + 4u * i);
-  __syncthreads();
-  const uint32_t rem1 = static_cast<uint32_t>(P.k) - above1;
-  select_bin(sm.hist, kBins1, rem1, sm.wsum, &sm.res[2], &sm.res[3]);
-  const uint32_t pref22 = (D1 << 11) | sm.res[2];
-  const uint32_t rem2 = rem1 - sm.res[3];
+  const uint32_t rem1 = static_cast<uint32_t>(k) - above1;
+  {
+    uint32_t h[4];
+    my_bins4(sm.hist, h);
+    select_bin<4>(h, rem1, sm.wsum, &sm.res[3]);
+  }
+  if (sm.res[3] == kNoBin) {
+    give_up();
+    pdl_trigger();
+    return;
+  }
+  const uint32_t pref22 = (D1 << 11) | sm.res[3];
+  const uint32_t rem2 = rem1 - sm.res[4];
   for (int i = tid; i < kBins1; i += kThreads) sm.hist[i] = 0;
   __syncthreads();
   for (int ch = 0; ch < nch; ++ch) {
@@ -522,61 +737,20 @@ __global__ void __launch_bounds__(kThreads, 2) topk_cluster_kernel(RowSel P) {
       if (((vm >> q) & 1u) && (key[q] >> 10) == pref22) atomicAdd(&sm.hist[key[q] & 0x3FFu], 1u);
   }
   __syncthreads();
-  for (int i = tid; i < kBins3; i += kThreads)
-    if (sm.hist[i]) red_add_cluster(lead3 + 4u * i, sm.hist[i]);
-  if (C > 1) cluster_sync();
-  else __syncthreads();
-  for (int i = tid; i < kBins3; i += kThreads) sm.hist[i] = ld_cluster(lead3 + 4u * i);
-  __syncthreads();
-  select_bin(sm.hist, kBins3, rem2, sm.wsum, &sm.res[4], &sm.res[5]);
-  const uint32_t T = (pref22 << 10) | sm.res[4];
-  const uint32_t take_eq = rem2 - sm.res[5];
-  pdl_trigger();
-  // every CTA writes its kept keys: keys > T, and keys == T while fewer than
-  // take_eq have been kept; offsets from the lower-ranked CTAs' counts (C > 1)
-  // or from the earlier chunks (C == 1)
-  uint32_t gt_off = 0, eq_off = 0;
-  if (C > 1) {
-    uint32_t ng = 0, ne = 0;
-    for (int ch = 0; ch < nch; ++ch) {
-      chunk(ch);
-      vm = load_slice(key);
-#pragma unroll
-      for (int q = 0; q < kPer; ++q) {
-        ng += (((vm >> q) & 1u) && key[q] > T) ? 1u : 0u;
-        ne += (((vm >> q) & 1u) && key[q] == T) ? 1u : 0u;
-      }
-    }
-    uint32_t tt;
-    block_excl_scan((ng << 16) | ne, sm.wsum, &tt);
-    if (tid == 0) {
-      sm.meta[2] = tt >> 16;
-      sm.meta[3] = tt & 0xFFFFu;
-    }
-    __syncthreads();
-    cluster_sync();
-    if (tid < 32) {
-      uint32_t g = 0, e = 0;
-      if (tid < static_cast<int>(c)) {
-        const uint32_t mp = map_rank(sm.meta, tid);
-        g = ld_cluster(mp + 8);
-        e = ld_cluster(mp + 12);
-      }
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        g += __shfl_xor_sync(0xffffffffu, g, off);
-        e += __shfl_xor_sync(0xffffffffu, e, off);
-      }
-      if (tid == 0) {
-        sm.res[6] = g;
-        sm.res[7] = e;
-      }
-    }
-    __syncthreads();
-    gt_off = sm.res[6];
-    eq_off = sm.res[7];
-    cluster_arrive();  // done reading the other CTAs' counts
+  {
+    uint32_t h[2];
+    my_bins2(sm.hist, h);
+    select_bin<2>(h, rem2, sm.wsum, &sm.res[6]);
   }
+  if (sm.res[6] == kNoBin) {
+    give_up();
+    pdl_trigger();
+    return;
+  }
+  const uint32_t T = (pref22 << 10) | sm.res[6];
+  const uint32_t take_eq = rem2 - sm.res[7];
+  pdl_trigger();
+  uint32_t gt_off = 0, eq_off = 0;
   for (int ch = 0; ch < nch; ++ch) {
     chunk(ch);
     vm = load_slice(key);
@@ -606,25 +780,62 @@ __global__ void __launch_bounds__(kThreads, 2) topk_cluster_kernel(RowSel P) {
     gt_off += tot >> 16;
     eq_off += tot & 0xFFFFu;
   }
-  if (C > 1) cluster_wait();  // nobody leaves while another CTA may read its counts
+  if (tid == 0 && gt_off + min(eq_off, take_eq) != static_cast<uint32_t>(k)) raise_error(P.err, kErrHistMismatch);
 }
 
 }  // namespace
 
 size_t topk_workspace_bytes(int, int, int, int) { return 0; }
 
+namespace {
+// Launch one instance (cluster dimension C) with PDL; its attributes are set
+// once per device.
+template <int kCtaChunks, int kListCap, int kMinBlocks>
+dsa_status_t launch_topk(const RowSel& P, int64_t rows, int C, int device, cudaStream_t stream) {
+  auto kern = topk_cluster_kernel<kCtaChunks, kListCap, kMinBlocks>;
+  const size_t smem = sizeof(TopkSmem<kListCap>);
+  static bool attr_done[64] = {};
+  if (device < 0 || device >= 64) return DSA_ERR_UNSUPPORTED;
+  if (!attr_done[device]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    attr_done[device] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(rows * C), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(C);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1] = pdl_attribute();
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kern, P) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+}  // namespace
+
 dsa_status_t topk_radix(const TopkArgs& a) {
   const int64_t rows = static_cast<int64_t>(a.B) * a.n_q;
   if (rows == 0) return DSA_OK;
-  static_assert(kSlice < 65536, "per-CTA counts are packed in 16 bits");
-  static_assert(kListCap % kThreads == 0, "candidates a thread");
+  static_assert(kClusterSlice < 65536 && kListCapCluster < 65536 && kListCapRow < 65536,
+                "per-warp and per-CTA counts are packed in 16 bits");
+  static_assert(kClusterSlice <= kListCapCluster, "a CTA of a cluster lists at most its slice");
+  static_assert(kMaxCluster <= 32, "per-CTA counts summed by one warp");
+  static_assert(kMaxCluster * kClusterChunks <= 64, "a walking CTA's chunk fits the entry's 6-bit field");
   const int64_t n_max = std::max(1, a.s_max);
-  int64_t C = (n_max + kSlice - 1) / kSlice;
+  if (n_max > static_cast<int64_t>(kMaxCluster) * kClusterSlice) return DSA_ERR_UNSUPPORTED;
+  int64_t C = (n_max + kClusterSlice - 1) / kClusterSlice;
   // many rows (prefill rounds): a CTA a row, walking it in chunks, so that
   // many rows are in flight; few long rows (decode): a cluster a row
   if (rows >= 2LL * std::max(1, device_sm_count(a.device))) C = 1;
-  if (C > kMaxCluster) return DSA_ERR_UNSUPPORTED;
   if (rows * C > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  if (a.k <= 0) return DSA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(a.scores) & 15u) != 0 || (a.ld & 3) != 0) return DSA_ERR_INVALID_ARG;
   RowSel P;
   P.scores = a.scores;
@@ -642,32 +853,11 @@ dsa_status_t topk_radix(const TopkArgs& a) {
   P.hist_parts = a.hist_parts;
   P.hist_per_cta = a.hist_per_cta;
   P.hist_tpr = a.hist_tpr;
+  P.err = a.err;
   if (P.hist_parts != nullptr && (P.hist_per_cta <= 0 || P.hist_tpr <= 0)) return DSA_ERR_INVALID_ARG;
-  const size_t smem = sizeof(TopkSmem);
-  static bool attr_done[64] = {};
-  if (a.device < 0 || a.device >= 64) return DSA_ERR_UNSUPPORTED;
-  if (!attr_done[a.device]) {
-    if (cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess ||
-        cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
-            cudaSuccess)
-      return DSA_ERR_CUDA;
-    attr_done[a.device] = true;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(rows * C), 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = a.stream;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(C);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1] = pdl_attribute();
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, topk_cluster_kernel, P) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  if (P.hist_parts != nullptr && (reinterpret_cast<uintptr_t>(P.hist_parts) & 15u) != 0) return DSA_ERR_INVALID_ARG;
+  if (C == 1) return launch_topk<kClusterChunks, kListCapRow, 2>(P, rows, 1, a.device, a.stream);
+  return launch_topk<kClusterChunks, kListCapCluster, 1>(P, rows, static_cast<int>(C), a.device, a.stream);
 }
 
 }  // namespace dsa

@@ -234,14 +234,15 @@ def test_topk_many_long_rows_walked_in_chunks():
 
 
 @pytest.mark.parametrize("B,n_q,S", [
-    (1, 600, 65536),   # a prefill round: one CTA a row, eight 8K-key chunks
-    (24, 1, 131072),   # decode rows: a cluster of eight CTAs a row
+    (1, 600, 65536),   # a prefill round: one CTA a row, eight 8K-key chunks, lists overflow
+    (24, 1, 131072),   # decode rows: a cluster of four CTAs a row, every list thousands long
 ])
-def test_topk_every_row_on_the_overflow_path(B, n_q, S):
-    """Every row's candidate bin (the first 11 key bits) holds far more than
-    the 4096 keys the leader's lists take: scores inside [1, 2) on a grid of
-    2^-12 (a quarter of the keys a first-digit bin, thousands of exact
-    ties), a few rows of one value.  Exact against the oracle."""
+def test_topk_every_row_with_huge_candidate_bins(B, n_q, S):
+    """Every row's candidate bin (the first 11 key bits) holds a quarter of
+    the row: scores inside [1, 2) on a grid of 2^-12 (thousands of exact
+    ties), a few rows of one value.  One CTA walking a 64K row cannot list
+    them (the overflow path); a CTA of a cluster lists its whole slice.
+    Exact against the oracle."""
     g = np.random.default_rng(31)
     sc = (1.0 + g.integers(0, 4096, size=(B, n_q, S)) / 4096.0).astype(np.float32)
     sc[0, 0] = np.float32(1.25)
@@ -285,6 +286,26 @@ def test_indexer_topk_handoff_equals_plain_topk(lengths):
     plain = _gpu_scores(shape, t)
     for b, L in enumerate(lengths):
         torch.testing.assert_close(sc[b, :, :L], plain[b, :, :L], rtol=0, atol=0)
+    assert dsa.get_error()[0] == 0
+
+
+def test_topk_hist_from_another_call_is_reported():
+    """Histograms written by one indexer call handed to a top-k over another
+    call's scores: the top-k's own count checks flag DSA_ERR_HIST_MISMATCH
+    (bounds-checked: nothing outside the buffers is touched), and the next
+    matched pair is exact again."""
+    wl = workloads.get("decode32k")
+    shape = dsa.shape_from_workload(wl)
+    ta = workloads.make_inputs(wl, DEV, seed=17, attention=False)
+    tb = workloads.make_inputs(wl, DEV, seed=18, attention=False)
+    hist = torch.empty(dsa.workspace_bytes(shape, dsa.WS_HIST), dtype=torch.uint8, device=DEV)
+    dsa.indexer_scores_hist(shape, ta["q_idx"], ta["k_idx"], ta["w"], ta["ctx_len"], ta["q_pos0"], hist)
+    sc_b = _gpu_scores(shape, tb)
+    dsa.topk_hist(shape, sc_b, tb["ctx_len"], tb["q_pos0"], hist)
+    rc, word = dsa.get_error(clear=True)
+    assert rc == 7 and word & 4, (rc, word)
+    sc, got, want = _hist_pair(shape, tb)
+    torch.testing.assert_close(got, want, rtol=0, atol=0)
     assert dsa.get_error()[0] == 0
 
 
