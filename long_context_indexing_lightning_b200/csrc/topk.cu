@@ -263,9 +263,9 @@ struct RowSel {
 };
 
 // Shared memory of one CTA (the same layout in every CTA of a cluster).
-template <int kListCap>
+template <int kEntWords>
 struct TopkSmem {
-  uint32_t ent[kListCap];    // this CTA's keys with first digit >= D1, in index order (one word each)
+  uint32_t ent[kEntWords];   // this CTA's keys with first digit >= D1, in index order (one word each)
   uint32_t hist[kBins1];     // first-digit counts when counted here; overflow rows: second/third-digit counts
   uint32_t hsum[kBins1];     // leader: the cluster's first-digit counts (counted here, C > 1)
   uint32_t h2[kBins1];       // leader: the row's second-digit counts
@@ -282,16 +282,18 @@ struct TopkSmem {
 
 // kCtaChunks: chunks a CTA of a cluster takes; kListCap: list entries;
 // kMinBlocks: CTAs an SM.  kStaged (the clustered instance): the CTA's slice
-// of the score row is copied into its list array first (one bulk copy, all
-// of it in flight at once) and the chunks are read from there; the list then
-// overwrites the slice from the front, never past the chunk being read.
+// of the score row is copied into its list array one chunk above the front
+// (one bulk copy, all of it in flight at once) and the chunks are read from
+// there; after chunk ch the list holds at most (ch + 1) kChunk entries, so it
+// never reaches keys not yet listed (chunk ch's keys start at (ch + 1) kChunk).
 template <int kCtaChunks, int kListCap, int kMinBlocks>
 __global__ void __launch_bounds__(kThreads, kMinBlocks) topk_cluster_kernel(RowSel P) {
   constexpr bool kStaged = kMinBlocks == 1;
-  static_assert(!kStaged || kCtaChunks * kChunk <= kListCap, "the slice fits the list array");
+  constexpr int kEntWords = kStaged ? kCtaChunks * kChunk + kChunk : kListCap;
+  static_assert(!kStaged || kCtaChunks * kChunk <= kListCap, "a clustered CTA lists at most its slice");
   pdl_wait();
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  TopkSmem<kListCap>& sm = *reinterpret_cast<TopkSmem<kListCap>*>(smem_raw);
+  TopkSmem<kEntWords>& sm = *reinterpret_cast<TopkSmem<kEntWords>*>(smem_raw);
   const int C = P.C;
   const uint32_t c = cluster_rank();
   const bool lead = (c == 0);
@@ -368,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) topk_cluster_kernel(RowS
   auto key_pos = [&](int i, int e) { return cbase + warp * (32 * kPer) + 4 * (32 * i + lane) + e; };
   // the keys of the chunk at `base` (this thread's kPer of them) and their
   // validity; staged: from the slice in shared memory
-  const float* staged = reinterpret_cast<const float*>(sm.ent) - chunk0 * kChunk;  // (index by row position)
+  const float* staged = reinterpret_cast<const float*>(sm.ent + kChunk) - chunk0 * kChunk;  // (by row position)
   auto load_at = [&](int base, uint32_t* key) -> uint32_t {
     uint32_t m = 0;
 #pragma unroll
@@ -407,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) topk_cluster_kernel(RowS
         const uint32_t bytes = static_cast<uint32_t>(hi - lo) * 4u;
         mbar_arrive_expect_tx(bar, bytes);
         asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                         smem_addr(sm.ent)),
+                         smem_addr(sm.ent + kChunk)),
                      "l"(row + lo), "r"(bytes), "r"(bar)
                      : "memory");
       } else {
@@ -536,26 +538,38 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) topk_cluster_kernel(RowS
       __syncthreads();
       const uint32_t wbase = own + sm.wsum[warp];
       own += sm.wsum[kWarps];
+      auto put = [&](uint32_t p, uint32_t kk, int pos) {
+        const bool sure = (kk >> 21) > D1;
+        const uint32_t d2 = (kk >> 10) & 0x7FFu;
+        if (!sure) atomicAdd(&my_h2[d2], 1u);
+        if (p < static_cast<uint32_t>(kListCap))
+          sm.ent[p] = (sure ? kSure : d2 << 19) | (static_cast<uint32_t>(ch) << 13) | static_cast<uint32_t>(pos - cbase);
+      };
+      if constexpr (kStaged) {
+        // only the listed keys (a few per warp), read again from the slice
+        for (uint32_t ff = f; ff != 0u; ff &= ff - 1u) {
+          const int q = __ffs(ff) - 1, i = q >> 2, e = q & 3;
+          const uint32_t p = wbase + bytes_before(tw, i) + byte_of(sl, i) +
+                             static_cast<uint32_t>(__popc(f & ((1u << q) - 1u) & (0xFu << (4 * i))));
+          const int pos = key_pos(i, e);
+          put(p, float_order_key(staged[pos]), pos);
+        }
+      } else {
 #pragma unroll
-      for (int i = 0; i < kSteps; ++i) {
-        uint32_t p = wbase + bytes_before(tw, i) + byte_of(sl, i);
+        for (int i = 0; i < kSteps; ++i) {
+          uint32_t p = wbase + bytes_before(tw, i) + byte_of(sl, i);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int q = 4 * i + e;
-          if ((f >> q) & 1u) {
-            const bool sure = (key[q] >> 21) > D1;
-            const uint32_t d2 = (key[q] >> 10) & 0x7FFu;
-            if (!sure) atomicAdd(&my_h2[d2], 1u);
-            if (p < static_cast<uint32_t>(kListCap))
-              sm.ent[p] = (sure ? kSure : d2 << 19) | (static_cast<uint32_t>(ch) << 13) |
-                          static_cast<uint32_t>(key_pos(i, e) - cbase);
-            ++p;
+          for (int e = 0; e < 4; ++e) {
+            const int q = 4 * i + e;
+            if ((f >> q) & 1u) {
+              put(p, key[q], key_pos(i, e));
+              ++p;
+            }
           }
         }
       }
       // (the next chunk writes wsum only after its first barrier, which every
-      // warp reaches after these reads; staged: this chunk's entries land at
-      // or before its own keys, which every warp read before those barriers)
+      // warp reaches after these reads)
     }
     own = min(own, static_cast<uint32_t>(kListCap));
     __syncthreads();
@@ -793,7 +807,8 @@ namespace {
 template <int kCtaChunks, int kListCap, int kMinBlocks>
 dsa_status_t launch_topk(const RowSel& P, int64_t rows, int C, int device, cudaStream_t stream) {
   auto kern = topk_cluster_kernel<kCtaChunks, kListCap, kMinBlocks>;
-  const size_t smem = sizeof(TopkSmem<kListCap>);
+  constexpr int kEntWords = kMinBlocks == 1 ? kCtaChunks * kChunk + kChunk : kListCap;  // as in the kernel
+  const size_t smem = sizeof(TopkSmem<kEntWords>);
   static bool attr_done[64] = {};
   if (device < 0 || device >= 64) return DSA_ERR_UNSUPPORTED;
   if (!attr_done[device]) {
