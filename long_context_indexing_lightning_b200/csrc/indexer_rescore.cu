@@ -113,14 +113,22 @@ __global__ void __launch_bounds__(kThreads, 1) indexer_rescore_kernel(RsParams P
   // gather of tile j into stage st: lane l of warp w moves chunk l % 16 of
   // tile row 8 i + 2 w + l / 16 for i = 0..15; rows past the list are zero
   bool bad = false;
+  // (the sixteen list entries a lane needs are loaded first, all in flight
+  // together, then the copies issued)
   auto gather = [&](int j, int st) {
     const int c = lane & 15;
     const uint32_t base = sbase + C::kOffK + st * C::kKTile + (c >> 3) * kAtom;
-#pragma unroll 4
+    int sv[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int slot = j * kTileRows + i * 8 + warp * 2 + (lane >> 4);
+      sv[i] = slot < nvalid ? __ldg(cand + slot) : -1;
+    }
+#pragma unroll
     for (int i = 0; i < 16; ++i) {
       const int row = i * 8 + warp * 2 + (lane >> 4);
       const int slot = j * kTileRows + row;
-      int s = slot < nvalid ? __ldg(cand + slot) : -1;
+      int s = sv[i];
       if (slot < nvalid && (s < 0 || s >= L)) {  // a listed key outside the cache: zero row, flagged
         bad = true;
         s = -1;

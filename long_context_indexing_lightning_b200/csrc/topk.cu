@@ -871,6 +871,10 @@ dsa_status_t topk_radix(const TopkArgs& a) {
   P.err = a.err;
   if (P.hist_parts != nullptr && (P.hist_per_cta <= 0 || P.hist_tpr <= 0)) return DSA_ERR_INVALID_ARG;
   if (P.hist_parts != nullptr && (reinterpret_cast<uintptr_t>(P.hist_parts) & 15u) != 0) return DSA_ERR_INVALID_ARG;
+  // one CTA a row: few rows that fit a staged slice (short decode contexts,
+  // candidate lists) take the staged instance, many rows walk theirs
+  if (C == 1 && rows < 2LL * std::max(1, device_sm_count(a.device)) && n_max <= kClusterSlice)
+    return launch_topk<kClusterChunks, kListCapCluster, 1>(P, rows, 1, a.device, a.stream);
   if (C == 1) return launch_topk<kClusterChunks, kListCapRow, 2>(P, rows, 1, a.device, a.stream);
   return launch_topk<kClusterChunks, kListCapCluster, 1>(P, rows, static_cast<int>(C), a.device, a.stream);
 }
