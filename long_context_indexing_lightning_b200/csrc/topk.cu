@@ -64,6 +64,8 @@ constexpr uint32_t kNoBin = 0xFFFFFFFFu;   // select found no bin: the counts do
 constexpr uint32_t kSure = 1u << 31;       // list entry: first digit > D1
 constexpr uint32_t kHasD3 = 1u << 30;      // list entry: bits 19..29 hold the third digit
 constexpr uint32_t kOffMask = kChunk - 1;  // list entry: offset in the chunk
+constexpr uint32_t kPosMask = (0x3Fu << 13) | kOffMask;  // list entry: chunk and offset
+constexpr int kBndCap = 64;                // boundary keys (second digit == D2) a row resolves directly
 static_assert(kChunk == 8192, "13-bit chunk offsets");
 
 // ------------------------------------------------- distributed shared memory --
@@ -263,7 +265,7 @@ struct RowSel {
 };
 
 // Shared memory of one CTA (the same layout in every CTA of a cluster).
-template <int kEntWords>
+template <int kEntWords, int kBndCtas>
 struct TopkSmem {
   uint32_t ent[kEntWords];   // this CTA's keys with first digit >= D1, in index order (one word each)
   uint32_t hist[kBins1];     // first-digit counts when counted here; overflow rows: second/third-digit counts
@@ -276,6 +278,12 @@ struct TopkSmem {
   uint32_t res[12];          // selected digits: [0..2] first, [3..5] second, [6..8] third
   uint32_t kept[kMaxCluster];  // leader: each CTA's kept keys (keys > T << 16 | keys == T)
   uint32_t wcnt[kWarps];     // a warp's keys > T and == T (gt << 16 | eq)
+  uint2 bnd[kBndCtas * kBndCap];  // leader: each CTA's boundary keys (key, index), kBndCap a CTA
+  uint2 bk[kBndCap];         // the row's boundary keys, gathered from the leader
+  uint32_t bslot[kBndCap];   // list slots of this CTA's boundary keys
+  uint32_t kbc[kMaxCluster];  // kept boundary keys of each CTA
+  uint32_t bpre[kMaxCluster];  // first slot of each CTA's boundary keys in bk
+  uint32_t bcount, gdsum, found;
   uint64_t kbar;             // clustered CTAs: the slice's bulk copy landed
   int abort_flag;
 };
@@ -290,10 +298,11 @@ template <int kCtaChunks, int kListCap, int kMinBlocks>
 __global__ void __launch_bounds__(kThreads, kMinBlocks) topk_cluster_kernel(RowSel P) {
   constexpr bool kStaged = kMinBlocks == 1;
   constexpr int kEntWords = kStaged ? kCtaChunks * kChunk + kChunk : kListCap;
+  constexpr int kBndCtas = kStaged ? kMaxCluster : 1;  // (the walking instance runs one-CTA clusters)
   static_assert(!kStaged || kCtaChunks * kChunk <= kListCap, "a clustered CTA lists at most its slice");
   pdl_wait();
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  TopkSmem<kEntWords>& sm = *reinterpret_cast<TopkSmem<kEntWords>*>(smem_raw);
+  TopkSmem<kEntWords, kBndCtas>& sm = *reinterpret_cast<TopkSmem<kEntWords, kBndCtas>*>(smem_raw);
   const int C = P.C;
   const uint32_t c = cluster_rank();
   const bool lead = (c == 0);
@@ -443,6 +452,12 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) topk_cluster_kernel(RowS
     if (P.hist_parts == nullptr) sm.hist[i] = 0;
   }
   for (int i = tid; i < kBins3; i += kThreads) sm.lh3[i] = 0;
+  if (tid < kMaxCluster) sm.kbc[tid] = 0;
+  if (tid == 0) {
+    sm.bcount = 0;
+    sm.gdsum = 0;
+    sm.found = 0;
+  }
   __syncthreads();
   if (C > 1) cluster_arrive();
   bool waited = (C == 1);
@@ -598,39 +613,146 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) topk_cluster_kernel(RowS
       return;
     }
     const uint32_t rem2 = rem1 - sm.res[4];
-    // third digit of this CTA's entries in bin D2 (few: their keys are read
-    // again), kept in place of their second digit; the row's counts in the leader
-    uint32_t* my_h3 = C > 1 ? sm.lh3 : sm.h3;
-    for (uint32_t i = tid; i < own; i += kThreads) {
-      const uint32_t en = sm.ent[i];
-      if (!(en & kSure) && ((en >> 19) & 0x7FFu) == D2) {
-        const int s_idx = entry_index(en);
-        const uint32_t d3 = s_idx < n ? float_order_key(__ldg(row + s_idx)) & 0x3FFu : 0u;
-        atomicAdd(&my_h3[d3], 1u);
-        sm.ent[i] = kHasD3 | (d3 << 19) | (en & ((0x3Fu << 13) | kOffMask));
+    const uint32_t nb = sm.res[5];  // the row's keys in bin D2: the boundary
+    uint32_t D3 = 0, take_eq = 0, gt_off = 0, eq_off = 0;
+    bool offsets_known = false;
+    if (nb <= static_cast<uint32_t>(kBndCap)) {
+      // ---- 3'. few boundary keys: they travel with the counts.  Each CTA
+      // publishes its boundary keys (read again for their full key) and its
+      // count of keys certainly kept (sure, or second digit > D2); every CTA
+      // then finds T among the row's boundary keys, the ties it keeps (lowest
+      // index first), and its own output offset, with no further barrier.
+      uint32_t gd = 0;
+      const uint32_t lbnd = map_rank(sm.bnd, 0) + 8u * (c * kBndCap);
+      for (uint32_t i = tid; i < own; i += kThreads) {
+        const uint32_t en = sm.ent[i];
+        const uint32_t d = (en >> 19) & 0x7FFu;
+        if ((en & kSure) || d > D2) {
+          ++gd;
+        } else if (d == D2) {
+          const uint32_t j = atomicAdd(&sm.bcount, 1u);
+          const int s_idx = entry_index(en);
+          const uint32_t kk = s_idx < n ? float_order_key(__ldg(row + s_idx)) : 0u;
+          if (j < static_cast<uint32_t>(kBndCap)) {
+            sm.bslot[j] = i;
+            st_cluster(lbnd + 8u * j, kk);
+            st_cluster(lbnd + 8u * j + 4u, static_cast<uint32_t>(s_idx));
+          }
+        }
       }
+      gd = __reduce_add_sync(0xffffffffu, gd);
+      if (lane == 0 && gd) atomicAdd(&sm.gdsum, gd);
+      __syncthreads();
+      const uint32_t my_nb = min(sm.bcount, static_cast<uint32_t>(kBndCap));
+      if (tid == 0) st_cluster(map_rank(sm.kept, 0) + 4u * c, (sm.gdsum << 16) | my_nb);
+      if (C > 1) cluster_sync();
+      else __syncthreads();
+      // every CTA's counts and boundary keys
+      const uint32_t x = lane < C ? ld_cluster(map_rank(sm.kept, 0) + 4u * lane) : 0u;
+      const uint32_t xb = x & 0xFFFFu, xi = warp_incl_scan(xb);
+      const uint32_t nb_all = __shfl_sync(0xffffffffu, xi, 31);
+      if (nb_all != nb) {  // (the counts do not add up: a mismatched histogram)
+        give_up();
+        leave();
+        return;
+      }
+      if (warp == 0) {  // gather: lane l < C copies CTA l's boundary keys
+        if (lane < C) {
+          sm.bpre[lane] = xi - xb;
+          const uint32_t src = map_rank(sm.bnd, 0) + 8u * (lane * kBndCap);
+          for (uint32_t j = 0; j < xb; ++j)
+            sm.bk[xi - xb + j] = make_uint2(ld_cluster(src + 8u * j), ld_cluster(src + 8u * j + 4u));
+        }
+      }
+      __syncthreads();
+      // T: the rem2-th largest boundary key
+      if (tid < nb) {
+        const uint32_t kt = sm.bk[tid].x;
+        uint32_t gt = 0, eq = 0;
+        for (uint32_t j = 0; j < nb; ++j) {
+          gt += sm.bk[j].x > kt ? 1u : 0u;
+          eq += sm.bk[j].x == kt ? 1u : 0u;
+        }
+        if (gt < rem2 && rem2 <= gt + eq) {
+          sm.res[6] = kt;
+          sm.res[7] = rem2 - gt;  // keys == T kept
+          sm.found = 1;
+        }
+      }
+      __syncthreads();
+      if (!sm.found) {
+        give_up();
+        leave();
+        return;
+      }
+      const uint32_t T = sm.res[6], keep_eq = sm.res[7];
+      // which boundary keys are kept (ties: the lowest indices); each CTA's
+      // kept count, and this CTA's own boundary entries rewritten as sure or
+      // dropped (an entry with second digit 0 and no flags is never kept)
+      if (tid < nb) {
+        const uint2 e = sm.bk[tid];
+        bool kept = e.x > T;
+        if (e.x == T) {
+          uint32_t rank = 0;
+          for (uint32_t j = 0; j < nb; ++j) rank += (sm.bk[j].x == T && sm.bk[j].y < e.y) ? 1u : 0u;
+          kept = rank < keep_eq;
+        }
+        int cc = 0;  // the CTA whose keys slot tid holds
+        while (cc + 1 < C && sm.bpre[cc + 1] <= tid) ++cc;
+        if (kept) atomicAdd(&sm.kbc[cc], 1u);
+        if (cc == static_cast<int>(c)) {
+          const uint32_t slot = sm.bslot[tid - sm.bpre[cc]];
+          sm.ent[slot] = (kept ? kSure : 0u) | (sm.ent[slot] & kPosMask);
+        }
+      }
+      __syncthreads();
+      // this CTA's output offset: the kept keys of the lower-ranked CTAs
+      {
+        const uint32_t kept_l = lane < C ? (x >> 16) + sm.kbc[lane] : 0u;
+        const uint32_t ki = warp_incl_scan(kept_l);
+        gt_off = __shfl_sync(0xffffffffu, ki - kept_l, static_cast<int>(c));
+        if (__shfl_sync(0xffffffffu, ki, 31) != static_cast<uint32_t>(k)) {
+          give_up();
+          leave();
+          return;
+        }
+      }
+      offsets_known = true;
+    } else {
+      // third digit of this CTA's entries in bin D2 (their keys are read
+      // again), kept in place of their second digit; the row's counts in the
+      // leader
+      uint32_t* my_h3 = C > 1 ? sm.lh3 : sm.h3;
+      for (uint32_t i = tid; i < own; i += kThreads) {
+        const uint32_t en = sm.ent[i];
+        if (!(en & kSure) && ((en >> 19) & 0x7FFu) == D2) {
+          const int s_idx = entry_index(en);
+          const uint32_t d3 = s_idx < n ? float_order_key(__ldg(row + s_idx)) & 0x3FFu : 0u;
+          atomicAdd(&my_h3[d3], 1u);
+          sm.ent[i] = kHasD3 | (d3 << 19) | (en & kPosMask);
+        }
+      }
+      __syncthreads();
+      if (C > 1) {
+        const uint32_t l3 = map_rank(sm.h3, 0);
+        for (int i = tid; i < kBins3; i += kThreads)
+          if (sm.lh3[i]) red_add_cluster(l3 + 4u * i, sm.lh3[i]);
+        cluster_sync();
+      }
+      {
+        const uint32_t l3 = map_rank(sm.h3, 0);
+        const uint2 v = make_uint2(ld_cluster(l3 + 4u * (kBins3 - 2 - 2 * tid)), ld_cluster(l3 + 4u * (kBins3 - 1 - 2 * tid)));
+        uint32_t h[2] = {v.y, v.x};
+        select_bin<2>(h, rem2, sm.wsum, &sm.res[6]);
+      }
+      D3 = sm.res[6];
+      if (D3 == kNoBin) {
+        give_up();
+        leave();
+        return;
+      }
+      take_eq = rem2 - sm.res[7];  // keys == T to keep, lowest index first
     }
-    __syncthreads();
-    if (C > 1) {
-      const uint32_t l3 = map_rank(sm.h3, 0);
-      for (int i = tid; i < kBins3; i += kThreads)
-        if (sm.lh3[i]) red_add_cluster(l3 + 4u * i, sm.lh3[i]);
-      cluster_sync();
-    }
-    {
-      const uint32_t l3 = map_rank(sm.h3, 0);
-      const uint2 v = make_uint2(ld_cluster(l3 + 4u * (kBins3 - 2 - 2 * tid)), ld_cluster(l3 + 4u * (kBins3 - 1 - 2 * tid)));
-      uint32_t h[2] = {v.y, v.x};
-      select_bin<2>(h, rem2, sm.wsum, &sm.res[6]);
-    }
-    const uint32_t D3 = sm.res[6];
-    if (D3 == kNoBin) {
-      give_up();
-      leave();
-      return;
-    }
-    const uint32_t take_eq = rem2 - sm.res[7];  // keys == T to keep, lowest index first
-
     // ---- 4. kept keys: key > T, or key == T among the row's first take_eq of
     // them.  This CTA's list, in index order, by warps taking G entries each;
     // a kept key's output slot is the row's keys > T before it plus min(keys
@@ -657,8 +779,11 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) topk_cluster_kernel(RowS
     const uint32_t wc = lane < kWarps ? sm.wcnt[lane] : 0u;
     const uint32_t wi = warp_incl_scan(wc);
     const uint32_t mine = __shfl_sync(0xffffffffu, wi, 31);  // this CTA's keys > T, == T
-    uint32_t gt_off = 0, eq_off = 0, row_gt = mine >> 16, row_eq = mine & 0xFFFFu;
-    if (C > 1) {
+    uint32_t row_gt = mine >> 16, row_eq = mine & 0xFFFFu;
+    if (offsets_known) {
+      row_gt = static_cast<uint32_t>(k);  // (checked with the boundary counts)
+      row_eq = 0;
+    } else if (C > 1) {
       // every CTA's counts through the leader: offsets from the lower ranks
       const uint32_t lk = map_rank(sm.kept, 0);
       if (tid == 0) st_cluster(lk + 4u * c, mine);
@@ -808,7 +933,10 @@ template <int kCtaChunks, int kListCap, int kMinBlocks>
 dsa_status_t launch_topk(const RowSel& P, int64_t rows, int C, int device, cudaStream_t stream) {
   auto kern = topk_cluster_kernel<kCtaChunks, kListCap, kMinBlocks>;
   constexpr int kEntWords = kMinBlocks == 1 ? kCtaChunks * kChunk + kChunk : kListCap;  // as in the kernel
-  const size_t smem = sizeof(TopkSmem<kEntWords>);
+  constexpr int kBndCtas = kMinBlocks == 1 ? kMaxCluster : 1;
+  const size_t smem = sizeof(TopkSmem<kEntWords, kBndCtas>);
+  static_assert(kMinBlocks == 1 || 2 * (sizeof(TopkSmem<kEntWords, kBndCtas>) + 1024) <= 233472,
+                "two CTAs an SM");
   static bool attr_done[64] = {};
   if (device < 0 || device >= 64) return DSA_ERR_UNSUPPORTED;
   if (!attr_done[device]) {
