@@ -531,13 +531,33 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) topk_cluster_kernel(RowS
     // its list; the candidates' second digits counted on the way
     uint32_t* my_h2 = C > 1 ? sm.lh2 : sm.h2;
     uint32_t own = 0;
+    // (staged) the test "first digit >= D1" on a float's raw bits b: the order
+    // key is b | 2^31 for b >= 0 and ~b for b < 0 (-0 mapped like +0), so it
+    // holds iff b >= pos_min (non-negative b) or b <= neg_max (negative b)
+    const uint32_t K0 = D1 << 21;
+    const uint32_t pos_min = K0 >= 0x80000000u ? K0 - 0x80000000u : 0u;
+    const uint32_t neg_max = K0 == 0x80000000u ? 0x80000000u : ~K0;  // (K0 > 2^31: ~K0 < 2^31, no negative b)
     wait_slice();
     for (int ch = 0; ch < nch; ++ch) {
       chunk(ch);
-      vm = load_slice(key);
       uint32_t f = 0;
+      if constexpr (kStaged) {
 #pragma unroll
-      for (int q = 0; q < kPer; ++q) f |= (((vm >> q) & 1u) && (key[q] >> 21) >= D1) ? (1u << q) : 0u;
+        for (int i = 0; i < kSteps; ++i) {
+          const int p0 = key_pos(i, 0);
+          const uint4 u = *reinterpret_cast<const uint4*>(staged + p0);  // (past n: masked below)
+          const uint32_t b[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const bool hit = static_cast<int32_t>(b[e]) >= 0 ? b[e] >= pos_min : b[e] <= neg_max;
+            f |= (hit && p0 + e < n) ? (1u << (4 * i + e)) : 0u;
+          }
+        }
+      } else {
+        vm = load_slice(key);
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) f |= (((vm >> q) & 1u) && (key[q] >> 21) >= D1) ? (1u << q) : 0u;
+      }
       const uint32_t cnt = step_counts(f);
       const uint32_t inc = warp_incl_scan(cnt);
       const uint32_t sl = inc - cnt;                                  // earlier lanes, a byte a step
