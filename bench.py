@@ -348,11 +348,40 @@ def run_ours(args, wl):
                     "ms_per_step": e2e["ms"],
                     # this box's pinned copy rates: the step cannot run faster than its own copies
                     "copy": e2e["copy"],
-                    "copy_bound_per_s": q_total / (max(e2e["copy"]["both_ms_per_step"], ms_per_step) * 1e-3)},
+                    "copy_bound_per_s": q_total / (max(e2e["copy"]["both_ms_per_step"], ms_per_step) * 1e-3),
+                    # host time to enqueue one step (the calls return before the work ends): a step
+                    # whose issue time exceeds its device time is bound by the host
+                    "host_issue_ms_per_step": e2e["host_issue_ms"],
+                    # host buffers pinned after binding to the GPU's nearest CPUs (their count), or null
+                    "near_gpu_cpus": e2e["near_cpus"]},
         }
     if ws > 1:
         torch.distributed.destroy_process_group()
     return res
+
+
+def _bind_near_gpu(dev):
+    """Restrict this process to the CPUs nearest the GPU (NVML's affinity set
+    for it), so the host buffers pinned afterwards are allocated on the GPU's
+    NUMA node: pinned memory on the far socket slows the GPU's reads of it
+    (host -> device copies) well below the link rate.  A host-side setting of
+    this process only; returns the CPU count bound to, or None if NVML cannot
+    tell."""
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        p = torch.cuda.get_device_properties(dev)
+        bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+        h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        words = pynvml.nvmlDeviceGetCpuAffinity(h, (os.cpu_count() + 63) // 64)
+        cpus = {w * 64 + b for w, m in enumerate(words) for b in range(64) if (m >> b) & 1}
+        cpus &= set(range(os.cpu_count()))
+        if not cpus:
+            return None
+        os.sched_setaffinity(0, cpus)
+        return len(cpus)
+    except Exception:
+        return None
 
 
 def _e2e(args, wl, dsa, shape, t, k_idx, k_scale, dev, stream, k_ref=None):
@@ -361,6 +390,8 @@ def _e2e(args, wl, dsa, shape, t, k_idx, k_scale, dev, stream, k_ref=None):
     runs under the next step's indexer and top-k), caches resident on the
     device.  The timed region ends when the last step's output is in host
     memory."""
+    all_cpus = os.sched_getaffinity(0)
+    near = _bind_near_gpu(dev)
     pin = lambda x: x.cpu().pin_memory()
     h = {k: pin(t[k]) for k in ("q_idx", "w", "q", "ctx_len", "q_pos0")}
     h_out = torch.empty(wl.batch, wl.n_q, wl.heads, wl.d_v, dtype=t["q"].dtype).pin_memory()
@@ -374,15 +405,20 @@ def _e2e(args, wl, dsa, shape, t, k_idx, k_scale, dev, stream, k_ref=None):
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize(dev)
     s.record(stream)
+    t_issue = time.perf_counter()
     for _ in range(args.steps):
         call()
+    t_issue = time.perf_counter() - t_issue  # host time to enqueue the steps (diagnostic)
     stream.wait_event(done)  # the last step's output is in host memory
     e.record(stream)
     torch.cuda.synchronize(dev)
     h2d = sum(v.numel() * v.element_size() for v in h.values())
     d2h = h_out.numel() * h_out.element_size()
     ms = s.elapsed_time(e) / args.steps
-    return {"ms": ms, "h2d": h2d, "d2h": d2h, "copy": _copy_rates(h["q"], h_out, dev)}
+    copy = _copy_rates(h["q"], h_out, dev)
+    os.sched_setaffinity(0, all_cpus)  # (the pinned pages stay where they were placed)
+    return {"ms": ms, "h2d": h2d, "d2h": d2h, "copy": copy,
+            "host_issue_ms": t_issue * 1e3 / args.steps, "near_cpus": near}
 
 
 def _copy_rates(h_in, h_out, dev, reps=10):

@@ -351,8 +351,12 @@ dsa_status_t dsa_forward(const dsa_shape_t *shape,
 /*
  * dsa_forward with the per-step tensors in HOST memory: q_idx, w, q,
  * ctx_len, q_pos0 (inputs) and out, lse (outputs; lse may be NULL) are HOST
- * pointers (page-locked memory gives asynchronous copies), while the caches
- * k_idx, k_scale, k_rescore, kv, v stay on the device as the layer's resident state.
+ * pointers (page-locked memory gives asynchronous copies; pinned on the
+ * GPU's own NUMA node -- e.g. allocated from a thread bound to the CPUs
+ * NVML reports as nearest the GPU -- host-to-device copies run at the link
+ * rate, pinned on the far socket they can run at a fraction of it), while
+ * the caches k_idx, k_scale, k_rescore, kv, v stay on the device as the
+ * layer's resident state.
  * The call copies the inputs in (one cudaMemcpyAsync each), runs the step,
  * copies the outputs back and synchronises `stream` before returning.
  * workspace: dsa_workspace_bytes(shape, DSA_WS_FORWARD_HOST) bytes: the

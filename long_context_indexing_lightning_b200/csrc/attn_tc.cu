@@ -794,22 +794,45 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
                                                            const float* __restrict__ part_ml,
                                                            __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
   constexpr int splits = kS;
+  constexpr int kBatch = kS < 8 ? kS : 8;  // splits whose loads are in flight together
   pdl_wait();
   __shared__ float coef[kMaxSplits][kCombineHeads];
   const int r = blockIdx.x;
   const int h0 = blockIdx.y * kCombineHeads;
   const int tid = threadIdx.x;
+  constexpr int kItr = kCombineHeads * (kDv / 4) / 256;  // output positions a thread
+  auto load_batch = [&](int i0, float4 (&o)[kItr][kBatch]) {
+#pragma unroll
+    for (int itr = 0; itr < kItr; ++itr) {
+      const int x = itr * 256 + tid;
+      const int h = h0 + x / (kDv / 4);
+      const int c4 = x % (kDv / 4);
+      const int hv = c4 / (kDvHalf / 4);
+      const int cc = (c4 % (kDvHalf / 4)) * 4;
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        if (i0 + i < kS) {
+          const int64_t it = (static_cast<int64_t>(r) * splits + i0 + i) * 2 + hv;
+          o[itr][i] = __ldg(reinterpret_cast<const float4*>(part_o + (it * kH + h) * kDvHalf + cc));
+        }
+      }
+    }
+  };
+  // the first batch of partial outputs is loaded before the weights are
+  // formed (it does not depend on them), so the two overlap
+  float4 o[kItr][kBatch];
+  load_batch(0, o);
   if (tid < kCombineHeads) {
     const int h = h0 + tid;
     float M = -INFINITY;
-    for (int i = 0; i < splits; ++i) {
+    for (int i = 0; i < kS; ++i) {
       const int64_t it = static_cast<int64_t>(r) * splits + i;
       const float m = part_ml[(it * 2 + 0) * kH + h];
       const float l = part_ml[(it * 2 + 1) * kH + h];
       if (l > 0.f) M = fmaxf(M, m);
     }
     float Ls = 0.f;
-    for (int i = 0; i < splits; ++i) {
+    for (int i = 0; i < kS; ++i) {
       const int64_t it = static_cast<int64_t>(r) * splits + i;
       const float m = part_ml[(it * 2 + 0) * kH + h];
       const float l = part_ml[(it * 2 + 1) * kH + h];
@@ -818,45 +841,40 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restri
       Ls += wgt * l;
     }
     const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-    for (int i = 0; i < splits; ++i) coef[i][tid] *= inv;
+    for (int i = 0; i < kS; ++i) coef[i][tid] *= inv;
     if (lse != nullptr)
       lse[static_cast<int64_t>(r) * kH + h] = Ls > 0.f ? (M + log2f(Ls)) * 0.6931471805599453f : -INFINITY;
   }
   __syncthreads();
-  constexpr int kItr = kCombineHeads * (kDv / 4) / 256;  // output positions a thread
-  float4 o[kItr][kS];
+  float4 acc[kItr];
 #pragma unroll
-  for (int itr = 0; itr < kItr; ++itr) {
-    const int x = itr * 256 + tid;
-    const int hl = x / (kDv / 4);
-    const int c4 = x % (kDv / 4);
-    const int h = h0 + hl;
-    const int hv = c4 / (kDvHalf / 4);
-    const int cc = (c4 % (kDvHalf / 4)) * 4;
+  for (int itr = 0; itr < kItr; ++itr) acc[itr] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int i = 0; i < kS; ++i) {
-      const int64_t it = (static_cast<int64_t>(r) * splits + i) * 2 + hv;
-      o[itr][i] = __ldg(reinterpret_cast<const float4*>(part_o + (it * kH + h) * kDvHalf + cc));
+  for (int i0 = 0; i0 < kS; i0 += kBatch) {
+    if (i0 > 0) load_batch(i0, o);
+#pragma unroll
+    for (int itr = 0; itr < kItr; ++itr) {
+      const int hl = (itr * 256 + tid) / (kDv / 4);
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        if (i0 + i < kS) {
+          const float c = coef[i0 + i][hl];
+          acc[itr].x = fmaf(c, o[itr][i].x, acc[itr].x);
+          acc[itr].y = fmaf(c, o[itr][i].y, acc[itr].y);
+          acc[itr].z = fmaf(c, o[itr][i].z, acc[itr].z);
+          acc[itr].w = fmaf(c, o[itr][i].w, acc[itr].w);
+        }
+      }
     }
   }
 #pragma unroll
   for (int itr = 0; itr < kItr; ++itr) {
     const int x = itr * 256 + tid;
-    const int hl = x / (kDv / 4);
+    const int h = h0 + x / (kDv / 4);
     const int c4 = x % (kDv / 4);
-    const int h = h0 + hl;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int i = 0; i < kS; ++i) {
-      const float c = coef[i][hl];
-      acc.x = fmaf(c, o[itr][i].x, acc.x);
-      acc.y = fmaf(c, o[itr][i].y, acc.y);
-      acc.z = fmaf(c, o[itr][i].z, acc.z);
-      acc.w = fmaf(c, o[itr][i].w, acc.w);
-    }
     uint2 v;
-    v.x = pack_bf16(acc.x, acc.y);
-    v.y = pack_bf16(acc.z, acc.w);
+    v.x = pack_bf16(acc[itr].x, acc[itr].y);
+    v.y = pack_bf16(acc[itr].z, acc[itr].w);
     *reinterpret_cast<uint2*>(out + (static_cast<int64_t>(r) * kH + h) * kDv + c4 * 4) = v;
   }
 }
