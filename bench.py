@@ -659,6 +659,66 @@ def run_topk_structures(args):
             "cases": out, "gpu_launches": args.steps * len(cases)}
 
 
+def run_proj(args):
+    """The indexer projections alone (tensor-core GEMMs, synthetic seeded
+    weights): wq_b on the query latent (1536 -> 64 x 128) and the fused index-
+    key + weights_proj projection of the hidden state (7168 -> 128 + 64), for
+    a decode step's 32 tokens and a 4096-token prefill round.  Reports each
+    case's time and TFLOP/s against the bf16 tensor peak, and the bytes moved
+    against HBM (the weight-bound decode case)."""
+    import long_context_indexing_lightning_b200 as dsa
+
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    hbm, tf, tf_sus, src = _peaks()
+    shape = dsa.make_shape(1, 1, 1024)
+    g = torch.Generator(device=dev).manual_seed(0)
+    rnd = lambda *sh, std=1.0: (torch.randn(*sh, generator=g, device=dev) * std).to(torch.bfloat16)
+    wq = rnd(64 * 128, 1536, std=1536 ** -0.5)
+    wkw = rnd(192, 7168, std=7168 ** -0.5)
+    out = {}
+    for T in (32, 4096):
+        lat, x = rnd(T, 1536), rnd(T, 7168)
+        q_idx = torch.empty(T, 64, 128, dtype=torch.bfloat16, device=dev)
+        k_new = torch.empty(T, 128, dtype=torch.bfloat16, device=dev)
+        w = torch.empty(T, 64, dtype=torch.float32, device=dev)
+        cases = {
+            f"wq_b T={T}": (lambda: dsa.indexer_proj_q(shape, lat, wq, q_idx=q_idx),
+                           2 * T * 1536 * 8192, (T * 1536 + 8192 * 1536 + T * 8192) * 2),
+            f"key+weights T={T}": (lambda: dsa.indexer_proj_kw(shape, x, wkw, k_new=k_new, w=w),
+                                  2 * T * 7168 * 192, (T * 7168 + 192 * 7168) * 2 + T * (128 * 2 + 64 * 4)),
+        }
+        for name, (call, flops, nbytes) in cases.items():
+            for _ in range(args.warmup):
+                call()
+            torch.cuda.synchronize(dev)
+            s_, e_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s_.record()
+            for _ in range(args.steps):
+                call()
+            e_.record()
+            torch.cuda.synchronize(dev)
+            ms = max_over_ranks(s_.elapsed_time(e_) / args.steps, dev)
+            out[name] = {"us": ms * 1e3, "tflops": flops / (ms * 1e-3) / 1e12,
+                         "frac_tensor": flops / (ms * 1e-3) / 1e12 / tf, "frac_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm}
+    rc, word = dsa.get_error(clear=True)
+    if rc != 0:
+        raise RuntimeError(f"device error word {word:#x}")
+    if rank != 0:
+        return None
+    main_case = out["wq_b T=4096"]
+    return {"metric": "indexer projection TFLOP/s (wq_b, 4096 tokens)", "value": main_case["tflops"],
+            "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": main_case["us"] * 1e-3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded weights and activations)",
+            "config": {"workload": "indexer projections: wq_b 1536->8192, key+weights 7168->192; 32 and 4096 tokens"},
+            "roofline": {"kernel": "proj_gemm", "bound": "tensor", "peak": tf, "unit": "TFLOP/s",
+                         "achieved": main_case["tflops"], "frac": main_case["frac_tensor"],
+                         "peak_source": f"{src} bf16_tflops (of {src})", "traffic": None},
+            "cases": out, "gpu_launches": args.steps * 4}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -670,9 +730,9 @@ def main():
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling runs)")
     ap.add_argument("--ctx", type=int, default=0, help="override the workload's cache length (profiling runs)")
     ap.add_argument("--q-chunk", type=int, default=4096, help="prefill: queries per indexer/top-k/attention round")
-    ap.add_argument("--op", default="step", choices=["step", "append", "topk"],
+    ap.add_argument("--op", default="step", choices=["step", "append", "topk", "proj"],
                     help="step: the layer step (default); append: the cache append of one prefill chunk; "
-                         "topk: top-k alone on structured 128K rows")
+                         "topk: top-k alone on structured 128K rows; proj: the indexer projections alone")
     ap.add_argument("--append-tokens", type=int, default=65536)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
@@ -685,8 +745,8 @@ def main():
         if workloads.get(args.workload).n_q > 1:
             over["n_q"] = args.ctx
     wl = workloads.get(args.workload, **over)
-    if args.op in ("append", "topk") and args.impl == "ours":
-        line = run_append(args) if args.op == "append" else run_topk_structures(args)
+    if args.op in ("append", "topk", "proj") and args.impl == "ours":
+        line = {"append": run_append, "topk": run_topk_structures, "proj": run_proj}[args.op](args)
         if line is not None:
             print(json.dumps(line), flush=True)
         return
