@@ -610,10 +610,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
       fence_proxy_async_smem();  // generic writes -> bulk-copy reads
       mbar_arrive(xout_written);
     };
-    // validity of this lane's row in tiles [vbase, vbase + 32), loaded in
-    // batches so that no global load is pending inside the loop
-    uint32_t vbits = 0;
-    int vbase = -32;
+    // validity of this lane's row in tiles [j0, j0 + 32): the 32 list entries
+    // are loaded together (one memory round trip), the first batch before
+    // the wait for tile 0's logits, where it overlaps the first gather
+    auto load_valid = [&](int j0) {
+      int ix[32];
+#pragma unroll
+      for (int t = 0; t < 32; ++t) {
+        const int rr = (j0 + t) * kRows + kh * 32 + lane;
+        ix[t] = (j0 + t < T && rr < nrows) ? __ldg(sel + rr) : -1;
+      }
+      uint32_t bits = 0;
+#pragma unroll
+      for (int t = 0; t < 32; ++t) bits |= ((ix[t] >= 0 && ix[t] < L) ? 1u : 0u) << t;
+      return bits;
+    };
+    uint32_t vbits = load_valid(0);
+    int vbase = 0;
     if (T > 0) {
       if (!mbar_wait_warp(s_full, 0, abort_flag, P.err)) {
         ok = false;
@@ -626,12 +639,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
       const int bb = j & 1;
       if (j >= vbase + 32) {
         vbase = j;
-        vbits = 0;
-        for (int t = 0; t < 32 && j + t < T; ++t) {
-          const int rr = (j + t) * kRows + kh * 32 + lane;
-          const int ix = rr < nrows ? __ldg(sel + rr) : -1;
-          vbits |= ((ix >= 0 && ix < L) ? 1u : 0u) << t;
-        }
+        vbits = load_valid(j);
       }
       const uint32_t valid = __ballot_sync(0xffffffffu, ((vbits >> (j - vbase)) & 1u) != 0);
       // tile j + 1's partial goes out first, from every warp at the same
