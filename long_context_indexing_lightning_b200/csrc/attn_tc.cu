@@ -81,6 +81,9 @@ constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 16 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory");
 static_assert(kStageBytes % 1024 == 0, "ring stages must stay 1024-aligned");
+// output staging: one slot per softmax warp in the ring, 32 rows of 144 bytes
+constexpr int kOutSlotBytes = 32 * 144;
+static_assert(kSoftWarps * kOutSlotBytes <= kStages * kStageBytes, "output staging fits in the ring");
 
 struct AttnParams {
   const uint16_t* q;        // [R][128][576] bf16
@@ -258,6 +261,16 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 template <int N>
 __device__ __forceinline__ void bulk_wait_read() {
   asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void st_shared_u4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ uint4 ld_shared_u4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+               : "memory");
+  return v;
 }
 __device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
   asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
@@ -732,9 +745,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
       tc_fence_after_sync();
       const int64_t rh = static_cast<int64_t>(r) * kH + h;
       const int c_lo = kh * 128, c_hi = c_lo + 128;
+      // Each warp moves its 32 heads x 32 columns a chunk through its own
+      // slot of the (now idle) ring: lane = head writes its row, then each
+      // store instruction covers whole row segments (stores straight from
+      // the lanes would touch 32 rows 1 KB apart per instruction).
+      const uint32_t stage = sbase + kOffKV + (warp - (kGatherWarps + 1)) * kOutSlotBytes;
+      const int h_w = quarter * 32;  // first head of this warp
       if (P.splits == 1) {
         const float inv = l_fin > 0.f ? 1.f / l_fin : 0.f;
-        __nv_bfloat16* dst = P.out + rh * kDv + crank * kDvHalf;
+        // bf16 row segment: 64 bytes, slot rows 80 bytes apart
+        __nv_bfloat16* dst = P.out + (static_cast<int64_t>(r) * kH + h_w) * kDv + crank * kDvHalf;
 #pragma unroll 1
         for (int c = c_lo; c < c_hi; c += 32) {
           float o[32];
@@ -748,14 +768,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
             v.y = pack_bf16(o[q * 8 + 2] * inv, o[q * 8 + 3] * inv);
             v.z = pack_bf16(o[q * 8 + 4] * inv, o[q * 8 + 5] * inv);
             v.w = pack_bf16(o[q * 8 + 6] * inv, o[q * 8 + 7] * inv);
-            *reinterpret_cast<uint4*>(dst + c + q * 8) = v;
+            st_shared_u4(stage + lane * 80 + q * 16, v);
           }
+          __syncwarp();
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int row = q * 8 + (lane >> 2), part = lane & 3;
+            const uint4 v = ld_shared_u4(stage + row * 80 + part * 16);
+            *reinterpret_cast<uint4*>(dst + static_cast<int64_t>(row) * kDv + c + part * 8) = v;
+          }
+          __syncwarp();
         }
         if (P.lse != nullptr && crank == 0 && kh == 0)
           P.lse[rh] = l_fin > 0.f ? (m_fin + log2f(l_fin)) * 0.6931471805599453f : -INFINITY;
       } else {
         const int64_t it = (static_cast<int64_t>(r) * P.splits + sp) * 2 + crank;
-        float* dst = P.part_o + (it * kH + h) * kDvHalf;
+        // fp32 row segment: 128 bytes, slot rows 144 bytes apart
+        float* dst = P.part_o + (it * kH + h_w) * kDvHalf;
 #pragma unroll 1
         for (int c = c_lo; c < c_hi; c += 32) {
           float o[32];
@@ -764,7 +793,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
             for (int i = 0; i < 32; ++i) o[i] = 0.f;
 #pragma unroll
           for (int q = 0; q < 8; ++q)
-            *reinterpret_cast<float4*>(dst + c + q * 4) = make_float4(o[q * 4], o[q * 4 + 1], o[q * 4 + 2], o[q * 4 + 3]);
+            st_shared_u4(stage + lane * 144 + q * 16,
+                         make_uint4(__float_as_uint(o[q * 4]), __float_as_uint(o[q * 4 + 1]),
+                                    __float_as_uint(o[q * 4 + 2]), __float_as_uint(o[q * 4 + 3])));
+          __syncwarp();
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int row = q * 4 + (lane >> 3), part = lane & 7;
+            const uint4 v = ld_shared_u4(stage + row * 144 + part * 16);
+            *reinterpret_cast<uint4*>(dst + row * kDvHalf + c + part * 4) = v;
+          }
+          __syncwarp();
         }
         if (crank == 0 && kh == 0) {
           const int64_t ms = static_cast<int64_t>(r) * P.splits + sp;
