@@ -330,7 +330,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) topk_cluster_kernel(RowS
 #pragma unroll
       for (int u = 0; u < kParts; ++u) {
         const int i = i0 + u;
-        const int slot = (static_cast<int64_t>(i) * P.hist_per_cta) / P.hist_tpr == r ? 0 : 1;
+        // CTA i's run starts in this row: slot 0 (a comparison, no division)
+        const int64_t run0 = static_cast<int64_t>(i) * P.hist_per_cta;
+        const int slot = (run0 >= tile0 && run0 < tile0 + P.hist_tpr) ? 0 : 1;
         const uint4* src = reinterpret_cast<const uint4*>(P.hist_parts + (static_cast<int64_t>(i) * 2 + slot) * kBins1 +
                                                           (kBins1 - 4 - 4 * tid));
         x[u] = i <= i_hi ? __ldg(src) : make_uint4(0u, 0u, 0u, 0u);
@@ -611,6 +613,13 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) topk_cluster_kernel(RowS
     auto entry_index = [&](uint32_t en) -> int {
       return (chunk0 + static_cast<int>((en >> 13) & 0x3Fu)) * kChunk + static_cast<int>(en & kOffMask);
     };
+    // the order key of the row's key s (s < n), read again: staged, from the
+    // slice while the list (entries [0, own)) has not reached its word
+    auto key_again = [&](int s_idx) -> uint32_t {
+      if (kStaged && kChunk + (s_idx - chunk0 * kChunk) >= static_cast<int>(own))
+        return float_order_key(staged[s_idx]);
+      return float_order_key(__ldg(row + s_idx));
+    };
 
     // ---- 3. second digit: the row's counts in the leader
     if (C > 1) {
@@ -652,7 +661,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) topk_cluster_kernel(RowS
         } else if (d == D2) {
           const uint32_t j = atomicAdd(&sm.bcount, 1u);
           const int s_idx = entry_index(en);
-          const uint32_t kk = s_idx < n ? float_order_key(__ldg(row + s_idx)) : 0u;
+          const uint32_t kk = s_idx < n ? key_again(s_idx) : 0u;
           if (j < static_cast<uint32_t>(kBndCap)) {
             sm.bslot[j] = i;
             st_cluster(lbnd + 8u * j, kk);
@@ -747,7 +756,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) topk_cluster_kernel(RowS
         const uint32_t en = sm.ent[i];
         if (!(en & kSure) && ((en >> 19) & 0x7FFu) == D2) {
           const int s_idx = entry_index(en);
-          const uint32_t d3 = s_idx < n ? float_order_key(__ldg(row + s_idx)) & 0x3FFu : 0u;
+          const uint32_t d3 = s_idx < n ? key_again(s_idx) & 0x3FFu : 0u;
           atomicAdd(&my_h3[d3], 1u);
           sm.ent[i] = kHasD3 | (d3 << 19) | (en & kPosMask);
         }
