@@ -158,8 +158,8 @@ def _attn_extra_launches(wl, dsa, shape):
 # keyed by workload and by the SHA-256 of the indexer source the counters were taken on;
 # a changed kernel reports null.  Filled in from profiles/indexer_tc_decode128k.md.
 TRAFFIC = {
-    # B=8 capture (268,660,480 read + 4,446,208 written) scaled by 4 to B=32: traffic grows with the key tiles
-    "decode128k": ("c9aab5751d3cfe68", 4 * (268660480 + 4446208)),
+    # B=8 capture (268,662,784 read + 5,580,032 written) scaled by 4 to B=32: traffic grows with the key tiles
+    "decode128k": ("6548dd981d6a5269", 4 * (268662784 + 5580032)),
 }
 
 

@@ -174,7 +174,7 @@ struct HistPlan {
 HistPlan hist_plan(const dsa_shape_t* s, int dev, int B, int n_q) {
   HistPlan h;
   if (s->idx_dtype == DSA_F32 || !indexer_tc_supported(s->idx_heads, s->idx_dim)) return h;
-  h.on = indexer_hist_plan(B, n_q, s->s_max, device_sm_count(dev), &h.per_cta, &h.tpr);
+  h.on = indexer_hist_plan(B, n_q, s->s_max, device_sm_count(dev), s->idx_dtype == DSA_E4M3, &h.per_cta, &h.tpr);
   return h;
 }
 

@@ -48,10 +48,16 @@ struct IndexerArgs {
 constexpr int kMaxHistCtas = 256;
 // Bytes of the histogram handoff between the indexer and the top-k.
 constexpr size_t kHistPartsBytes = static_cast<size_t>(kMaxHistCtas) * 2 * 2048 * 4;
+// CTAs of the indexer's one-query (decode) schedule on num_sms SMs.  The
+// e4m3 instance is paced by its epilogue and takes every SM; the bf16 one is
+// bound by HBM, which 7/8 of the SMs already saturate (128K decode, 148 SMs:
+// 167 us at 128-132 CTAs against 177 us at 148, where the extra CTAs' loads
+// only queue).
+int indexer_decode_grid(int num_sms, bool fp8);
 // Whether the indexer's one-query schedule for (B, n_q, s_max) on num_sms SMs
 // can emit score histograms (every CTA's run spans at most two rows); if so,
 // the run length (tiles per CTA) and the key tiles per row.
-bool indexer_hist_plan(int B, int n_q, int s_max, int num_sms, int* per_cta, int* tpr);
+bool indexer_hist_plan(int B, int n_q, int s_max, int num_sms, bool fp8, int* per_cta, int* tpr);
 
 struct TopkArgs {
   int device;

@@ -509,7 +509,7 @@ dsa_status_t launch_indexer_tc(const IndexerArgs& a) {
   S.NC = (S.tpr + S.TPC - 1) / S.TPC;
   S.nunits = static_cast<int>(static_cast<int64_t>(a.B) * S.G * S.NC);
   const int64_t work = decode_like ? total_tiles : S.nunits;
-  const int grid = static_cast<int>(std::min<int64_t>(work, num_sms));
+  const int grid = static_cast<int>(std::min<int64_t>(work, decode_like ? indexer_decode_grid(num_sms, kFP8) : num_sms));
   S.per_cta = static_cast<int>((total_tiles + grid - 1) / grid);
   // multiplier coprime to nunits for the scrambled order
   int64_t mult = 40503;
@@ -537,13 +537,15 @@ dsa_status_t launch_indexer_tc(const IndexerArgs& a) {
 
 }  // namespace
 
-bool indexer_hist_plan(int B, int n_q, int s_max, int num_sms, int* per_cta, int* tpr) {
+int indexer_decode_grid(int num_sms, bool fp8) { return fp8 ? num_sms : std::max(1, num_sms * 7 / 8); }
+
+bool indexer_hist_plan(int B, int n_q, int s_max, int num_sms, bool fp8, int* per_cta, int* tpr) {
   // the decode schedule: one query per tile, each CTA a contiguous run of
   // key tiles; histograms only when a run spans at most two score rows
   if (n_q != 1 || B <= 0 || s_max <= 0 || num_sms <= 0 || num_sms > kMaxHistCtas) return false;
   const int64_t t = (s_max + kTileKeys - 1) / kTileKeys;
   const int64_t total = static_cast<int64_t>(B) * t;
-  const int64_t grid = std::min<int64_t>(total, num_sms);
+  const int64_t grid = std::min<int64_t>(total, indexer_decode_grid(num_sms, fp8));
   const int64_t pc = (total + grid - 1) / grid;
   if (pc > t || total > INT32_MAX / 2) return false;
   *per_cta = static_cast<int>(pc);
@@ -559,7 +561,7 @@ dsa_status_t indexer_tc(const IndexerArgs& a) {
   const bool hist = a.hist_parts != nullptr;
   if (hist) {
     int pc = 0, tp = 0;
-    if (!indexer_hist_plan(a.B, a.n_q, a.s_max, device_sm_count(a.device), &pc, &tp)) return DSA_ERR_UNSUPPORTED;
+    if (!indexer_hist_plan(a.B, a.n_q, a.s_max, device_sm_count(a.device), fp8, &pc, &tp)) return DSA_ERR_UNSUPPORTED;
   }
 #define DSA_IDX_CASE(HI, QGP)                                                                  \
   if (a.H == HI) {                                                                             \
