@@ -102,6 +102,10 @@ __device__ __forceinline__ void red_add_cluster(uint32_t addr, uint32_t v) {
 __device__ __forceinline__ void cluster_arrive() {
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
 }
+// Arrival that publishes nothing (this CTA's earlier writes are its own).
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
@@ -430,11 +434,22 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) topk_cluster_kernel(RowS
   }
   // (staged) every thread waits for the slice before its first key read
   bool have_slice = !kStaged;
+  bool lead_arrived = false;  // (clusters) the leader's arrival at the barrier after the zeroing
+  auto lead_arrive = [&]() {
+    if (C > 1 && lead && !lead_arrived) {
+      cluster_arrive();
+      lead_arrived = true;
+    }
+  };
+  // (every call comes after the sums below are zeroed) the leader publishes
+  // its zeroed sums once its own slice has landed: a release-ordered arrival
+  // with the bulk copy still in flight waited ~1 us for it
   auto wait_slice = [&]() {
     if (kStaged && !have_slice) {
       mbar_wait(smem_addr(&sm.kbar), 0, &sm.abort_flag, P.err);
       have_slice = true;
     }
+    lead_arrive();
   };
   auto chunk = [&](int ch) { cbase = (chunk0 + ch) * kChunk; };
   uint32_t key[kPer];
@@ -461,10 +476,13 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) topk_cluster_kernel(RowS
     sm.found = 0;
   }
   __syncthreads();
-  if (C > 1) cluster_arrive();
+  // (only the leader's sums are read across the cluster: the others' arrivals
+  // publish nothing; the leader arrives in wait_slice)
+  if (C > 1 && !lead) cluster_arrive_relaxed();
   bool waited = (C == 1);
   auto wait_zeroed = [&]() {  // before the first access to the leader's sums
     if (!waited) {
+      lead_arrive();
       cluster_wait();
       waited = true;
     }
