@@ -44,7 +44,8 @@ struct IdxCfg {
   static constexpr int kKTile = kTileKeys * kRowBytes;       // bytes of one key tile
   static constexpr int kQTile = N * kRowBytes;               // bytes of one query block
   static constexpr int kNumMma = kRowBytes / 32;             // each MMA consumes 32 bytes of K
-  static constexpr int kNumAcc = (N <= 64) ? 4 : (512 / N);  // TMEM accumulators
+  // one query a tile with 12 epilogue warps: three groups, two accumulators each
+  static constexpr int kNumAcc = (kQG == 1 && kEpiWarps == 12) ? 6 : (N <= 64) ? 4 : (512 / N);  // TMEM accumulators
   static constexpr int kTmemCols = (kNumAcc * N <= 256) ? 256 : 512;
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
   static constexpr int kEpiThreads = 32 * kEpiWarps;
@@ -63,11 +64,18 @@ struct IdxCfg {
   static_assert(N % 16 == 0 && N >= 16 && N <= 256, "MMA N");
   static_assert(kHI % 16 == 0, "heads per query");
   // 8 epilogue warps: two groups of four split the query block (kQG even),
-  // or take alternate key tiles (one query a tile)
-  static constexpr bool kAltTiles = (kEpiWarps == 8 && kQG == 1);
+  // or take alternate key tiles (one query a tile); 12 (one query a tile):
+  // three groups take every third key tile
+  static constexpr bool kAltTiles = (kEpiWarps >= 8 && kQG == 1);
+  static constexpr int kGroups = kAltTiles ? kEpiWarps / 4 : 1;
   static constexpr int kAccArrivals = kAltTiles ? 128 : kEpiThreads;
-  static_assert(kEpiWarps == 4 || (kEpiWarps == 8 && (kQG % 2 == 0 || kQG == 1)), "epilogue split");
-  static_assert(!kAltTiles || kNumAcc % 2 == 0, "alternate tiles need an even accumulator count");
+  // the query's head weights: in registers (one query a tile, up to 8
+  // epilogue warps), else in shared memory
+  static constexpr bool kWRegs = (kQG == 1 && kEpiWarps <= 8);
+  static_assert(kEpiWarps == 4 || (kEpiWarps == 8 && (kQG % 2 == 0 || kQG == 1)) || (kEpiWarps == 12 && kQG == 1),
+                "epilogue split");
+  static_assert(!kAltTiles || kNumAcc % kGroups == 0, "every group needs the same accumulators");
+  static_assert(kNumAcc * N <= 512, "tensor memory");
   static_assert(kKTile % 1024 == 0 && kQTile % 1024 == 0, "swizzle atom alignment");
 };
 
@@ -308,15 +316,15 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
     const int grp = e >> 2;  // warp group
     const int jbeg = (kEpiWarps == 8 && !C::kAltTiles) ? grp * (kQG / 2) : 0;
     const int jend = (kEpiWarps == 8 && !C::kAltTiles) ? jbeg + kQG / 2 : kQG;
-    // alternate tiles: group g takes the CTA's computed tiles n = g, g + 2, ...
-    // (accumulator n % kNumAcc, phase (n / kNumAcc) & 1)
-    constexpr int kStep = C::kAltTiles ? 2 : 1;
+    // alternate tiles: group g takes the CTA's computed tiles n = g, g + G, ...
+    // for G groups (accumulator n % kNumAcc, phase (n / kNumAcc) & 1)
+    constexpr int kStep = C::kAltTiles ? C::kGroups : 1;
     int ncomp = 0;  // tiles the CTA computed in earlier units
     const int tid_e = threadIdx.x - 64;
     int ab = C::kAltTiles ? grp : 0, wb = 0;
     uint32_t aph = 0;
     int last_bg = -1;
-    float wreg[kQG == 1 ? kHI : 1];
+    float wreg[C::kWRegs ? kHI : 1];
     UnitIter it = iter_begin(S, cta);
     // histogram slot of a score row: 0 for the first row of this CTA's run, 1 for the next
     const int first_bg = S.tpr > 0 ? it.i / S.tpr : 0;
@@ -324,7 +332,7 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
     while (iter_next<kQG>(S, it, cta, U, ctx_len, q_pos0)) {
       if (U.kt_end <= U.kt0) continue;
       uint32_t* hslot = hist_s + ((U.b * S.G + U.t0 / kQG) == first_bg ? 0 : kHistBins);
-      if (kQG == 1 && U.kt_comp > U.kt0) {
+      if (C::kWRegs && U.kt_comp > U.kt0) {
         // one query: its head weights live in registers
         const int bg = U.b * S.G + U.t0;
         if (bg != last_bg) {
@@ -368,7 +376,7 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
       auto load_ks = [&](int t) -> float {
         return (t < U.kt_comp && t * kTileKeys + row < U.L) ? __ldg(ks_row + t * kTileKeys) : 1.f;
       };
-      const int kt_first = C::kAltTiles ? U.kt0 + ((grp - ncomp) & 1) : U.kt0;
+      const int kt_first = C::kAltTiles ? U.kt0 + (((grp - ncomp) % kStep) + kStep) % kStep : U.kt0;
       if (C::kAltTiles && U.kt_comp > U.kt0) ncomp += U.kt_comp - U.kt0;
       // One key tile of the epilogue (FP8: its keys' scale ks); false if a
       // wait expired.
@@ -383,10 +391,13 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
           float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
 #pragma unroll
           for (int x = 0; x < 32; x += 2) {
-            acc0 = fmaf(wreg[x], fmaxf(v0[x], 0.f), acc0);
-            acc1 = fmaf(wreg[x + 1], fmaxf(v0[x + 1], 0.f), acc1);
-            acc2 = fmaf(wreg[32 + x], fmaxf(v1[x], 0.f), acc2);
-            acc3 = fmaf(wreg[33 + x], fmaxf(v1[x + 1], 0.f), acc3);
+            // (weights from shared memory: every lane reads the same word)
+            const float w0 = C::kWRegs ? wreg[x] : wd[x], w1 = C::kWRegs ? wreg[x + 1] : wd[x + 1];
+            const float w2 = C::kWRegs ? wreg[32 + x] : wd[32 + x], w3 = C::kWRegs ? wreg[33 + x] : wd[33 + x];
+            acc0 = fmaf(w0, fmaxf(v0[x], 0.f), acc0);
+            acc1 = fmaf(w1, fmaxf(v0[x + 1], 0.f), acc1);
+            acc2 = fmaf(w2, fmaxf(v1[x], 0.f), acc2);
+            acc3 = fmaf(w3, fmaxf(v1[x + 1], 0.f), acc3);
           }
           if (s < U.L) {
             const int p = U.p0 + U.t0;
@@ -565,9 +576,9 @@ dsa_status_t indexer_tc(const IndexerArgs& a) {
   }
 #define DSA_IDX_CASE(HI, QGP)                                                                  \
   if (a.H == HI) {                                                                             \
-    if (one && hist) return fp8 ? launch_indexer_tc<true, 1, HI, 8, 12, 2, true>(a)             \
+    if (one && hist) return fp8 ? launch_indexer_tc<true, 1, HI, ((HI) == 64 ? 12 : 8), 12, 2, true>(a) \
                                 : launch_indexer_tc<false, 1, HI, 4, 5, 2, true>(a);           \
-    if (one) return fp8 ? launch_indexer_tc<true, 1, HI, 8, 12, 2, false>(a)                    \
+    if (one) return fp8 ? launch_indexer_tc<true, 1, HI, ((HI) == 64 ? 12 : 8), 12, 2, false>(a)        \
                         : launch_indexer_tc<false, 1, HI, 4, 5, 2, false>(a);                  \
     return fp8 ? launch_indexer_tc<true, QGP, HI, ((QGP) % 2 == 0 ? 8 : 4), 6, 1, false>(a)    \
                : launch_indexer_tc<false, QGP, HI, ((QGP) % 2 == 0 ? 8 : 4), 4, 1, false>(a);  \
