@@ -313,7 +313,8 @@ __device__ __forceinline__ void gather_rope(uint32_t dst0, const char* kv_b, int
 constexpr uint32_t kLayoutSW64 = 4;
 
 __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) {
-  pdl_wait();
+  // (the set-up below reads no global memory: it runs before the wait for
+  // the previous kernel, under its tail)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
@@ -350,7 +351,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
   const int sp = item % P.splits;
   const int r = item / P.splits;
   const int b = r / P.n_q;
-  const int L = min(max(__ldg(P.ctx_len + b), 0), P.s_max);
   const int row0 = sp * P.rows_per_split;
   const int nrows = max(0, min(P.rows_per_split, P.k - row0));
   const int T = (nrows + kRows - 1) / kRows;
@@ -392,6 +392,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_mla_tc_kernel(AttnParams P) 
   tc_fence_after_sync();
   cluster_sync_all();  // both CTAs' barriers exist (and are armed) before any remote arrival
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+  const int L = min(max(__ldg(P.ctx_len + b), 0), P.s_max);
 
   if (warp == kCommWarp) {
     // --------------------------------------- copies and cross-CTA signals --
