@@ -411,6 +411,14 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) topk_cluster_kernel(RowS
     return m;
   };
   auto load_slice = [&](uint32_t* key) -> uint32_t { return load_at(cbase, key); };
+  // (walking) pull chunk ch's lines into L2 ahead of its register loads, so
+  // that each chunk costs an L2 round trip instead of an HBM one
+  auto prefetch_chunk = [&](int ch) {
+    if (!kStaged && ch < nch && tid < kChunk / 32) {
+      const int p = (chunk0 + ch) * kChunk + tid * 32;
+      if (p < n) asm volatile("prefetch.global.L2 [%0];" ::"l"(row + p));
+    }
+  };
   if constexpr (kStaged) {
     // the slice [chunk0 kChunk, + kCtaChunks kChunk) clipped to the row (to a
     // multiple of 4 keys: the row's storage is), in one bulk copy
@@ -508,7 +516,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) topk_cluster_kernel(RowS
   // ---- 1. first digit
   if (P.hist_parts == nullptr) {
     wait_slice();
+    prefetch_chunk(1);
     for (int ch = 0; ch < nch; ++ch) {
+      prefetch_chunk(ch + 2);
       chunk(ch);
       vm = load_slice(key);
 #pragma unroll
@@ -558,7 +568,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) topk_cluster_kernel(RowS
     const uint32_t pos_min = K0 >= 0x80000000u ? K0 - 0x80000000u : 0u;
     const uint32_t neg_max = K0 == 0x80000000u ? 0x80000000u : ~K0;  // (K0 > 2^31: ~K0 < 2^31, no negative b)
     wait_slice();
+    prefetch_chunk(1);
     for (int ch = 0; ch < nch; ++ch) {
+      prefetch_chunk(ch + 2);
       chunk(ch);
       uint32_t f = 0;
       if constexpr (kStaged) {
@@ -892,7 +904,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) topk_cluster_kernel(RowS
   // then the kept keys written chunk by chunk at running offsets
   for (int i = tid; i < kBins1; i += kThreads) sm.hist[i] = 0;
   __syncthreads();
+  prefetch_chunk(1);
   for (int ch = 0; ch < nch; ++ch) {
+    prefetch_chunk(ch + 2);
     chunk(ch);
     vm = load_slice(key);
 #pragma unroll
@@ -915,7 +929,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) topk_cluster_kernel(RowS
   const uint32_t rem2 = rem1 - sm.res[4];
   for (int i = tid; i < kBins1; i += kThreads) sm.hist[i] = 0;
   __syncthreads();
+  prefetch_chunk(1);
   for (int ch = 0; ch < nch; ++ch) {
+    prefetch_chunk(ch + 2);
     chunk(ch);
     vm = load_slice(key);
 #pragma unroll
@@ -937,7 +953,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) topk_cluster_kernel(RowS
   const uint32_t take_eq = rem2 - sm.res[7];
   pdl_trigger();
   uint32_t gt_off = 0, eq_off = 0;
+  prefetch_chunk(1);
   for (int ch = 0; ch < nch; ++ch) {
+    prefetch_chunk(ch + 2);
     chunk(ch);
     vm = load_slice(key);
     uint32_t fg = 0, fe = 0;
