@@ -72,7 +72,8 @@ struct IdxCfg {
   // the query's head weights: in registers (one query a tile, up to 8
   // epilogue warps), else in shared memory
   static constexpr bool kWRegs = (kQG == 1 && kEpiWarps <= 8);
-  static_assert(kEpiWarps == 4 || (kEpiWarps == 8 && (kQG % 2 == 0 || kQG == 1)) || (kEpiWarps == 12 && kQG == 1),
+  static_assert(kEpiWarps == 4 || (kEpiWarps == 8 && (kQG % 2 == 0 || kQG == 1)) || (kEpiWarps == 12 && kQG == 1) ||
+                    (kEpiWarps == 16 && kQG % 4 == 0),
                 "epilogue split");
   static_assert(!kAltTiles || kNumAcc % kGroups == 0, "every group needs the same accumulators");
   static_assert(kNumAcc * N <= 512, "tensor memory");
@@ -314,8 +315,10 @@ __global__ void __launch_bounds__(IdxCfg<kFP8, kQG, kHI, kEpiWarps, kStages, kQB
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;  // key within the tile == TMEM lane
     const int grp = e >> 2;  // warp group
-    const int jbeg = (kEpiWarps == 8 && !C::kAltTiles) ? grp * (kQG / 2) : 0;
-    const int jend = (kEpiWarps == 8 && !C::kAltTiles) ? jbeg + kQG / 2 : kQG;
+    // (a query block split over the groups: kQG / (kEpiWarps / 4) queries each)
+    constexpr int kQPer = (kEpiWarps >= 8 && !C::kAltTiles) ? kQG / (kEpiWarps / 4) : kQG;
+    const int jbeg = (kEpiWarps >= 8 && !C::kAltTiles) ? grp * kQPer : 0;
+    const int jend = jbeg + kQPer;
     // alternate tiles: group g takes the CTA's computed tiles n = g, g + G, ...
     // for G groups (accumulator n % kNumAcc, phase (n / kNumAcc) & 1)
     constexpr int kStep = C::kAltTiles ? C::kGroups : 1;
@@ -581,7 +584,7 @@ dsa_status_t indexer_tc(const IndexerArgs& a) {
     if (one) return fp8 ? launch_indexer_tc<true, 1, HI, ((HI) == 64 ? 12 : 8), 12, 2, false>(a)        \
                         : launch_indexer_tc<false, 1, HI, 4, 5, 2, false>(a);                  \
     return fp8 ? launch_indexer_tc<true, QGP, HI, ((QGP) % 2 == 0 ? 8 : 4), 6, 1, false>(a)    \
-               : launch_indexer_tc<false, QGP, HI, ((QGP) % 2 == 0 ? 8 : 4), 4, 1, false>(a);  \
+               : launch_indexer_tc<false, QGP, HI, ((QGP) % 4 == 0 ? 16 : (QGP) % 2 == 0 ? 8 : 4), 4, 1, false>(a);  \
   }
   DSA_IDX_CASE(64, 4)
   DSA_IDX_CASE(32, 8)
