@@ -63,9 +63,10 @@ struct IdxCfg {
   static_assert(!kHist || kQG == 1, "score histograms are built in the one-query (decode) schedule");
   static_assert(N % 16 == 0 && N >= 16 && N <= 256, "MMA N");
   static_assert(kHI % 16 == 0, "heads per query");
-  // 8 epilogue warps: two groups of four split the query block (kQG even),
-  // or take alternate key tiles (one query a tile); 12 (one query a tile):
-  // three groups take every third key tile
+  // Epilogue warps in groups of four (one warp per TMEM lane quarter): with
+  // one query a tile the groups take turns by key tile (8 warps: alternate
+  // tiles; 12: every third), else they split the query block (8: two groups
+  // of kQG / 2 queries; 16: four groups of kQG / 4)
   static constexpr bool kAltTiles = (kEpiWarps >= 8 && kQG == 1);
   static constexpr int kGroups = kAltTiles ? kEpiWarps / 4 : 1;
   static constexpr int kAccArrivals = kAltTiles ? 128 : kEpiThreads;
