@@ -158,8 +158,8 @@ def _attn_extra_launches(wl, dsa, shape):
 # keyed by workload and by the SHA-256 of the indexer source the counters were taken on;
 # a changed kernel reports null.  Filled in from profiles/indexer_tc_decode128k.md.
 TRAFFIC = {
-    # B=8 capture (268,660,992 read + 4,826,368 written) scaled by 4 to B=32: traffic grows with the key tiles
-    "decode128k": ("192c3912d83b6872", 4 * (268660992 + 4826368)),
+    # B=8 capture (268,660,736 read + 4,674,816 written) scaled by 4 to B=32: traffic grows with the key tiles
+    "decode128k": ("3092c7447fe712d5", 4 * (268660736 + 4674816)),
 }
 
 
