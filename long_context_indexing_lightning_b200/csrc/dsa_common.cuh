@@ -163,7 +163,7 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 
 // The same load with an L2 eviction-priority hint (a policy from
 // l2_evict_first()): for data read once, so that it does not push out what a
-// later kernel reads (this GPU's own memory; no multicast).
+// later kernel reads (this GPU's own memory, one destination CTA).
 __device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
                                                  uint64_t policy) {
   asm volatile(
